@@ -1,0 +1,11 @@
+"""Grouped-query scaled-dot-product attention for NVIDIA B200 (sm_100a).
+
+The computation lives in the C-ABI library ``libgqa.so`` (declared in
+``include/gqa.h``): a tcgen05/TMEM/TMA prefill kernel, a split-KV decode
+kernel with a log-sum-exp combine, an fp32 path and a head-folding kernel.
+This package is its Python binding; PyTorch is used for device memory and
+streams only.  The library is loaded on first use and there is no CPU
+fallback: a missing or unloadable library raises.
+"""
+
+from .api import attn, attn_f32, decode, decode_workspace_size, device_status, fold_kv  # noqa: F401

@@ -1,0 +1,131 @@
+"""Tensor-level calls on top of the C ABI.
+
+PyTorch supplies device memory, shapes and the current stream; every step of
+the computation runs in libgqa.so.  Non-OK statuses become exceptions:
+``ValueError`` for invalid arguments and workspace problems,
+``NotImplementedError`` for unsupported shapes, ``RuntimeError`` otherwise.
+"""
+
+import math
+
+import torch
+
+from . import _binding as _b
+
+_EXC = {
+    _b.GQA_ERR_INVALID_ARG: ValueError,
+    _b.GQA_ERR_WORKSPACE: ValueError,
+    _b.GQA_ERR_UNSUPPORTED: NotImplementedError,
+}
+
+
+def _check(rc, what):
+    if rc != _b.GQA_OK:
+        raise _EXC.get(rc, RuntimeError)(f"{what}: {_b.gqa_last_error()} (status {rc})")
+
+
+def _stream(t):
+    return torch.cuda.current_stream(t.device).cuda_stream
+
+
+def _need(t, name, dtype, ndim):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if t.dim() != ndim:
+        raise ValueError(f"{name} must have {ndim} dims, got shape {tuple(t.shape)}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def _shapes(q, k, v):
+    B, Tq, Hq, d = q.shape
+    Bk, Tkv, Hkv, dk = k.shape
+    if Bk != B or dk != d or tuple(v.shape) != tuple(k.shape):
+        raise ValueError(f"shape mismatch: q {tuple(q.shape)}, k {tuple(k.shape)}, v {tuple(v.shape)}")
+    return B, Tq, Tkv, Hq, Hkv, d
+
+
+def attn(q, k, v, causal=True, scale=None, out=None, return_lse=False):
+    """Grouped-query attention forward, bf16.
+
+    q [B, Tq, Hq, d], k/v [B, Tkv, Hkv, d] (bf16, contiguous, on one GPU);
+    query head h reads K/V head h // (Hq // Hkv).  Returns o [B, Tq, Hq, d]
+    (and lse [B, Hq, Tq] fp32 when ``return_lse``).
+    """
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _need(t, n, torch.bfloat16, 4)
+    B, Tq, Tkv, Hq, Hkv, d = _shapes(q, k, v)
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    o = torch.empty_like(q) if out is None else out
+    _need(o, "out", torch.bfloat16, 4)
+    lse = torch.empty((B, Hq, Tq), dtype=torch.float32, device=q.device) if return_lse else None
+    rc = _b.gqa_attn_fwd_lse(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
+                             lse.data_ptr() if lse is not None else None,
+                             B, Tq, Tkv, Hq, Hkv, d, int(bool(causal)), scale, _stream(q))
+    _check(rc, "gqa_attn_fwd")
+    return (o, lse) if return_lse else o
+
+
+def attn_f32(q, k, v, causal=True, scale=None, return_lse=False):
+    """The same operation in fp32 (FP32 pipe); q/k/v fp32 in the same layouts."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _need(t, n, torch.float32, 4)
+    B, Tq, Tkv, Hq, Hkv, d = _shapes(q, k, v)
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    o = torch.empty_like(q)
+    lse = torch.empty((B, Hq, Tq), dtype=torch.float32, device=q.device) if return_lse else None
+    rc = _b.gqa_attn_fwd_f32(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
+                             lse.data_ptr() if lse is not None else None,
+                             B, Tq, Tkv, Hq, Hkv, d, int(bool(causal)), scale, _stream(q))
+    _check(rc, "gqa_attn_fwd_f32")
+    return (o, lse) if return_lse else o
+
+
+def decode_workspace_size(B, Hq, Hkv, d, Lmax):
+    return int(_b.gqa_decode_workspace_size(B, Hq, Hkv, d, Lmax))
+
+
+def decode(q, k_cache, v_cache, seqlens, scale=None, workspace=None, out=None):
+    """One query token per sequence against a bf16 KV cache.
+
+    q [B, Hq, d], caches [B, Lmax, Hkv, d], seqlens int32 [B] on the device.
+    ``workspace``: a uint8 CUDA tensor of at least decode_workspace_size(...)
+    bytes (allocated here when None).
+    """
+    _need(q, "q", torch.bfloat16, 3)
+    _need(k_cache, "k_cache", torch.bfloat16, 4)
+    _need(v_cache, "v_cache", torch.bfloat16, 4)
+    _need(seqlens, "seqlens", torch.int32, 1)
+    B, Hq, d = q.shape
+    Bc, Lmax, Hkv, dc = k_cache.shape
+    if Bc != B or dc != d or tuple(v_cache.shape) != tuple(k_cache.shape) or seqlens.shape[0] != B:
+        raise ValueError("decode shape mismatch")
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    need = decode_workspace_size(B, Hq, Hkv, d, Lmax)
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
+    o = torch.empty_like(q) if out is None else out
+    rc = _b.gqa_decode(q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(), seqlens.data_ptr(),
+                       o.data_ptr(), B, Hq, Hkv, d, Lmax, scale, workspace.data_ptr(),
+                       workspace.numel(), _stream(q))
+    _check(rc, "gqa_decode")
+    return o
+
+
+def fold_kv(kv, g):
+    """Mean-pool the heads of a bf16 [B, T, H, d] K or V tensor into g contiguous groups."""
+    _need(kv, "kv", torch.bfloat16, 4)
+    B, T, H, d = kv.shape
+    out = torch.empty((B, T, g, d), dtype=kv.dtype, device=kv.device)
+    rc = _b.gqa_fold_kv(kv.data_ptr(), out.data_ptr(), B, T, H, g, d, _stream(kv))
+    _check(rc, "gqa_fold_kv")
+    return out
+
+
+def device_status(reset=True):
+    """Synchronise, then raise if a kernel recorded an error (e.g. a wait timeout)."""
+    _check(_b.gqa_device_status(int(bool(reset))), "gqa_device_status")

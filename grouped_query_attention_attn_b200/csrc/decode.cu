@@ -1,0 +1,401 @@
+// decode.cu -- split-KV grouped-query decode (one query token per sequence)
+// and the log-sum-exp combine of the splits.
+//
+// Work unit: one CTA per (split, KV head, sequence).  A split is `chunk`
+// consecutive cache rows; the CTA streams its K and V rows from HBM exactly
+// once through a TMA ring in shared memory and uses each row for all
+// G = Hq / Hkv query heads of the group, which sit as the M rows of warp-level
+// bf16 tensor-core tiles (m16n8k16; G <= 16 per tile, padding rows are zero).
+//   - warp 4 (one thread) issues the TMA copies: per stage 64 keys of K and V
+//     (four 64-column panels with 128-byte swizzle for d = 128);
+//   - warps 0-3 each take 16 keys of every stage: S = Q K^T, the running-max
+//     softmax of the course's step 1 (mask of keys past the sequence end,
+//     max subtracted, exp2 with scale * log2 e folded in), then O += P V;
+//     row max / sum reductions are warp shuffles inside each quad of lanes;
+//   - at the end the four warps' (m, l, O) are merged through shared memory
+//     and the split's normalised O and natural-log lse go to the workspace.
+// The combine kernel then merges the splits of each (sequence, query head):
+//   O = sum_s e^(lse_s - M) O_s / sum_s e^(lse_s - M),  M = max_s lse_s.
+#include <cuda_bf16.h>
+
+#include "device.cuh"
+#include "internal.h"
+
+namespace gqa {
+
+constexpr int kDecBK = 64;                         // keys per pipeline stage
+constexpr int kDecWarps = 4;                       // consumer warps, 16 keys each per stage
+constexpr int kDecThreads = (kDecWarps + 1) * 32;  // + one producer warp
+constexpr int kDecStages = 3;
+constexpr int kDecChunk = 512;                     // keys per split
+
+template <int D>
+struct DecLayout {
+    static constexpr int kPanels = D / 64;                 // 64 bf16 = one 128-byte row
+    static constexpr int kPanelBytes = kDecBK * 128;
+    static constexpr int kTileBytes = kPanels * kPanelBytes;
+    static constexpr int kStageBytes = 2 * kTileBytes;     // K tile then V tile
+    static constexpr int kRingBytes = kDecStages * kStageBytes;
+    static constexpr int kSmemBytes = kRingBytes + 1024;   // + alignment slack
+};
+
+__device__ __forceinline__ uint32_t ld_b32(const __nv_bfloat16 *p) {
+    return *reinterpret_cast<const uint32_t *>(p);
+}
+
+// Byte offset of 16-byte chunk `cg` (0 .. D/8-1) of tile row `row` in a tile
+// made of 64-column panels written by TMA with 128-byte swizzle.
+template <int D>
+__device__ __forceinline__ uint32_t swz_off(int row, int cg) {
+    return (cg >> 3) * DecLayout<D>::kPanelBytes + row * 128 + (((cg & 7) ^ (row & 7)) << 4);
+}
+
+template <int D, int MB>
+__global__ void __launch_bounds__(kDecThreads)
+decode_split_kernel(const __grid_constant__ CUtensorMap tm_k,
+                    const __grid_constant__ CUtensorMap tm_v,
+                    const __nv_bfloat16 *__restrict__ q, const int32_t *__restrict__ seqlens,
+                    float *__restrict__ part_o, float *__restrict__ part_lse, int B, int Hq,
+                    int Hkv, int Lmax, int chunk, float scale_log2, int *status) {
+    using Lay = DecLayout<D>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    __shared__ uint64_t full_bar[kDecStages], empty_bar[kDecStages];
+    __shared__ int abort_flag;
+
+    const int split = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z;
+    int L = seqlens[b];
+    if (L > Lmax || L < 0) {
+        if (threadIdx.x == 0 && split == 0 && kvh == 0) record_status(status, GQA_ERR_INVALID_ARG);
+        L = L < 0 ? 0 : Lmax;
+    }
+    const int start = split * chunk;
+    if (start >= L) return;                         // whole block: nothing in this split
+    const int end = min(start + chunk, L);
+    const int n_stages = (end - start + kDecBK - 1) / kDecBK;
+    const int G = Hq / Hkv;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kDecStages; ++s) {
+            mbar_init(&full_bar[s], 1);
+            mbar_init(&empty_bar[s], kDecWarps);
+        }
+        abort_flag = 0;
+        fence_mbar_init();
+    }
+    __syncthreads();
+
+    if (warp == kDecWarps) {                        // ---- TMA producer ----
+        if (lane == 0) {
+            tma_prefetch_desc(&tm_k);
+            tma_prefetch_desc(&tm_v);
+            for (int t = 0; t < n_stages; ++t) {
+                const int st = t % kDecStages;
+                const uint32_t ph = (t / kDecStages) & 1;
+                if (!mbar_wait(&empty_bar[st], ph ^ 1, &abort_flag, status)) break;
+                uint8_t *kt = smem + st * Lay::kStageBytes;
+                uint8_t *vt = kt + Lay::kTileBytes;
+                mbar_expect_tx(&full_bar[st], Lay::kStageBytes);
+                const int j0 = start + t * kDecBK;
+#pragma unroll
+                for (int p = 0; p < Lay::kPanels; ++p) {
+                    tma_load_4d(kt + p * Lay::kPanelBytes, &tm_k, &full_bar[st], p * 64, kvh, j0, b);
+                    tma_load_4d(vt + p * Lay::kPanelBytes, &tm_v, &full_bar[st], p * 64, kvh, j0, b);
+                }
+            }
+        }
+        return;                                     // consumers sync with named barrier 1 only
+    }
+
+    // ---- consumers: query fragments of the G heads of this group ----
+    const int gq = lane >> 2, tq = lane & 3;        // quad row, lane in quad
+    const __nv_bfloat16 *qg = q + (static_cast<size_t>(b) * Hq + static_cast<size_t>(kvh) * G) * D;
+    uint32_t qa[MB][D / 16][4];
+#pragma unroll
+    for (int mb = 0; mb < MB; ++mb) {
+        const int r0 = mb * 16 + gq, r1 = r0 + 8;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+            const int c0 = kk * 16 + 2 * tq, c1 = c0 + 8;
+            qa[mb][kk][0] = r0 < G ? ld_b32(qg + r0 * D + c0) : 0u;
+            qa[mb][kk][1] = r1 < G ? ld_b32(qg + r1 * D + c0) : 0u;
+            qa[mb][kk][2] = r0 < G ? ld_b32(qg + r0 * D + c1) : 0u;
+            qa[mb][kk][3] = r1 < G ? ld_b32(qg + r1 * D + c1) : 0u;
+        }
+    }
+    float oacc[MB][D / 8][4];
+    float m_run[MB][2], l_run[MB][2];
+#pragma unroll
+    for (int mb = 0; mb < MB; ++mb) {
+#pragma unroll
+        for (int nd = 0; nd < D / 8; ++nd)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) oacc[mb][nd][e] = 0.0f;
+        m_run[mb][0] = m_run[mb][1] = -INFINITY;
+        l_run[mb][0] = l_run[mb][1] = 0.0f;
+    }
+
+    for (int t = 0; t < n_stages; ++t) {
+        const int st = t % kDecStages;
+        const uint32_t ph = (t / kDecStages) & 1;
+        // warp-uniform outcome: ldmatrix and mma.sync below are warp-collective
+        if (!__all_sync(0xffffffffu, mbar_wait(&full_bar[st], ph, &abort_flag, status))) break;
+        uint8_t *kt = smem + st * Lay::kStageBytes;
+        uint8_t *vt = kt + Lay::kTileBytes;
+        const int key0 = start + t * kDecBK + warp * 16;  // first key of this warp's slice
+        const int n_valid = end - key0;                   // keys of the slice inside the split
+        const bool partial = n_valid > 0 && n_valid < 16;
+        if (partial) {
+            // Rows past the split end may be another split's keys or the
+            // caller's padding (anything, NaN included): zero their V rows so
+            // P = 0 there multiplies exact zeros.
+            for (int idx = lane; idx < (16 - n_valid) * (D / 8); idx += 32) {
+                const int r = warp * 16 + n_valid + idx / (D / 8);
+                *reinterpret_cast<uint4 *>(vt + swz_off<D>(r, idx % (D / 8))) =
+                    make_uint4(0u, 0u, 0u, 0u);
+            }
+            __syncwarp();
+        }
+        if (n_valid > 0) {
+            float sacc[MB][2][4];
+#pragma unroll
+            for (int mb = 0; mb < MB; ++mb)
+#pragma unroll
+                for (int nb = 0; nb < 2; ++nb)
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) sacc[mb][nb][e] = 0.0f;
+            const uint32_t kbase = smem_u32(kt);
+            const int krow = warp * 16 + (lane & 7) + ((lane >> 4) << 3);
+#pragma unroll
+            for (int kk = 0; kk < D / 16; ++kk) {
+                uint32_t kb[4];
+                ldsm_x4(kb, kbase + swz_off<D>(krow, 2 * kk + ((lane >> 3) & 1)));
+#pragma unroll
+                for (int mb = 0; mb < MB; ++mb) {
+                    mma_16816(sacc[mb][0], qa[mb][kk], kb[0], kb[1]);
+                    mma_16816(sacc[mb][1], qa[mb][kk], kb[2], kb[3]);
+                }
+            }
+            uint32_t pa[MB][4];
+#pragma unroll
+            for (int mb = 0; mb < MB; ++mb) {
+                float s[2][4], mx[2] = {-INFINITY, -INFINITY};
+#pragma unroll
+                for (int nb = 0; nb < 2; ++nb)
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const int kl = nb * 8 + 2 * tq + (e & 1);
+                        s[nb][e] = kl < n_valid ? sacc[mb][nb][e] * scale_log2 : -INFINITY;
+                        mx[e >> 1] = fmaxf(mx[e >> 1], s[nb][e]);
+                    }
+                float alpha[2], m_use[2];
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    mx[h] = fmaxf(mx[h], __shfl_xor_sync(0xffffffffu, mx[h], 1));
+                    mx[h] = fmaxf(mx[h], __shfl_xor_sync(0xffffffffu, mx[h], 2));
+                    const float m_new = fmaxf(m_run[mb][h], mx[h]);
+                    m_use[h] = (m_new == -INFINITY) ? 0.0f : m_new;
+                    alpha[h] = fast_exp2(m_run[mb][h] - m_use[h]);
+                    m_run[mb][h] = m_new;
+                }
+                float psum[2] = {0.0f, 0.0f};
+#pragma unroll
+                for (int nb = 0; nb < 2; ++nb)
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        s[nb][e] = fast_exp2(s[nb][e] - m_use[e >> 1]);
+                        psum[e >> 1] += s[nb][e];
+                    }
+#pragma unroll
+                for (int h = 0; h < 2; ++h) l_run[mb][h] = l_run[mb][h] * alpha[h] + psum[h];
+#pragma unroll
+                for (int nd = 0; nd < D / 8; ++nd) {
+                    oacc[mb][nd][0] *= alpha[0];
+                    oacc[mb][nd][1] *= alpha[0];
+                    oacc[mb][nd][2] *= alpha[1];
+                    oacc[mb][nd][3] *= alpha[1];
+                }
+                pa[mb][0] = pack_bf16x2(s[0][0], s[0][1]);
+                pa[mb][1] = pack_bf16x2(s[0][2], s[0][3]);
+                pa[mb][2] = pack_bf16x2(s[1][0], s[1][1]);
+                pa[mb][3] = pack_bf16x2(s[1][2], s[1][3]);
+            }
+            const uint32_t vbase = smem_u32(vt);
+            const int vrow = warp * 16 + (lane & 7) + (((lane >> 3) & 1) << 3);
+#pragma unroll
+            for (int dd = 0; dd < D / 16; ++dd) {
+                uint32_t vb[4];
+                ldsm_x4_trans(vb, vbase + swz_off<D>(vrow, 2 * dd + (lane >> 4)));
+#pragma unroll
+                for (int mb = 0; mb < MB; ++mb) {
+                    mma_16816(oacc[mb][2 * dd], pa[mb], vb[0], vb[1]);
+                    mma_16816(oacc[mb][2 * dd + 1], pa[mb], vb[2], vb[3]);
+                }
+            }
+        }
+        if (partial) fence_proxy_async_smem();      // zeroing before the ring slot is refilled
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty_bar[st]);
+    }
+
+    // ---- merge the four warps' partial softmax states ----
+#pragma unroll
+    for (int mb = 0; mb < MB; ++mb)
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            l_run[mb][h] += __shfl_xor_sync(0xffffffffu, l_run[mb][h], 1);
+            l_run[mb][h] += __shfl_xor_sync(0xffffffffu, l_run[mb][h], 2);
+        }
+    named_barrier_sync(1, kDecWarps * 32);          // every stage consumed: reuse the ring
+    constexpr int kRows = MB * 16;
+    float *s_o = reinterpret_cast<float *>(smem);             // [warp][row][D]
+    float *s_m = s_o + kDecWarps * kRows * D;                 // [warp][row]
+    float *s_l = s_m + kDecWarps * kRows;                     // [warp][row]
+#pragma unroll
+    for (int mb = 0; mb < MB; ++mb) {
+#pragma unroll
+        for (int nd = 0; nd < D / 8; ++nd)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const int r = mb * 16 + gq + ((e >> 1) << 3);
+                const int c = nd * 8 + 2 * tq + (e & 1);
+                s_o[(warp * kRows + r) * D + c] = oacc[mb][nd][e];
+            }
+        if (tq == 0) {
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const int r = mb * 16 + gq + h * 8;
+                s_m[warp * kRows + r] = m_run[mb][h];
+                s_l[warp * kRows + r] = l_run[mb][h];
+            }
+        }
+    }
+    named_barrier_sync(1, kDecWarps * 32);
+    const size_t row0 = (static_cast<size_t>(split) * B + b) * Hq + static_cast<size_t>(kvh) * G;
+    for (int idx = threadIdx.x; idx < G * D; idx += kDecWarps * 32) {
+        const int r = idx / D, c = idx % D;
+        float M = -INFINITY;
+#pragma unroll
+        for (int w = 0; w < kDecWarps; ++w) M = fmaxf(M, s_m[w * kRows + r]);
+        float wsum = 0.0f, acc = 0.0f;
+#pragma unroll
+        for (int w = 0; w < kDecWarps; ++w) {
+            const float f = fast_exp2(s_m[w * kRows + r] - M);   // 0 for a warp with no key
+            wsum += f * s_l[w * kRows + r];
+            acc += f * s_o[(w * kRows + r) * D + c];
+        }
+        part_o[(row0 + r) * D + c] = acc / wsum;
+        if (c == 0) part_lse[row0 + r] = (M + __log2f(wsum)) * 0.69314718055994531f;
+    }
+}
+
+template <int D>
+__global__ void __launch_bounds__(128)
+decode_combine_kernel(const float *__restrict__ part_o, const float *__restrict__ part_lse,
+                      const int32_t *__restrict__ seqlens, __nv_bfloat16 *__restrict__ o, int B,
+                      int Hq, int Lmax, int chunk) {
+    constexpr int kPer = D / 32;
+    const int row = blockIdx.x * 4 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
+    if (row >= B * Hq) return;
+    const int b = row / Hq;
+    int L = seqlens[b];
+    L = L < 0 ? 0 : (L > Lmax ? Lmax : L);
+    const int n = (L + chunk - 1) / chunk;
+    const size_t plane = static_cast<size_t>(B) * Hq;
+    float acc[kPer];
+#pragma unroll
+    for (int e = 0; e < kPer; ++e) acc[e] = 0.0f;
+    if (n > 0) {
+        float M = -INFINITY;
+        for (int s = 0; s < n; ++s) M = fmaxf(M, part_lse[s * plane + row]);
+        float wsum = 0.0f;
+        for (int s = 0; s < n; ++s) {
+            const float w = __expf(part_lse[s * plane + row] - M);
+            wsum += w;
+            const float *src = part_o + (s * plane + row) * D + lane * kPer;
+#pragma unroll
+            for (int e = 0; e < kPer; ++e) acc[e] += w * src[e];
+        }
+        const float inv = 1.0f / wsum;
+#pragma unroll
+        for (int e = 0; e < kPer; ++e) acc[e] *= inv;
+    }
+    __nv_bfloat16 *dst = o + static_cast<size_t>(row) * D + lane * kPer;
+#pragma unroll
+    for (int e = 0; e < kPer; e += 2)
+        *reinterpret_cast<__nv_bfloat162 *>(dst + e) = __floats2bfloat162_rn(acc[e], acc[e + 1]);
+}
+
+int decode_chunk(int /*B*/, int /*Hkv*/, int /*Lmax*/) { return kDecChunk; }
+
+static size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+size_t decode_workspace_bytes(int B, int Hq, int Hkv, int d, int Lmax) {
+    const int chunk = decode_chunk(B, Hkv, Lmax);
+    const size_t splits = (static_cast<size_t>(Lmax) + chunk - 1) / chunk;
+    const size_t rows = splits * B * Hq;
+    return align256(rows * d * sizeof(float)) + align256(rows * sizeof(float));
+}
+
+template <int D, int MB>
+static int launch_split(const CUtensorMap &tk, const CUtensorMap &tv, const void *q,
+                        const int32_t *seqlens, float *part_o, float *part_lse, int B, int Hq,
+                        int Hkv, int Lmax, int chunk, float scale_log2, int *status,
+                        cudaStream_t stream) {
+    auto kern = decode_split_kernel<D, MB>;
+    const int smem = DecLayout<D>::kSmemBytes;
+    if (int rc = check_cuda(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                 smem), "cudaFuncSetAttribute(decode)"))
+        return rc;
+    dim3 grid((Lmax + chunk - 1) / chunk, Hkv, B);
+    kern<<<grid, kDecThreads, smem, stream>>>(tk, tv, static_cast<const __nv_bfloat16 *>(q),
+                                              seqlens, part_o, part_lse, B, Hq, Hkv, Lmax, chunk,
+                                              scale_log2, status);
+    return check_cuda(cudaGetLastError(), "decode_split_kernel launch");
+}
+
+int launch_decode(const void *q, const void *k_cache, const void *v_cache,
+                  const int32_t *seqlens, void *o, int B, int Hq, int Hkv, int d, int Lmax,
+                  float scale, void *workspace, cudaStream_t stream) {
+    if (B > 65535 || Hkv > 65535)
+        return set_error(GQA_ERR_UNSUPPORTED, "decode: B and Hkv must be <= 65535");
+    int *status = device_status_ptr();
+    if (!status) return GQA_ERR_CUDA;
+    const int chunk = decode_chunk(B, Hkv, Lmax);
+    const size_t splits = (static_cast<size_t>(Lmax) + chunk - 1) / chunk;
+    const size_t rows = splits * B * Hq;
+    float *part_o = static_cast<float *>(workspace);
+    float *part_lse = reinterpret_cast<float *>(static_cast<uint8_t *>(workspace) +
+                                                align256(rows * d * sizeof(float)));
+    const int G = Hq / Hkv;
+    const float scale_log2 = scale * 1.4426950408889634f;
+    if (splits > 0) {
+        CUtensorMap tk, tv;
+        if (int rc = encode_tmap_bf16_4d(&tk, k_cache, d, Hkv, Lmax, B, 64, 1, kDecBK, 1, 1)) return rc;
+        if (int rc = encode_tmap_bf16_4d(&tv, v_cache, d, Hkv, Lmax, B, 64, 1, kDecBK, 1, 1)) return rc;
+        int rc;
+        if (d == 128)
+            rc = G <= 16 ? launch_split<128, 1>(tk, tv, q, seqlens, part_o, part_lse, B, Hq, Hkv,
+                                                Lmax, chunk, scale_log2, status, stream)
+                         : launch_split<128, 2>(tk, tv, q, seqlens, part_o, part_lse, B, Hq, Hkv,
+                                                Lmax, chunk, scale_log2, status, stream);
+        else
+            rc = G <= 16 ? launch_split<64, 1>(tk, tv, q, seqlens, part_o, part_lse, B, Hq, Hkv,
+                                               Lmax, chunk, scale_log2, status, stream)
+                         : launch_split<64, 2>(tk, tv, q, seqlens, part_o, part_lse, B, Hq, Hkv,
+                                               Lmax, chunk, scale_log2, status, stream);
+        if (rc) return rc;
+    }
+    const int blocks = (B * Hq + 3) / 4;
+    if (d == 128)
+        decode_combine_kernel<128><<<blocks, 128, 0, stream>>>(
+            part_o, part_lse, seqlens, static_cast<__nv_bfloat16 *>(o), B, Hq, Lmax, chunk);
+    else
+        decode_combine_kernel<64><<<blocks, 128, 0, stream>>>(
+            part_o, part_lse, seqlens, static_cast<__nv_bfloat16 *>(o), B, Hq, Lmax, chunk);
+    return check_cuda(cudaGetLastError(), "decode_combine_kernel launch");
+}
+
+}  // namespace gqa

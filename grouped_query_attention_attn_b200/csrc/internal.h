@@ -1,0 +1,57 @@
+// internal.h -- declarations shared by the library's translation units.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cstddef>
+#include <cstdint>
+
+#include "gqa.h"
+
+namespace gqa {
+
+// Record a message for gqa_last_error() on this host thread; returns `code`.
+int set_error(int code, const char *fmt, ...);
+
+// Map a CUDA runtime error to GQA_ERR_CUDA with a message; GQA_OK on success.
+int check_cuda(cudaError_t e, const char *what);
+
+// GQA_OK when the current device is an sm_100 part, else GQA_ERR_UNSUPPORTED.
+int require_sm100();
+
+// Device address of the library's status word on the current device
+// (looked up once per device); nullptr with a message set on failure.
+int *device_status_ptr();
+
+// 4-D bf16 tensor map over a [n3][n2][n1][n0] contiguous array (n0 innermost),
+// box (b0, b1, b2, b3), 128-byte swizzle when swizzle128 != 0, zero fill out
+// of bounds.  Returns GQA_OK or GQA_ERR_CUDA.
+int encode_tmap_bf16_4d(CUtensorMap *map, const void *base, uint64_t n0, uint64_t n1,
+                        uint64_t n2, uint64_t n3, uint32_t b0, uint32_t b1, uint32_t b2,
+                        uint32_t b3, int swizzle128);
+
+// ---- launchers (arguments already validated by the C-ABI layer) ----------
+int launch_fwd_f32(const float *q, const float *k, const float *v, float *o, float *lse,
+                   int B, int Tq, int Tkv, int Hq, int Hkv, int d, int causal, float scale,
+                   cudaStream_t stream);
+
+int launch_empty_rows(void *o, float *lse, int elem_bytes, int B, int Tq, int Hq, int d,
+                      cudaStream_t stream);
+
+int launch_fold_kv(const void *in, void *out, int B, int T, int H, int g, int d,
+                   cudaStream_t stream);
+
+// Keys per decode split for these sizes (a multiple of the stage size).
+int decode_chunk(int B, int Hkv, int Lmax);
+size_t decode_workspace_bytes(int B, int Hq, int Hkv, int d, int Lmax);
+int launch_decode(const void *q, const void *k_cache, const void *v_cache,
+                  const int32_t *seqlens, void *o, int B, int Hq, int Hkv, int d, int Lmax,
+                  float scale, void *workspace, cudaStream_t stream);
+
+int launch_prefill(const void *q, const void *k, const void *v, void *o, float *lse,
+                   int B, int Tq, int Tkv, int Hq, int Hkv, int d, int causal, float scale,
+                   cudaStream_t stream);
+
+int selftest_wait_timeout(int timeout_us);
+
+}  // namespace gqa

@@ -1,0 +1,159 @@
+/*
+ * gqa.h -- C ABI of libgqa.so, grouped-query scaled-dot-product attention for
+ * NVIDIA B200 (sm_100a).
+ *
+ * The operation (TT Lab "キー・バリューヘッドだけ減らしてみる", steps 1-5; course
+ * "Неделя 7. Внимание", steps 1-2):
+ *
+ *   Hq query heads are split into Hkv contiguous groups of G = Hq / Hkv heads;
+ *   query head hq reads K/V head hq / G (the repeat_interleave expansion of
+ *   the K3 notes "GVA", subsection "Forward: repeat_interleave", never
+ *   materialised).  For query row i of head hq:
+ *       s_j = scale * <q_i, k_j>                      (scale = 1/sqrt(d) usually)
+ *       s_j = -inf  if causal and j > i + (Tkv - Tq)  (mask before the softmax)
+ *       o_i = sum_j softmax(s)_j v_j                  (max subtracted first)
+ *   MHA (Hkv = Hq) and MQA (Hkv = 1) are the end cases.
+ *
+ * Conventions shared by every entry point
+ *   - Layouts are row-major and contiguous: q, o [B, Tq, Hq, d];
+ *     k, v [B, Tkv, Hkv, d]; lse [B, Hq, Tq].
+ *   - All tensor pointers are DEVICE pointers owned by the caller.  The
+ *     library keeps no pointer after a call returns and allocates no device
+ *     memory; scratch space is the caller's `workspace`.
+ *   - Work is enqueued asynchronously on `stream` (a cudaStream_t; NULL is the
+ *     legacy default stream).  A GQA_OK return means "validated and
+ *     launched"; kernel-side problems are reported by gqa_device_status().
+ *   - Arguments are validated on the host before anything is launched; a
+ *     non-zero status is returned and gqa_last_error() gives a message.
+ *     Nothing is launched when a call fails validation.
+ *   - Causal alignment is bottom-right: with Tq != Tkv, query row i sees keys
+ *     j <= i + (Tkv - Tq).  A row that sees no key gets o = 0, lse = -inf.
+ *   - Empty problems (B == 0 or Tq == 0) are valid and launch nothing.
+ */
+#ifndef GQA_H
+#define GQA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+struct CUstream_st;                     /* the type behind cudaStream_t */
+typedef struct CUstream_st *gqa_stream_t;
+
+typedef enum {
+    GQA_OK = 0,
+    GQA_ERR_INVALID_ARG = 1,   /* bad shape, Hq % Hkv != 0, null/misaligned pointer, bad scale */
+    GQA_ERR_UNSUPPORTED = 2,   /* valid but not built: head dim or group size, no sm_100 GPU */
+    GQA_ERR_CUDA = 3,          /* a CUDA runtime/driver call failed (launch, tensor map) */
+    GQA_ERR_WORKSPACE = 4,     /* decode workspace missing or too small */
+    GQA_ERR_TIMEOUT = 5        /* a bounded device-side wait ran out (see gqa_device_status) */
+} gqa_status;
+
+/*
+ * gqa_attn_fwd -- prefill / full-sequence forward, bf16 in, bf16 out, fp32
+ * accumulation and fp32 online softmax on tcgen05 tensor cores.
+ *
+ *   q  [B, Tq,  Hq,  d] bf16      k, v [B, Tkv, Hkv, d] bf16
+ *   o  [B, Tq,  Hq,  d] bf16 (written)
+ *   B, Tq, Tkv >= 0; Hq, Hkv >= 1 with Hq % Hkv == 0 (the lab's ValueError
+ *   becomes GQA_ERR_INVALID_ARG); G = Hq/Hkv <= 128 (else UNSUPPORTED);
+ *   d in {64, 128} (else UNSUPPORTED); causal 0/1; scale > 0 and finite
+ *   (callers normally pass 1/sqrt(d)).  Pointers must be 16-byte aligned
+ *   (tensor-memory-access copies need it).
+ */
+int gqa_attn_fwd(const void *q, const void *k, const void *v, void *o,
+                 int B, int Tq, int Tkv, int Hq, int Hkv, int d,
+                 int causal, float scale, gqa_stream_t stream);
+
+/*
+ * gqa_attn_fwd_lse -- as gqa_attn_fwd, and also writes the natural-log
+ * log-sum-exp of each row's scaled, masked scores:
+ *   lse [B, Hq, Tq] fp32, lse = m + ln(sum_j exp(s_j - m)); -inf for a row
+ *   with no visible key.  lse may be NULL (then identical to gqa_attn_fwd).
+ */
+int gqa_attn_fwd_lse(const void *q, const void *k, const void *v, void *o, float *lse,
+                     int B, int Tq, int Tkv, int Hq, int Hkv, int d,
+                     int causal, float scale, gqa_stream_t stream);
+
+/*
+ * gqa_attn_fwd_f32 -- the same operation in fp32 end to end (fp32 FFMA,
+ * no tensor cores).  Same layouts; fp32 tensors; any 1 <= d <= 256; pointers
+ * 4-byte aligned; lse may be NULL.  A correctness path for fp32 callers, not
+ * a throughput path.
+ */
+int gqa_attn_fwd_f32(const float *q, const float *k, const float *v, float *o, float *lse,
+                     int B, int Tq, int Tkv, int Hq, int Hkv, int d,
+                     int causal, float scale, gqa_stream_t stream);
+
+/*
+ * gqa_decode_workspace_size -- bytes of device scratch gqa_decode needs for
+ * these sizes (partial outputs and log-sum-exp of every KV split).  Returns 0
+ * for invalid sizes.  Pure host function, no CUDA call.
+ */
+size_t gqa_decode_workspace_size(int B, int Hq, int Hkv, int d, int Lmax);
+
+/*
+ * gqa_decode -- one new query token per sequence against a KV cache
+ * (the course's KV-cache motivation, step 2; the causal mask leaves every
+ * cached key visible to the newest token).
+ *
+ *   q        [B, Hq, d] bf16
+ *   k_cache, v_cache [B, Lmax, Hkv, d] bf16; rows >= seqlens[b] are never read
+ *   seqlens  [B] int32 DEVICE array, 0 <= seqlens[b] <= Lmax
+ *   o        [B, Hq, d] bf16 (written; a sequence of length 0 gets zeros)
+ *   workspace: device scratch of at least gqa_decode_workspace_size(...)
+ *   bytes, 256-byte aligned; its contents on entry do not matter.
+ *   d in {64, 128}; Hq % Hkv == 0; G = Hq/Hkv <= 64.
+ * Each split of the KV length is streamed from HBM once for all G query heads
+ * of its group, and the splits are merged with the log-sum-exp identity by a
+ * second kernel on the same stream.  A seqlens[b] above Lmax is clamped to
+ * Lmax and flagged in gqa_device_status (GQA_ERR_INVALID_ARG).
+ */
+int gqa_decode(const void *q, const void *k_cache, const void *v_cache,
+               const int32_t *seqlens, void *o,
+               int B, int Hq, int Hkv, int d, int Lmax, float scale,
+               void *workspace, size_t workspace_bytes, gqa_stream_t stream);
+
+/*
+ * gqa_fold_kv -- MHA -> GQA conversion of a K or V tensor by mean pooling
+ * (TT Lab step 2, course step 2: average the heads of each contiguous group).
+ *   in  [B, T, H, d] bf16, out [B, T, g, d] bf16 (written), H % g == 0.
+ * Members of a group are added in head order in fp32, divided by H/g in fp32
+ * and rounded to bf16 (nearest even).  d must be a multiple of 8 and both
+ * pointers 16-byte aligned.
+ */
+int gqa_fold_kv(const void *in, void *out, int B, int T, int H, int g, int d,
+                gqa_stream_t stream);
+
+/*
+ * gqa_last_error -- message for the last non-OK status returned on the
+ * calling host thread ("" if none).  Valid until the next call on the thread.
+ */
+const char *gqa_last_error(void);
+
+/*
+ * gqa_device_status -- synchronises the current device, then reports the
+ * first error a kernel recorded since the last reset (GQA_OK if none):
+ * GQA_ERR_TIMEOUT when a bounded wait inside a kernel ran out (the kernel
+ * then stopped early and its output is incomplete), GQA_ERR_INVALID_ARG for a
+ * decode length above Lmax.  reset != 0 clears the record.
+ */
+int gqa_device_status(int reset);
+
+/*
+ * gqa_selftest_wait_timeout -- launches a one-warp kernel that waits on a
+ * shared-memory barrier nothing will ever arrive at, bounded by timeout_us
+ * microseconds, and returns what that kernel recorded: GQA_ERR_TIMEOUT when
+ * the bound works.  Exercises the failure path of every bounded wait without
+ * hanging or faulting the GPU; synchronises the device; resets the record.
+ */
+int gqa_selftest_wait_timeout(int timeout_us);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GQA_H */

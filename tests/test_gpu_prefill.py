@@ -1,0 +1,144 @@
+"""tcgen05 prefill kernel against the double oracle (2e-2 max-abs on o, lse)."""
+
+import numpy as np
+import pytest
+import torch
+
+import grouped_query_attention_attn_b200 as gqa
+from grouped_query_attention_attn_b200 import workloads
+from oracle import ref
+from parity import BF16_TOL, gather_lse, gather_rows, max_abs, sample_rows
+
+pytestmark = pytest.mark.gpu
+
+
+def check_full(q, k, v, causal, tol=BF16_TOL):
+    o_ref, lse_ref = ref.attn_fwd(q, k, v, causal)
+    o, lse = gqa.attn(q.cuda(), k.cuda(), v.cuda(), causal=causal, return_lse=True)
+    gqa.device_status()
+    err = max_abs(o, o_ref)
+    assert err <= tol, err
+    l = lse.cpu().numpy().astype(np.float64)
+    fin = np.isfinite(lse_ref)
+    assert np.array_equal(np.isneginf(l), ~fin)
+    assert np.max(np.abs(l[fin] - lse_ref[fin]), initial=0.0) <= tol
+    return o
+
+
+CASES = [
+    # B, Tq, Tkv, Hq, Hkv, d, causal
+    (1, 128, 128, 1, 1, 128, False),     # one tile, MHA
+    (1, 128, 128, 1, 1, 128, True),
+    (1, 300, 300, 8, 2, 128, True),      # several tiles and a ragged tail, G = 4
+    (2, 300, 300, 8, 2, 128, False),
+    (1, 257, 257, 8, 8, 128, True),      # MHA end case
+    (1, 200, 200, 8, 1, 128, True),      # MQA end case, G = 8
+    (1, 100, 100, 32, 1, 64, True),      # G = 32, d = 64
+    (1, 90, 90, 12, 4, 128, True),       # G = 3: 42 positions x 3 heads per tile
+    (1, 77, 77, 6, 1, 64, False),        # G = 6
+    (2, 100, 300, 8, 2, 128, True),      # Tq < Tkv: bottom-right causal alignment
+    (1, 300, 100, 8, 2, 128, True),      # Tq > Tkv: early rows see no key
+    (1, 1, 1, 4, 2, 128, True),          # one token
+    (1, 1, 500, 4, 2, 64, True),
+    (1, 520, 520, 128, 1, 64, True),     # G = 128: one position per tile
+    (3, 64, 64, 4, 2, 128, False),
+]
+
+
+@pytest.mark.parametrize("B,Tq,Tkv,Hq,Hkv,d,causal", CASES)
+def test_prefill_small(gqa_lib, B, Tq, Tkv, Hq, Hkv, d, causal):
+    q, k, v = workloads.prefill_inputs(B, Tq, Hq, Hkv, d, Tkv=Tkv,
+                                       seeds=(Tq + 1, Tkv + 2, Hq + d))
+    check_full(q, k, v, causal)
+
+
+def test_large_logits_small(gqa_lib):
+    # q, k ~ N(0,1) x 8: logits with sigma ~ 64 (the long-context stress values)
+    q, k, v = workloads.prefill_inputs(1, 400, 16, 2, 128, qk_std=8.0, seeds=(7, 8, 9))
+    check_full(q, k, v, True)
+
+
+def test_empty_keys(gqa_lib):
+    q = torch.randn(1, 5, 4, 128, device="cuda").bfloat16()
+    k = torch.empty(1, 0, 2, 128, device="cuda", dtype=torch.bfloat16)
+    o, lse = gqa.attn(q, k, k.clone(), causal=True, return_lse=True)
+    assert torch.all(o == 0) and torch.all(torch.isneginf(lse))
+
+
+def test_no_future_leakage(gqa_lib):
+    q, k, v = workloads.prefill_inputs(1, 384, 8, 2, 128, seeds=(11, 12, 13))
+    o1 = gqa.attn(q.cuda(), k.cuda(), v.cuda(), causal=True)
+    k2, v2 = k.clone(), v.clone()
+    k2[:, 200:] = k2[:, 200:] * 3 + 1
+    v2[:, 200:] = -v2[:, 200:]
+    o2 = gqa.attn(q.cuda(), k2.cuda(), v2.cuda(), causal=True)
+    assert torch.equal(o1[:, :200], o2[:, :200])
+    assert not torch.equal(o1[:, 200:], o2[:, 200:])
+
+
+def test_mha_equals_each_head_alone(gqa_lib):
+    q, k, v = workloads.prefill_inputs(1, 300, 4, 4, 128, seeds=(21, 22, 23))
+    qc, kc, vc = q.cuda(), k.cuda(), v.cuda()
+    o = gqa.attn(qc, kc, vc, causal=True)
+    for h in range(4):
+        oh = gqa.attn(qc[:, :, h:h + 1].contiguous(), kc[:, :, h:h + 1].contiguous(),
+                      vc[:, :, h:h + 1].contiguous(), causal=True)
+        assert torch.equal(o[:, :, h:h + 1], oh)
+
+
+def test_gqa_equals_expanded_kv(gqa_lib):
+    # reading K/V head hq // G equals MHA on repeat_interleave'd K/V
+    q, k, v = workloads.prefill_inputs(2, 260, 8, 2, 128, seeds=(31, 32, 33))
+    qc, kc, vc = q.cuda(), k.cuda(), v.cuda()
+    o = gqa.attn(qc, kc, vc, causal=True)
+    oe = gqa.attn(qc, kc.repeat_interleave(4, 2).contiguous(),
+                  vc.repeat_interleave(4, 2).contiguous(), causal=True)
+    assert max_abs(o, oe.float().cpu().numpy()) <= 1e-2
+    ow = gqa.attn(qc, kc.repeat(1, 1, 4, 1).contiguous(), vc.repeat(1, 1, 4, 1).contiguous(),
+                  causal=True)
+    assert max_abs(o, ow.float().cpu().numpy()) > 0.1        # interleaved order is wrong
+
+
+def test_deterministic(gqa_lib):
+    q, k, v = workloads.prefill_inputs(1, 333, 8, 2, 128, seeds=(41, 42, 43))
+    args = (q.cuda(), k.cuda(), v.cuda())
+    assert torch.equal(gqa.attn(*args, causal=True), gqa.attn(*args, causal=True))
+
+
+# ----------------------------------------------------- full workload sizes --
+
+def check_sampled(q, k, v, causal, n_rows, seed):
+    B, Tq, Hq, _ = q.shape
+    o, lse = gqa.attn(q.cuda(), k.cuda(), v.cuda(), causal=causal, return_lse=True)
+    gqa.device_status()
+    rows = sample_rows(B, Tq, Hq, n_rows, seed)
+    o_ref, lse_ref = ref.attn_fwd_rows(q, k, v, rows, causal)
+    assert max_abs(gather_rows(o, rows, Tq, Hq), o_ref) <= BF16_TOL
+    assert max_abs(gather_lse(lse, rows), lse_ref) <= BF16_TOL
+    assert bool(torch.isfinite(o).all())
+
+
+def test_llama3_8b_causal_t4096(gqa_lib):
+    q, k, v = workloads.prefill_inputs(1, 4096, 32, 8, 128)
+    check_sampled(q, k, v, True, 768, 1)
+
+
+@pytest.mark.parametrize("Hkv", [32, 8, 1])
+def test_head_sharing_sweep_t2048(gqa_lib, Hkv):
+    # K/V for Hkv < 32 are the fold (mean of contiguous head groups) of the
+    # Hkv = 32 tensors: folded on the GPU for the kernel, by the oracle for it
+    q, k32, v32 = workloads.prefill_inputs(4, 2048, 32, 32, 128)
+    k_ref, v_ref = ref.fold_kv_tensor(k32, Hkv), ref.fold_kv_tensor(v32, Hkv)
+    kg, vg = gqa.fold_kv(k32.cuda(), Hkv), gqa.fold_kv(v32.cuda(), Hkv)
+    assert torch.equal(kg.cpu(), k_ref) and torch.equal(vg.cpu(), v_ref)
+    B, Tq, Hq, _ = q.shape
+    o, lse = gqa.attn(q.cuda(), kg, vg, causal=True, return_lse=True)
+    rows = sample_rows(B, Tq, Hq, 512, Hkv)
+    o_ref, lse_ref = ref.attn_fwd_rows(q, k_ref, v_ref, rows, True)
+    assert max_abs(gather_rows(o, rows, Tq, Hq), o_ref) <= BF16_TOL
+    assert max_abs(gather_lse(lse, rows), lse_ref) <= BF16_TOL
+
+
+def test_long_context_t32768(gqa_lib):
+    q, k, v = workloads.prefill_inputs(1, 32768, 64, 8, 128, qk_std=8.0)
+    check_sampled(q, k, v, True, 2048, 5)
