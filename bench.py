@@ -1,0 +1,421 @@
+#!/usr/bin/env python
+"""Throughput benchmark of the grouped-query attention hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+One step = one pass of the whole hot path over one batch of synthetic input:
+  1. causal prefill, B=1, Hq=32, Hkv=8, T=4096, d=128 (Llama-3-8B head
+     shapes), bf16 in/out, fp32 accumulation -- the headline workload;
+  2. batched decode, B=64 sequences, Hq=32, Hkv=8, d=128, cache lengths
+     uniform on [1024, 8192], split-KV kernel + log-sum-exp combine.
+Inputs are seeded synthetic tensors already resident in HBM.  L2 (126 MB) is
+flushed by writing a 256 MB buffer before every timed launch; each launch is
+timed with CUDA events on the stream it runs on.
+
+The JSON line's ``value`` is prefill TFLOP/s (algorithmic FLOPs: 4*B*Hq*d*
+unmasked pairs, all ranks) and ``decode.value`` is decode KV GB/s.  ``e2e``
+repeats the prefill through host (pinned) buffers with the copies timed.
+``cpu_baseline`` times the CPU oracle on a sample of query rows of the same
+workload.  With --gpus N > 1 (torchrun) every rank runs its own copy of the
+workload (the path has no exchange step): weak scaling, time = max over ranks.
+
+``--impl reference`` times the CPU oracle instead (rank 0 only), on bounded
+samples of the same workload, and prints the same metric.
+"""
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "GQA prefill TFLOP/s and decode KV GB/s on 1 B200 (% of roofline)"
+PREFILL = dict(B=1, Hq=32, Hkv=8, T=4096, d=128, causal=True)
+DECODE = dict(B=64, Hq=32, Hkv=8, d=128, Lmin=1024, Lmax=8192)
+WORKLOAD = "prefill_causal_llama3_8b_t4096 + decode_b64_l1024_8192"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.txt")
+
+
+def prefill_flops(c):
+    pairs = c["T"] * (c["T"] + 1) // 2 if c["causal"] else c["T"] * c["T"]
+    return 4 * c["B"] * c["Hq"] * c["d"] * pairs
+
+
+def decode_bytes(seqlens, c):
+    kv = int(seqlens.sum()) * c["Hkv"] * c["d"] * 2 * 2
+    return kv + 2 * c["B"] * c["Hq"] * c["d"] * 2          # + q and o
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return p, "measured"
+    except (OSError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def kernel_source_hash(names):
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "grouped_query_attention_attn_b200", "csrc")
+    for n in names:
+        with open(os.path.join(csrc, n), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(kernel, src_hash):
+    """DRAM bytes per launch from the committed ncu summary, if the kernel is unchanged.
+
+    profiles/traffic.txt lines: <kernel> <source sha256[:16]> <dram read+write bytes>."""
+    try:
+        with open(TRAFFIC_FILE) as f:
+            for line in f:
+                parts = line.split()
+                if len(parts) == 3 and parts[0] == kernel and parts[1] == src_hash:
+                    return int(parts[2])
+    except OSError:
+        pass
+    return None
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle sampling while the timed region runs."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device):
+        self.proc = None
+        try:
+            self.uuid = "GPU-" + str(torch.cuda.get_device_properties(device).uuid)
+        except Exception:
+            self.uuid = None
+
+    def start(self):
+        cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+               "-lms", "50"]
+        if self.uuid:
+            cmd += ["-i", self.uuid]
+        try:
+            self.proc = subprocess.Popen(cmd, stdout=subprocess.PIPE, stderr=subprocess.DEVNULL,
+                                         text=True)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        out, _ = self.proc.communicate(timeout=10)
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 6:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                smax = float(parts[1])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[2:6]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax,
+                "samples": len(sm), "reasons": sorted(reasons)}
+
+
+def dist_init(n_gpus):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != n_gpus and world > 1:
+        raise SystemExit(f"--gpus {n_gpus} but WORLD_SIZE={world}")
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x, world, device):
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ------------------------------------------------------------ CPU oracle --
+
+def oracle_prefill_sample(q, k, v, n_rows, seed=0):
+    """Time the oracle on n_rows query rows of the prefill workload.
+
+    Returns (seconds, algorithmic FLOPs of the rows, rows, outputs)."""
+    import numpy as np
+    from oracle import ref
+    B, T, Hq, d = q.shape
+    rng = np.random.default_rng(seed)
+    rows = np.sort(rng.choice(B * Hq * T, size=n_rows, replace=False)).astype(np.int64)
+    pos = rows % T
+    flops = int(4 * d * (pos + 1).sum())                # causal: row i sees i+1 keys
+    t = time.perf_counter()
+    o, lse = ref.attn_fwd_rows(q, k, v, rows, causal=True)
+    return time.perf_counter() - t, flops, rows, o
+
+
+def calibrate_row_seconds(q, k, v, n=256):
+    """Oracle seconds per random query row of the prefill workload."""
+    secs, _, _, _ = oracle_prefill_sample(q, k, v, n, seed=12345)
+    return max(secs / n, 1e-7)
+
+
+def run_reference(args, world, rank):
+    """The CPU oracle as the reference arm: rank 0 only, bounded samples."""
+    if rank != 0:
+        return
+    from grouped_query_attention_attn_b200 import workloads
+    from oracle import ref
+    c = PREFILL
+    q, k, v = workloads.prefill_inputs(c["B"], c["T"], c["Hq"], c["Hkv"], c["d"])
+    ref.build_oracle()
+    for i in range(args.warmup):
+        oracle_prefill_sample(q, k, v, 64, seed=1000 + i)
+    # rows per step sized so that all K steps take about args.ref_budget seconds
+    per_row = calibrate_row_seconds(q, k, v)
+    rows = int(min(max(args.ref_budget / args.steps / per_row, 16), c["B"] * c["Hq"] * c["T"]))
+    secs, flops = 0.0, 0
+    for i in range(args.steps):
+        s, f, _, _ = oracle_prefill_sample(q, k, v, rows, seed=i)
+        secs += s
+        flops += f
+    value = flops / secs / 1e12
+    cores = ref.num_threads()
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000 * secs / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "impl": "reference",
+        "config": {"workload": WORKLOAD, "prefill": c, "decode": DECODE,
+                   "l2": "flushed (256 MB write) before every timed launch",
+                   "parallelism": "1 GPU"},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+                         "sample": f"{rows} random query rows of the causal T=4096 "
+                                   f"prefill per step (C double oracle, OpenMP)"},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------- GPU path --
+
+def run_ours(args, world, rank, local):
+    import grouped_query_attention_attn_b200 as gqa
+    from grouped_query_attention_attn_b200 import workloads
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+    do_pre = args.only in (None, "prefill")
+    do_dec = args.only in (None, "decode")
+
+    c, dc = PREFILL, DECODE
+    stream = torch.cuda.current_stream(dev)
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    if do_pre:
+        q_h, k_h, v_h = workloads.prefill_inputs(c["B"], c["T"], c["Hq"], c["Hkv"], c["d"])
+        q, k, v = q_h.to(dev), k_h.to(dev), v_h.to(dev)
+        o = torch.empty_like(q)
+    if do_dec:
+        dq_h, kc_h, vc_h, sl_h = workloads.decode_inputs(dc["B"], dc["Hq"], dc["Hkv"], dc["d"],
+                                                         dc["Lmin"], dc["Lmax"])
+        dq, kc, vc, sl = dq_h.to(dev), kc_h.to(dev), vc_h.to(dev), sl_h.to(dev)
+        do = torch.empty_like(dq)
+        ws = torch.empty(gqa.decode_workspace_size(dc["B"], dc["Hq"], dc["Hkv"], dc["d"],
+                                                   dc["Lmax"]), dtype=torch.uint8, device=dev)
+
+    def step(evs=None):
+        if do_pre:
+            flush.zero_()
+            if evs:
+                evs[0].record(stream)
+            gqa.attn(q, k, v, causal=True, out=o)
+            if evs:
+                evs[1].record(stream)
+        if do_dec:
+            flush.zero_()
+            if evs:
+                evs[2].record(stream)
+            gqa.decode(dq, kc, vc, sl, workspace=ws, out=do)
+            if evs:
+                evs[3].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    gqa.device_status()
+    K = args.steps
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(K)]
+    sampler = ClockSampler(dev)
+    sampler.start()
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    t_wall = time.perf_counter()
+    for i in range(K):
+        step(evs[i])
+    torch.cuda.synchronize(dev)
+    barrier(world)
+    wall = time.perf_counter() - t_wall
+    clocks = sampler.stop()
+    gqa.device_status()
+    pre_ms = sum(e[0].elapsed_time(e[1]) for e in evs) if do_pre else 0.0
+    dec_ms = sum(e[2].elapsed_time(e[3]) for e in evs) if do_dec else 0.0
+    pre_ms = max_over_ranks(pre_ms, world, dev)
+    dec_ms = max_over_ranks(dec_ms, world, dev)
+    peaks, peak_kind = load_peaks()
+
+    value, roofline, e2e, cpu = None, None, None, None
+    if do_pre:
+        p_flops = prefill_flops(c)
+        value = world * p_flops * K / (pre_ms / 1e3) / 1e12
+        launch_ms = pre_ms / K
+        roofline = {"bound": "tensor", "achieved": p_flops / (launch_ms / 1e3) / 1e12,
+                    "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                    "peak_kind": f"{peak_kind} bf16 burst (kernel timed alone)",
+                    "traffic": recorded_traffic("prefill_kernel",
+                                                kernel_source_hash(["prefill.cu", "device.cuh"])),
+                    "kernel": "prefill_kernel<128>", "flops_per_launch": p_flops,
+                    "launch_ms": launch_ms}
+        roofline["frac"] = roofline["achieved"] / roofline["peak"]
+        roofline["frac_of_nominal_2250"] = roofline["achieved"] / 2250.0
+
+        # ---- end to end through host buffers (the headline metric) ----
+        if not args.no_e2e:
+            qp, kp, vp = q_h.pin_memory(), k_h.pin_memory(), v_h.pin_memory()
+            op = torch.empty(o.shape, dtype=o.dtype).pin_memory()
+            n_e2e = max(3, min(K, 50))
+
+            def e2e_step():
+                qd = qp.to(dev, non_blocking=True)
+                kd = kp.to(dev, non_blocking=True)
+                vd = vp.to(dev, non_blocking=True)
+                od = gqa.attn(qd, kd, vd, causal=True)
+                op.copy_(od, non_blocking=True)
+
+            for _ in range(3):
+                e2e_step()
+            torch.cuda.synchronize(dev)
+            barrier(world)
+            s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            s0.record(stream)
+            for _ in range(n_e2e):
+                e2e_step()
+            s1.record(stream)
+            torch.cuda.synchronize(dev)
+            e2e_ms = max_over_ranks(s0.elapsed_time(s1), world, dev)
+            e2e = {"value": world * p_flops * n_e2e / (e2e_ms / 1e3) / 1e12, "unit": "TFLOP/s",
+                   "h2d_bytes_per_step": sum(t.numel() * t.element_size() for t in (qp, kp, vp)),
+                   "d2h_bytes_per_step": op.numel() * op.element_size(), "steps": n_e2e}
+
+        if rank == 0 and not args.no_cpu:
+            import numpy as np
+            from oracle import ref
+            ref.build_oracle()
+            per_row = calibrate_row_seconds(q_h, k_h, v_h)
+            n_rows = int(min(max(args.cpu_seconds / per_row, 256), c["B"] * c["Hq"] * c["T"]))
+            secs, flops, rows, o_ref = oracle_prefill_sample(q_h, k_h, v_h, n_rows)
+            T, Hq = c["T"], c["Hq"]
+            r = torch.as_tensor(rows)
+            got = o[(r // (T * Hq)).to(dev), (r % T).to(dev), ((r // T) % Hq).to(dev)]
+            err = float(np.max(np.abs(got.float().cpu().numpy() - o_ref)))
+            cpu = {"value": flops / secs / 1e12, "unit": "TFLOP/s", "cores": ref.num_threads(),
+                   "kind": "oracle", "seconds": secs,
+                   "sample": f"{n_rows} random query rows of the causal T=4096 prefill "
+                             f"(C double oracle, OpenMP)",
+                   "max_abs_err_vs_gpu": err}
+
+    dec = None
+    if do_dec:
+        d_bytes = decode_bytes(sl_h, dc)
+        launch_ms = dec_ms / K
+        dec_roof = {"bound": "hbm", "achieved": d_bytes / (launch_ms / 1e3) / 1e9,
+                    "peak": peaks["hbm_gbs"], "unit": "GB/s", "peak_kind": f"{peak_kind} copy",
+                    "traffic": recorded_traffic("decode_split_kernel",
+                                                kernel_source_hash(["decode.cu", "device.cuh"])),
+                    "bytes_per_step": d_bytes, "launch_ms": launch_ms,
+                    "kernels": "decode_split_kernel<128,1> + decode_combine_kernel<128>"}
+        dec_roof["frac"] = dec_roof["achieved"] / dec_roof["peak"]
+        dec_roof["frac_of_nominal_8000"] = dec_roof["achieved"] / 8000.0
+        dec = {"value": world * d_bytes * K / (dec_ms / 1e3) / 1e9, "unit": "GB/s",
+               "roofline": dec_roof}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value if do_pre else (dec or {}).get("value"),
+            "unit": "TFLOP/s" if do_pre else "GB/s", "n_gpus": world,
+            "steps": K, "warmup": args.warmup, "ms_per_step": (pre_ms + dec_ms) / K,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic",
+            "config": {"workload": WORKLOAD if args.only is None else args.only,
+                       "prefill": c if do_pre else None, "decode": dc if do_dec else None,
+                       "l2": "flushed (256 MB write) before every timed launch",
+                       "parallelism": f"{world} independent replicas" if world > 1 else "1 GPU"},
+            "decode": dec,
+            "roofline": roofline if do_pre else (dec or {}).get("roofline"),
+            "clocks": clocks,
+            "e2e": e2e,
+            "gpu_launches": K * ((1 if do_pre else 0) + (2 if do_dec else 0)),
+            "wall_s_timed_region": wall,
+            "cpu_baseline": cpu,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=1000)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0,
+                    help="target seconds of oracle work for the CPU baseline")
+    ap.add_argument("--ref-budget", type=float, default=90.0,
+                    help="target seconds of oracle work for all steps of --impl reference")
+    ap.add_argument("--only", choices=["prefill", "decode"], default=None,
+                    help="time one kernel family only (profiling runs)")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        raise SystemExit("--warmup must be >= 3")
+    world, rank, local = dist_init(args.gpus)
+    if args.impl == "reference":
+        run_reference(args, world, rank)
+        return
+    run_ours(args, world, rank, local)
+
+
+if __name__ == "__main__":
+    main()
