@@ -31,6 +31,7 @@ _SIGNATURES = {
     "gqa_attn_fwd_f32": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _P]),
     "gqa_decode_workspace_size": (ctypes.c_size_t, [_I, _I, _I, _I, _I]),
     "gqa_decode": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _P, ctypes.c_size_t, _P]),
+    "gqa_decode_static": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _P]),
     "gqa_fold_kv": (_I, [_P, _P, _I, _I, _I, _I, _I, _P]),
     "gqa_last_error": (ctypes.c_char_p, []),
     "gqa_device_status": (_I, [_I]),
@@ -74,6 +75,12 @@ def gqa_decode(q, k_cache, v_cache, seqlens, o, B, Hq, Hkv, d, Lmax, scale, work
                workspace_bytes, stream):
     return lib().gqa_decode(q, k_cache, v_cache, seqlens, o, B, Hq, Hkv, d, Lmax, scale,
                             workspace, workspace_bytes, stream)
+
+
+def gqa_decode_static(q, k_cache, v_cache, seqlens, o, B, Hq, Hkv, d, Lmax, scale, stream):
+    """Decode with the library's built-in scratch, for callers that cannot allocate."""
+    return lib().gqa_decode_static(q, k_cache, v_cache, seqlens, o, B, Hq, Hkv, d, Lmax, scale,
+                                   stream)
 
 
 def gqa_fold_kv(inp, out, B, T, H, g, d, stream):

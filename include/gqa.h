@@ -118,6 +118,39 @@ int gqa_decode(const void *q, const void *k_cache, const void *v_cache,
                void *workspace, size_t workspace_bytes, gqa_stream_t stream);
 
 /*
+ * gqa_decode_static -- gqa_decode for callers that cannot allocate device
+ * memory.  (The pages have no counterpart: this is a library convenience.)
+ *
+ * Who needs it: code that may not call cudaMalloc where it decodes -- a
+ * runtime whose memory pool or arena owns all device memory, a plugin whose
+ * host framework forbids allocation on its hot path, or code that must not
+ * risk the device-wide synchronisation cudaMalloc/cudaFree can cause.
+ * gqa_decode needs scratch for the partial results of its KV splits; this
+ * entry point uses a scratch array built into the library instead of a
+ * caller `workspace`.  Inputs and outputs are the caller's, exactly as for
+ * gqa_decode (same arguments minus workspace, same validation and errors).
+ *
+ * Limits and behaviour:
+ *   - The built-in scratch is 32 MiB per GPU, held by every GPU that loads
+ *     the library's code until the process exits.  Sizes whose
+ *     gqa_decode_workspace_size(...) exceeds it are rejected with
+ *     GQA_ERR_WORKSPACE and nothing is launched (B=64, Hq=32, d=128,
+ *     Lmax=8192 fits).
+ *   - The first call with a given device current looks up the scratch's
+ *     device address (cudaGetSymbolAddress) and caches it; make that first
+ *     call on each device before any stream capture.
+ *   - All calls on a device share the one scratch array, which keeps the last
+ *     call's contents.  Nothing in it needs to start at zero, but calls whose
+ *     kernels overlap on the GPU (different streams, or several host threads)
+ *     race on it: serialise them, e.g. on one stream.
+ *   - No cudaMalloc, cudaFree or other allocating routine is called.
+ */
+int gqa_decode_static(const void *q, const void *k_cache, const void *v_cache,
+                      const int32_t *seqlens, void *o,
+                      int B, int Hq, int Hkv, int d, int Lmax, float scale,
+                      gqa_stream_t stream);
+
+/*
  * gqa_fold_kv -- MHA -> GQA conversion of a K or V tensor by mean pooling
  * (TT Lab step 2, course step 2: average the heads of each contiguous group).
  *   in  [B, T, H, d] bf16, out [B, T, g, d] bf16 (written), H % g == 0.
