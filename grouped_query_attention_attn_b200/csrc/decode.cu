@@ -200,16 +200,19 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tm_k,
                     alpha[h] = fast_exp2(m_run[mb][h] - m_use[h]);
                     m_run[mb][h] = m_new;
                 }
-                float psum[2] = {0.0f, 0.0f};
 #pragma unroll
                 for (int nb = 0; nb < 2; ++nb)
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        s[nb][e] = fast_exp2(s[nb][e] - m_use[e >> 1]);
-                        psum[e >> 1] += s[nb][e];
-                    }
-#pragma unroll
-                for (int h = 0; h < 2; ++h) l_run[mb][h] = l_run[mb][h] * alpha[h] + psum[h];
+                    for (int e = 0; e < 4; ++e) s[nb][e] = fast_exp2(s[nb][e] - m_use[e >> 1]);
+                pa[mb][0] = pack_bf16x2(s[0][0], s[0][1]);   // row gq
+                pa[mb][1] = pack_bf16x2(s[0][2], s[0][3]);   // row gq + 8
+                pa[mb][2] = pack_bf16x2(s[1][0], s[1][1]);   // row gq
+                pa[mb][3] = pack_bf16x2(s[1][2], s[1][3]);   // row gq + 8
+                // l sums the bf16 weights the PV product uses (see prefill.cu)
+                const float2 w0 = bf16x2_to_float2(pa[mb][0]), w1 = bf16x2_to_float2(pa[mb][1]);
+                const float2 w2 = bf16x2_to_float2(pa[mb][2]), w3 = bf16x2_to_float2(pa[mb][3]);
+                l_run[mb][0] = l_run[mb][0] * alpha[0] + ((w0.x + w0.y) + (w2.x + w2.y));
+                l_run[mb][1] = l_run[mb][1] * alpha[1] + ((w1.x + w1.y) + (w3.x + w3.y));
 #pragma unroll
                 for (int nd = 0; nd < D / 8; ++nd) {
                     oacc[mb][nd][0] *= alpha[0];
@@ -217,10 +220,6 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tm_k,
                     oacc[mb][nd][2] *= alpha[1];
                     oacc[mb][nd][3] *= alpha[1];
                 }
-                pa[mb][0] = pack_bf16x2(s[0][0], s[0][1]);
-                pa[mb][1] = pack_bf16x2(s[0][2], s[0][3]);
-                pa[mb][2] = pack_bf16x2(s[1][0], s[1][1]);
-                pa[mb][3] = pack_bf16x2(s[1][2], s[1][3]);
             }
             const uint32_t vbase = smem_u32(vt);
             const int vrow = warp * 16 + (lane & 7) + (((lane >> 3) & 1) << 3);

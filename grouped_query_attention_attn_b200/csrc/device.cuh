@@ -260,9 +260,105 @@ __device__ __forceinline__ float fast_exp2(float x) {
     return y;
 }
 
+// Packed fp32 pairs (sm_100 FFMA2 / FADD2 / FMUL2): one instruction, two lanes.
+// Operands are packed inside the asm so no local ever needs an address.
+__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) {
+    float2 r;
+    asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
+        "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\tmov.b64 rc, {%6, %7};\n\t"
+        "fma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(r.x), "=f"(r.y)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+    return r;
+}
+
+__device__ __forceinline__ float2 add2(float2 a, float2 b) {
+    float2 r;
+    asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+        "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+        "add.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(r.x), "=f"(r.y)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+    return r;
+}
+
+__device__ __forceinline__ float2 mul2(float2 a, float2 b) {
+    float2 r;
+    asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+        "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+        "mul.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(r.x), "=f"(r.y)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+    return r;
+}
+
+__device__ __forceinline__ float max3f(float a, float b, float c) {
+    float r;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+    return r;
+}
+
+// Per-warpgroup register budget changes (all four warps of the group execute them).
+template <uint32_t N>
+__device__ __forceinline__ void regs_dec() {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <uint32_t N>
+__device__ __forceinline__ void regs_inc() {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
     return *reinterpret_cast<uint32_t *>(&v);
+}
+
+// bf16 pair by truncation: the high halves of lo and hi (one byte permute on
+// the integer pipe instead of a conversion).
+__device__ __forceinline__ uint32_t pack_hi16(float lo, float hi) {
+    uint32_t r;
+    asm("prmt.b32 %0, %1, %2, 0x7632;" : "=r"(r) : "r"(__float_as_uint(lo)), "r"(__float_as_uint(hi)));
+    return r;
+}
+
+// 2^x for a pair, mostly on the FMA pipe.  Cody-Waite reduction x = n + f
+// with n = round(x) (adding 1.5 * 2^23 rounds to an integer in the low
+// mantissa bits) and f in [-1/2, 1/2]; 2^f from a degree-3 minimax polynomial
+// fitted by csrc/fit_exp2_poly.py (max relative error 7.5e-5); 2^n applied by
+// adding n to the exponent field with an integer multiply-add
+// (bits(t) * 2^23 == n << 23 mod 2^32 because the constant's low 9 bits are
+// zero).  x is clamped to >= -126 so the result stays a normal float
+// (2^-126 stands in for anything smaller).  Not for x = -inf: masked scores
+// use the MUFU path.
+__device__ __forceinline__ float2 exp2_poly2(float2 x) {
+    constexpr float kC0 = 9.999280572e-01f, kC1 = 6.932609677e-01f;
+    constexpr float kC2 = 2.426111251e-01f, kC3 = 5.517166853e-02f;
+    constexpr float kRound = 12582912.0f;                    // 1.5 * 2^23
+    x.x = fmaxf(x.x, -126.0f);
+    x.y = fmaxf(x.y, -126.0f);
+    const float2 t = add2(x, make_float2(kRound, kRound));  // round(x) in the low bits
+    const float2 n = add2(t, make_float2(-kRound, -kRound));
+    const float2 f = add2(x, make_float2(-n.x, -n.y));
+    float2 p = fma2(f, make_float2(kC3, kC3), make_float2(kC2, kC2));
+    p = fma2(p, f, make_float2(kC1, kC1));
+    p = fma2(p, f, make_float2(kC0, kC0));
+    uint32_t r0, r1;
+    asm("mad.lo.u32 %0, %1, 8388608, %2;" : "=r"(r0) : "r"(__float_as_uint(t.x)), "r"(__float_as_uint(p.x)));
+    asm("mad.lo.u32 %0, %1, 8388608, %2;" : "=r"(r1) : "r"(__float_as_uint(t.y)), "r"(__float_as_uint(p.y)));
+    return make_float2(__uint_as_float(r0), __uint_as_float(r1));
+}
+
+// acc + (the two bf16 halves of w), with mixed-precision adds (sm_100).
+__device__ __forceinline__ float add_bf16x2(float acc, uint32_t w) {
+    asm("{\n\t.reg .b16 lo, hi;\n\tmov.b32 {lo, hi}, %1;\n\t"
+        "add.rn.f32.bf16 %0, lo, %0;\n\tadd.rn.f32.bf16 %0, hi, %0;\n\t}"
+        : "+f"(acc) : "r"(w));
+    return acc;
+}
+
+// The two bf16 halves of a packed word, widened to fp32 (exact).
+__device__ __forceinline__ float2 bf16x2_to_float2(uint32_t w) {
+    return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u));
 }
 
 __device__ __forceinline__ void named_barrier_sync(int id, int nthreads) {

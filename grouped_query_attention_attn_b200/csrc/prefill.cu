@@ -33,8 +33,13 @@ namespace gqa {
 
 constexpr int kPfBM = 128;      // rows per M tile
 constexpr int kPfBN = 128;      // keys per K/V tile
-constexpr int kPfThreads = 384;
+constexpr int kPfThreads = 640;   // 4 warps producer / MMA + 2 x 8 softmax warps
 constexpr int kPfStages = 2;
+constexpr float kRescaleLog2 = 8.0f;  // lazy rescale threshold (log2 units)
+#ifndef GQA_POLY_PER4
+#define GQA_POLY_PER4 1
+#endif
+constexpr int kPolyPer4 = GQA_POLY_PER4;  // pairs per 4 on the exp2 polynomial
 
 template <int D>
 struct PfLayout {
@@ -63,6 +68,26 @@ struct PfParams {
     int *status;
 };
 
+// 32 scores of one row -> 16 packed bf16 probabilities (truncated) and their
+// running sum over four accumulators.  With kPoly, kPolyPer4 of every 4 pairs
+// use the exp2 polynomial to take load off the MUFU unit.
+template <bool kPoly>
+__device__ __forceinline__ void softmax_chunk(const uint32_t (&s)[32], float2 cc, float2 nm,
+                                              uint32_t (&pk)[16], float (&acc)[4]) {
+#pragma unroll
+    for (int e = 0; e < 16; ++e) {
+        const float2 x = fma2(make_float2(__uint_as_float(s[2 * e]), __uint_as_float(s[2 * e + 1])),
+                              cc, nm);
+        float2 pe;
+        if (kPoly && (e & 3) < kPolyPer4)
+            pe = exp2_poly2(x);
+        else
+            pe = make_float2(fast_exp2(x.x), fast_exp2(x.y));
+        pk[e] = pack_hi16(pe.x, pe.y);
+        acc[e & 3] = add_bf16x2(acc[e & 3], pk[e]);
+    }
+}
+
 template <int D>
 __global__ void __launch_bounds__(kPfThreads, 1)
 prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -74,6 +99,9 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     __shared__ uint64_t q_full, k_full[kPfStages], k_empty[kPfStages], v_full[kPfStages],
         v_empty[kPfStages], s_full[2], p_full[2], o_done[2], mma_drain;
     __shared__ uint32_t tmem_base_sh;
+    // row-max / l exchange between the two warps that share rows:
+    // [phase parity][tile][half][row]
+    __shared__ float xchg[2][2][2][kPfBM];
     __shared__ int abort_flag;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -98,7 +126,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         }
         for (int k = 0; k < 2; ++k) {
             mbar_init(&s_full[k], 1);
-            mbar_init(&p_full[k], 4);
+            mbar_init(&p_full[k], 8);   // every softmax warp of the tile
             mbar_init(&o_done[k], 1);
         }
         mbar_init(&mma_drain, 1);
@@ -120,34 +148,45 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
 
     if (warp == 0) {
         // ------------------------------------------------ TMA producer ----
-        if (lane == 0 && n_kv > 0) {
-            tma_prefetch_desc(&tm_q);
-            tma_prefetch_desc(&tm_k);
-            tma_prefetch_desc(&tm_v);
-            const int q_box_bytes = 64 * p.G * p.P * 2;
-            mbar_expect_tx(&q_full, 2 * Lay::kPanels * q_box_bytes);
-            for (int mt = 0; mt < 2; ++mt)
-                for (int pn = 0; pn < Lay::kPanels; ++pn)
-                    tma_load_4d(sQ + mt * Lay::kQTile + pn * Lay::kQPanel, &tm_q, &q_full, pn * 64,
-                                kvh * p.G, t0 + mt * p.P, b);
+        // The whole warp runs the schedule (barrier waits stay warp-uniform);
+        // one elected lane issues the copies.
+        if (n_kv > 0) {
+            const bool leader = elect_one();
+            if (leader) {
+                tma_prefetch_desc(&tm_q);
+                tma_prefetch_desc(&tm_k);
+                tma_prefetch_desc(&tm_v);
+                const int q_box_bytes = 64 * p.G * p.P * 2;
+                mbar_expect_tx(&q_full, 2 * Lay::kPanels * q_box_bytes);
+                for (int mt = 0; mt < 2; ++mt)
+                    for (int pn = 0; pn < Lay::kPanels; ++pn)
+                        tma_load_4d(sQ + mt * Lay::kQTile + pn * Lay::kQPanel, &tm_q, &q_full,
+                                    pn * 64, kvh * p.G, t0 + mt * p.P, b);
+            }
+            __syncwarp();
             int issued = 0;
             for (int j = 0; j < n_kv; ++j) {
                 const int st = j % kPfStages;
                 const uint32_t ph = (j / kPfStages) & 1;
-                if (!mbar_wait(&k_empty[st], ph ^ 1, &abort_flag, p.status)) break;
-                mbar_expect_tx(&k_full[st], Lay::kKTile);
-                for (int pn = 0; pn < Lay::kPanels; ++pn)
-                    tma_load_4d(sK + st * Lay::kKTile + pn * Lay::kKPanel, &tm_k, &k_full[st],
-                                pn * 64, kvh, j * kPfBN, b);
-                if (!mbar_wait(&v_empty[st], ph ^ 1, &abort_flag, p.status)) {
-                    issued = j + 1;
+                if (!__all_sync(0xffffffffu, mbar_wait(&k_empty[st], ph ^ 1, &abort_flag, p.status)))
                     break;
+                if (leader) {
+                    mbar_expect_tx(&k_full[st], Lay::kKTile);
+                    for (int pn = 0; pn < Lay::kPanels; ++pn)
+                        tma_load_4d(sK + st * Lay::kKTile + pn * Lay::kKPanel, &tm_k, &k_full[st],
+                                    pn * 64, kvh, j * kPfBN, b);
                 }
-                mbar_expect_tx(&v_full[st], Lay::kKTile);
-                for (int pn = 0; pn < Lay::kPanels; ++pn)
-                    tma_load_4d(sV + st * Lay::kKTile + pn * Lay::kKPanel, &tm_v, &v_full[st],
-                                pn * 64, kvh, j * kPfBN, b);
+                __syncwarp();
                 issued = j + 1;
+                if (!__all_sync(0xffffffffu, mbar_wait(&v_empty[st], ph ^ 1, &abort_flag, p.status)))
+                    break;
+                if (leader) {
+                    mbar_expect_tx(&v_full[st], Lay::kKTile);
+                    for (int pn = 0; pn < Lay::kPanels; ++pn)
+                        tma_load_4d(sV + st * Lay::kKTile + pn * Lay::kKPanel, &tm_v, &v_full[st],
+                                    pn * 64, kvh, j * kPfBN, b);
+                }
+                __syncwarp();
             }
             if (abort_flag) {
                 // let copies already in flight land before the block exits
@@ -161,171 +200,255 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         }
     } else if (warp == 1) {
         // ------------------------------------------------- MMA issuer ----
-        if (lane == 0 && n_kv > 0) {
+        // The whole warp follows the schedule; one elected lane issues every
+        // tcgen05.mma and tcgen05.commit (a commit tracks its own thread's MMAs).
+        if (n_kv > 0) {
+            const bool leader = elect_one();
             constexpr uint32_t idesc_s = umma_idesc_bf16(kPfBM, kPfBN, 0, 0);
             constexpr uint32_t idesc_o = umma_idesc_bf16(kPfBM, D, 0, 1);
             const uint32_t sQa = smem_u32(sQ), sKa = smem_u32(sK), sVa = smem_u32(sV);
-            bool ok = mbar_wait(&q_full, 0, &abort_flag, p.status);
+            bool ok = __all_sync(0xffffffffu, mbar_wait(&q_full, 0, &abort_flag, p.status));
             tc_fence_after();
-            // S_k = Q_k K_st^T : K-major A and B, 16 keys of d per instruction
+            // Descriptors are built once; stepping along K only moves the start
+            // address field (low bits, 16-byte units): +32 B per 16 elements
+            // inside a 64-column panel of Q / K, +2048 B per 16 keys of V.
+            static_assert(kPfStages == 2, "descriptor selects assume a 2-deep ring");
+            const uint64_t dq0 = umma_smem_desc(sQa, 16, 1024);
+            const uint64_t dq1 = umma_smem_desc(sQa + Lay::kQTile, 16, 1024);
+            const uint64_t dk0 = umma_smem_desc(sKa, 16, 1024);
+            const uint64_t dk1 = umma_smem_desc(sKa + Lay::kKTile, 16, 1024);
+            const uint64_t dv0 = umma_smem_desc(sVa, Lay::kKPanel, 1024);
+            const uint64_t dv1 = umma_smem_desc(sVa + Lay::kKTile, Lay::kKPanel, 1024);
+            // S_k = Q_k K_st^T : K-major A and B, 16 elements of d per instruction
             auto issue_s = [&](int k, int st) {
+                const uint32_t ts = tmem + (k ? Lay::kColS1 : Lay::kColS0);
+                const uint64_t a = k ? dq1 : dq0, bk = st ? dk1 : dk0;
+                if (leader) {
 #pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint32_t off = (kk >> 2) * Lay::kQPanel + (kk & 3) * 32;
-                    const uint64_t ad = umma_smem_desc(sQa + k * Lay::kQTile + off, 16, 1024);
-                    const uint64_t bd = umma_smem_desc(sKa + st * Lay::kKTile + off, 16, 1024);
-                    umma_ss(tmem + (k ? Lay::kColS1 : Lay::kColS0), ad, bd, idesc_s, kk > 0);
+                    for (int kk = 0; kk < D / 16; ++kk) {
+                        const uint32_t off = ((kk >> 2) * Lay::kQPanel + (kk & 3) * 32) >> 4;
+                        umma_ss(ts, a + off, bk + off, idesc_s, kk > 0);
+                    }
                 }
+                __syncwarp();
             };
             // O_k (+)= P_k V_st : P from tensor memory, V MN-major (d contiguous)
             auto issue_pv = [&](int k, int st, bool acc) {
+                const uint32_t ts = tmem + (k ? Lay::kColS1 : Lay::kColS0);
+                const uint32_t to = tmem + (k ? Lay::kColO1 : Lay::kColO0);
+                const uint64_t bv = st ? dv1 : dv0;
+                if (leader) {
 #pragma unroll
-                for (int kk = 0; kk < kPfBN / 16; ++kk) {
-                    const uint64_t bd = umma_smem_desc(sVa + st * Lay::kKTile + kk * 2048,
-                                                       Lay::kKPanel, 1024);
-                    umma_ts(tmem + (k ? Lay::kColO1 : Lay::kColO0),
-                            tmem + (k ? Lay::kColS1 : Lay::kColS0) + kk * 8, bd, idesc_o,
-                            (acc || kk > 0) ? 1u : 0u);
+                    for (int kk = 0; kk < kPfBN / 16; ++kk)
+                        umma_ts(to, ts + kk * 8, bv + kk * (2048 >> 4), idesc_o,
+                                (acc || kk > 0) ? 1u : 0u);
                 }
+                __syncwarp();
+            };
+            auto commit = [&](uint64_t *bar) {
+                if (leader) tc_commit(bar);
+                __syncwarp();
+            };
+            auto wait_all = [&](uint64_t *bar, uint32_t parity) {
+                return __all_sync(0xffffffffu, mbar_wait(bar, parity, &abort_flag, p.status));
             };
             for (int j = 0; ok && j < n_kv; ++j) {
                 const int st = j % kPfStages;
                 const uint32_t ph = (j / kPfStages) & 1;
                 const int sp = (j + kPfStages - 1) % kPfStages;          // stage of tile j-1
                 const uint32_t php = ((j - 1) / kPfStages) & 1;
-                if (!(ok = mbar_wait(&k_full[st], ph, &abort_flag, p.status))) break;
+                if (!(ok = wait_all(&k_full[st], ph))) break;
                 tc_fence_after();
                 if (j > 0) {
-                    if (!(ok = mbar_wait(&v_full[sp], php, &abort_flag, p.status))) break;
-                    if (!(ok = mbar_wait(&p_full[0], (j - 1) & 1, &abort_flag, p.status))) break;
+                    if (!(ok = wait_all(&v_full[sp], php))) break;
+                    if (!(ok = wait_all(&p_full[0], (j - 1) & 1))) break;
                     tc_fence_after();
                     issue_pv(0, sp, j > 1);
                 }
                 issue_s(0, st);
-                tc_commit(&s_full[0]);
+                commit(&s_full[0]);
                 if (j > 0) {
-                    if (!(ok = mbar_wait(&p_full[1], (j - 1) & 1, &abort_flag, p.status))) break;
+                    if (!(ok = wait_all(&p_full[1], (j - 1) & 1))) break;
                     tc_fence_after();
                     issue_pv(1, sp, j > 1);
-                    tc_commit(&v_empty[sp]);
+                    commit(&v_empty[sp]);
                 }
                 issue_s(1, st);
-                tc_commit(&s_full[1]);
-                tc_commit(&k_empty[st]);
+                commit(&s_full[1]);
+                commit(&k_empty[st]);
             }
             if (ok) {
                 const int sl = (n_kv - 1) % kPfStages;
                 const uint32_t phl = ((n_kv - 1) / kPfStages) & 1;
-                ok = mbar_wait(&v_full[sl], phl, &abort_flag, p.status) &&
-                     mbar_wait(&p_full[0], (n_kv - 1) & 1, &abort_flag, p.status);
+                ok = wait_all(&v_full[sl], phl) && wait_all(&p_full[0], (n_kv - 1) & 1);
                 if (ok) {
                     tc_fence_after();
                     issue_pv(0, sl, n_kv > 1);
-                    tc_commit(&o_done[0]);
-                    ok = mbar_wait(&p_full[1], (n_kv - 1) & 1, &abort_flag, p.status);
+                    commit(&o_done[0]);
+                    ok = wait_all(&p_full[1], (n_kv - 1) & 1);
                 }
                 if (ok) {
                     tc_fence_after();
                     issue_pv(1, sl, n_kv > 1);
-                    tc_commit(&o_done[1]);
-                    tc_commit(&v_empty[sl]);
+                    commit(&o_done[1]);
+                    commit(&v_empty[sl]);
                 }
             }
-            // every MMA this thread issued has finished before tensor memory is freed
-            tc_commit(&mma_drain);
+            // every MMA this warp issued has finished before tensor memory is freed
+            commit(&mma_drain);
             mbar_wait(&mma_drain, 0, &abort_flag, p.status, 1000000000ull);
         }
     } else if (warp >= 4) {
         // -------------------------------------------- softmax + epilogue ----
-        const int k = (warp - 4) >> 2;                  // M tile of this warpgroup
-        const int r = ((warp & 3) << 5) + lane;         // row = tensor-memory lane
-        const uint32_t lane_addr = tmem + ((static_cast<uint32_t>(warp & 3) * 32u) << 16);
-        const uint32_t colS = k ? Lay::kColS1 : Lay::kColS0;
-        const uint32_t colO = k ? Lay::kColO1 : Lay::kColO0;
+        // Two threads per row: warps 4-11 serve M tile 0, warps 12-19 M tile 1;
+        // within a tile, half h = 0 owns S/O columns 0-63 and h = 1 columns
+        // 64-127 of the 32 rows of tensor-memory lane group (warp % 4).
+        const int k = (warp - 4) >> 3;                  // M tile
+        const int h = ((warp - 4) >> 2) & 1;            // column half
+        const int g4 = warp & 3;                        // lane group = SM sub-partition
+        const int r = (g4 << 5) + lane;                 // row = tensor-memory lane
+        const uint32_t lane_addr = tmem + ((static_cast<uint32_t>(g4) * 32u) << 16);
+        const uint32_t colS = (k ? Lay::kColS1 : Lay::kColS0) + 64u * h;
+        const uint32_t colP = (k ? Lay::kColS1 : Lay::kColS0) + 32u * h;
+        const uint32_t colO = (k ? Lay::kColO1 : Lay::kColO0) + (D / 2) * h;
+        const int bar_id = 1 + k * 4 + g4;              // the two warps sharing these rows
+        // Publish a value for my row and take the other half's.  Both warps of
+        // the pair reach every exchange (the loop's continue / abort decision is
+        // taken jointly from the exchanged values), so the hardware barrier
+        // always completes.  Slots alternate by phase so a fast warp cannot
+        // overwrite a value its partner has not read yet.
+        auto exchange = [&](float mine, uint32_t ph, float &other) {
+            xchg[ph][k][h][r] = mine;
+            named_barrier_sync(bar_id, 64);
+            other = xchg[ph][k][h ^ 1][r];
+        };
         const int pos = t0 + k * p.P + r / p.G;
         const int head = kvh * p.G + r % p.G;
         const bool row_real = (r < p.P * p.G) && (pos < p.Tq);
         // last visible key of this row (keys past Tkv never count)
         int lim = p.Tkv - 1;
         if (p.causal && row_real) lim = min(lim, pos + (p.Tkv - p.Tq));
-        float m_run = -INFINITY, l_run = 0.0f;
+        // Online softmax with a lazily moved reference max: O and l stay scaled
+        // by exp2(-m_ref) and m_ref only moves when a row's max exceeds it by
+        // more than kRescaleLog2 (P then stays <= 2^kRescaleLog2).  Exact in
+        // real arithmetic: the epilogue divides by l taken at the same m_ref.
+        // Both halves of a row see the same row max, so they take identical
+        // m_ref / alpha decisions; each keeps the partial l of its columns.
+        float m_ref = -INFINITY, l_run = 0.0f;
+        const float c2 = p.scale_log2;
         bool ok = true;
         for (int j = 0; j < n_kv; ++j) {
             // warp-uniform outcome: the tensor-memory accesses below are .sync.aligned
             ok = __all_sync(0xffffffffu, mbar_wait(&s_full[k], j & 1, &abort_flag, p.status));
-            if (!ok) break;
+            if (!ok) {
+                float dummy;
+                exchange(__int_as_float(0x7fc00001), j & 1, dummy);   // tell the partner
+                break;
+            }
             tc_fence_after();
-            uint32_t sr[4][32];
-#pragma unroll
-            for (int c = 0; c < 4; ++c) tmem_ld32(lane_addr + colS + 32 * c, sr[c]);
+            uint32_t sr[2][32];
+            tmem_ld32(lane_addr + colS, sr[0]);
+            tmem_ld32(lane_addr + colS + 32, sr[1]);
             tmem_wait_ld();
-            const int cut = lim - j * kPfBN;            // columns > cut are masked
-            float mx = -INFINITY;
-            if (__any_sync(0xffffffffu, cut < kPfBN - 1)) {
+            const int cut = lim - j * kPfBN - 64 * h;   // my columns > cut are masked
+            const bool masked = __any_sync(0xffffffffu, cut < 63);
+            if (masked) {
 #pragma unroll
-                for (int c = 0; c < 4; ++c)
+                for (int c = 0; c < 2; ++c)
 #pragma unroll
-                    for (int e = 0; e < 32; ++e) {
-                        float x = __uint_as_float(sr[c][e]) * p.scale_log2;
-                        x = (32 * c + e <= cut) ? x : -INFINITY;
-                        sr[c][e] = __float_as_uint(x);
-                        mx = fmaxf(mx, x);
-                    }
+                    for (int e = 0; e < 32; ++e)
+                        if (32 * c + e > cut) sr[c][e] = __float_as_uint(-INFINITY);
+            }
+            // row max of the raw scores (scale > 0 keeps the order), then the
+            // other half's max through shared memory
+            float mx4[4];
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {                // 4 independent chains of 16 scores
+                const uint32_t *v = &sr[c >> 1][(c & 1) * 16];
+                float m = __uint_as_float(v[0]);
+#pragma unroll
+                for (int e = 1; e < 15; e += 2)
+                    m = max3f(m, __uint_as_float(v[e]), __uint_as_float(v[e + 1]));
+                mx4[c] = fmaxf(m, __uint_as_float(v[15]));
+            }
+            float mx2[2] = {fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3])};
+            const float mx_mine = fmaxf(mx2[0], mx2[1]);
+            float mx_other;
+            tc_fence_before();                          // my S loads precede the other half's P stores
+            exchange(mx_mine, j & 1, mx_other);
+            tc_fence_after();
+            // the partner's abort marker (a NaN payload no max can produce)
+            if (__any_sync(0xffffffffu, __float_as_int(mx_other) == 0x7fc00001)) {
+                ok = false;
+                break;
+            }
+            const float mxs = fmaxf(mx_mine, mx_other) * c2;
+            const bool move = mxs > m_ref + kRescaleLog2;  // always true on the first key seen
+            float alpha = 1.0f;
+            if (move) {
+                alpha = fast_exp2(m_ref - mxs);         // 0 when nothing was seen before
+                m_ref = mxs;
+            }
+            const float m_use = (m_ref == -INFINITY) ? 0.0f : m_ref;
+            const float2 cc = make_float2(c2, c2), nm = make_float2(-m_use, -m_use);
+            float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+            // P = exp2(s * scale * log2e - m_ref), truncated to bf16; P overwrites
+            // the first 64 columns of S (this half: packed columns 32h..32h+31).
+            // l sums exactly the bf16 weights the PV product uses, so O / l is
+            // a convex combination of V rows.  Tiles with masked (-inf) scores
+            // use the MUFU exp only; full tiles send part of the pairs to the
+            // FMA-pipe polynomial.
+            if (masked) {
+#pragma unroll
+                for (int c = 0; c < 2; ++c) {
+                    uint32_t pk[16];
+                    softmax_chunk<false>(sr[c], cc, nm, pk, acc);
+                    tmem_st16(lane_addr + colP + 16 * c, pk);
+                }
             } else {
 #pragma unroll
-                for (int c = 0; c < 4; ++c)
-#pragma unroll
-                    for (int e = 0; e < 32; ++e) {
-                        const float x = __uint_as_float(sr[c][e]) * p.scale_log2;
-                        sr[c][e] = __float_as_uint(x);
-                        mx = fmaxf(mx, x);
-                    }
+                for (int c = 0; c < 2; ++c) {
+                    uint32_t pk[16];
+                    softmax_chunk<true>(sr[c], cc, nm, pk, acc);
+                    tmem_st16(lane_addr + colP + 16 * c, pk);
+                }
             }
-            const float m_new = fmaxf(m_run, mx);
-            const float m_use = (m_new == -INFINITY) ? 0.0f : m_new;
-            const float alpha = fast_exp2(m_run - m_use);   // 0 while nothing was seen
-            // O holds tiles < j scaled by exp2(-m_run); bring it to m_new
-            if (j > 0 && __any_sync(0xffffffffu, m_new > m_run)) {
+            l_run = l_run * alpha + ((acc[0] + acc[1]) + (acc[2] + acc[3]));
+            // O holds tiles < j at the old reference: rescale rows whose reference moved
+            if (j > 0 && __any_sync(0xffffffffu, move)) {
+                const float2 a2 = make_float2(alpha, alpha);
 #pragma unroll
-                for (int c = 0; c < D / 32; ++c) {
+                for (int c = 0; c < D / 64; ++c) {
                     uint32_t orr[32];
                     tmem_ld32(lane_addr + colO + 32 * c, orr);
                     tmem_wait_ld();
 #pragma unroll
-                    for (int e = 0; e < 32; ++e)
-                        orr[e] = __float_as_uint(__uint_as_float(orr[e]) * alpha);
+                    for (int e = 0; e < 32; e += 2) {
+                        const float2 v2 = mul2(make_float2(__uint_as_float(orr[e]),
+                                                           __uint_as_float(orr[e + 1])), a2);
+                        orr[e] = __float_as_uint(v2.x);
+                        orr[e + 1] = __float_as_uint(v2.y);
+                    }
                     tmem_st32(lane_addr + colO + 32 * c, orr);
                 }
             }
-            m_run = m_new;
-            float psum = 0.0f;
-            uint32_t pp[2][32];
-#pragma unroll
-            for (int c = 0; c < 4; ++c)
-#pragma unroll
-                for (int e = 0; e < 32; e += 2) {
-                    const float a = fast_exp2(__uint_as_float(sr[c][e]) - m_use);
-                    const float bb = fast_exp2(__uint_as_float(sr[c][e + 1]) - m_use);
-                    psum += a + bb;
-                    pp[c >> 1][(c & 1) * 16 + (e >> 1)] = pack_bf16x2(a, bb);
-                }
-            l_run = l_run * alpha + psum;
-            tmem_st32(lane_addr + colS, pp[0]);
-            tmem_st32(lane_addr + colS + 32, pp[1]);
             tmem_wait_st();
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&p_full[k]);
         }
-        // ---- epilogue: O / l -> bf16, lse ----
+        // ---- epilogue: O / l -> bf16, lse (each half writes its d/2 columns) ----
+        float l_other = 0.0f;
+        if (ok) exchange(l_run, n_kv & 1, l_other);
+        const float l_row = l_run + l_other;
         if (ok && n_kv > 0)
             ok = __all_sync(0xffffffffu, mbar_wait(&o_done[k], 0, &abort_flag, p.status));
         tc_fence_after();
-        const float inv_l = (l_run > 0.0f) ? 1.0f / l_run : 0.0f;
+        const float inv_l = (l_row > 0.0f) ? 1.0f / l_row : 0.0f;
         __nv_bfloat16 *dst =
-            p.o + ((static_cast<size_t>(b) * p.Tq + pos) * p.Hq + head) * D;
+            p.o + ((static_cast<size_t>(b) * p.Tq + pos) * p.Hq + head) * D + (D / 2) * h;
 #pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
+        for (int c = 0; c < D / 64; ++c) {
             uint32_t orr[32];
             if (ok && n_kv > 0) {
                 tmem_ld32(lane_addr + colO + 32 * c, orr);
@@ -346,9 +469,9 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                     d4[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
             }
         }
-        if (p.lse && row_real)
+        if (p.lse && row_real && h == 0)
             p.lse[(static_cast<size_t>(b) * p.Hq + head) * p.Tq + pos] =
-                (l_run > 0.0f) ? (m_run + __log2f(l_run)) * 0.69314718055994531f : -INFINITY;
+                (l_row > 0.0f) ? (m_ref + __log2f(l_row)) * 0.69314718055994531f : -INFINITY;
     }
 
     tc_fence_before();
