@@ -26,17 +26,26 @@ namespace gqa {
 constexpr int kDecBK = 64;                         // keys per pipeline stage
 constexpr int kDecWarps = 4;                       // consumer warps, 16 keys each per stage
 constexpr int kDecThreads = (kDecWarps + 1) * 32;  // + one producer warp
-constexpr int kDecStages = 3;
-constexpr int kDecChunk = 512;                     // keys per split
+#ifndef GQA_DEC_STAGES
+#define GQA_DEC_STAGES 2
+#endif
+#ifndef GQA_DEC_CHUNK
+#define GQA_DEC_CHUNK 1024
+#endif
+constexpr int kDecStages = GQA_DEC_STAGES;         // TMA ring depth
+constexpr int kDecChunk = GQA_DEC_CHUNK;           // keys per split (multiple of kDecBK)
 
-template <int D>
+template <int D, int MB = 1>
 struct DecLayout {
     static constexpr int kPanels = D / 64;                 // 64 bf16 = one 128-byte row
     static constexpr int kPanelBytes = kDecBK * 128;
     static constexpr int kTileBytes = kPanels * kPanelBytes;
     static constexpr int kStageBytes = 2 * kTileBytes;     // K tile then V tile
     static constexpr int kRingBytes = kDecStages * kStageBytes;
-    static constexpr int kSmemBytes = kRingBytes + 1024;   // + alignment slack
+    // the end-of-split merge reuses the ring: per warp 16*MB rows of O, m and l
+    static constexpr int kMergeBytes = kDecWarps * 16 * MB * (D + 2) * 4;
+    static constexpr int kBytes = kRingBytes > kMergeBytes ? kRingBytes : kMergeBytes;
+    static constexpr int kSmemBytes = kBytes + 1024;       // + alignment slack
 };
 
 __device__ __forceinline__ uint32_t ld_b32(const __nv_bfloat16 *p) {
@@ -57,13 +66,15 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tm_k,
                     const __nv_bfloat16 *__restrict__ q, const int32_t *__restrict__ seqlens,
                     float *__restrict__ part_o, float *__restrict__ part_lse, int B, int Hq,
                     int Hkv, int Lmax, int chunk, float scale_log2, int *status) {
-    using Lay = DecLayout<D>;
+    using Lay = DecLayout<D, MB>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
     __shared__ uint64_t full_bar[kDecStages], empty_bar[kDecStages];
     __shared__ int abort_flag;
 
+    // the combine grid may be scheduled now; it waits for this grid's results
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     const int split = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z;
     int L = seqlens[b];
     if (L > Lmax || L < 0) {
@@ -296,6 +307,9 @@ decode_combine_kernel(const float *__restrict__ part_o, const float *__restrict_
                       const int32_t *__restrict__ seqlens, __nv_bfloat16 *__restrict__ o, int B,
                       int Hq, int Lmax, int chunk) {
     constexpr int kPer = D / 32;
+    // launched as a programmatic dependent of the split kernel: wait until all of
+    // its memory operations are complete and visible
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     const int row = blockIdx.x * 4 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
     if (row >= B * Hq) return;
     const int b = row / Hq;
@@ -344,7 +358,7 @@ static int launch_split(const CUtensorMap &tk, const CUtensorMap &tv, const void
                         int Hkv, int Lmax, int chunk, float scale_log2, int *status,
                         cudaStream_t stream) {
     auto kern = decode_split_kernel<D, MB>;
-    const int smem = DecLayout<D>::kSmemBytes;
+    const int smem = DecLayout<D, MB>::kSmemBytes;
     if (int rc = check_cuda(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                                  smem), "cudaFuncSetAttribute(decode)"))
         return rc;
@@ -387,13 +401,24 @@ int launch_decode(const void *q, const void *k_cache, const void *v_cache,
                                                Lmax, chunk, scale_log2, status, stream);
         if (rc) return rc;
     }
-    const int blocks = (B * Hq + 3) / 4;
-    if (d == 128)
-        decode_combine_kernel<128><<<blocks, 128, 0, stream>>>(
-            part_o, part_lse, seqlens, static_cast<__nv_bfloat16 *>(o), B, Hq, Lmax, chunk);
-    else
-        decode_combine_kernel<64><<<blocks, 128, 0, stream>>>(
-            part_o, part_lse, seqlens, static_cast<__nv_bfloat16 *>(o), B, Hq, Lmax, chunk);
+    // The combine kernel is a programmatic dependent launch: it is scheduled
+    // while the split kernel drains and waits (griddepcontrol.wait) for its results.
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((B * Hq + 3) / 4);
+    cfg.blockDim = dim3(128);
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    __nv_bfloat16 *ob = static_cast<__nv_bfloat16 *>(o);
+    const cudaError_t e =
+        d == 128 ? cudaLaunchKernelEx(&cfg, decode_combine_kernel<128>, (const float *)part_o,
+                                      (const float *)part_lse, seqlens, ob, B, Hq, Lmax, chunk)
+                 : cudaLaunchKernelEx(&cfg, decode_combine_kernel<64>, (const float *)part_o,
+                                      (const float *)part_lse, seqlens, ob, B, Hq, Lmax, chunk);
+    if (int rc = check_cuda(e, "decode_combine_kernel launch")) return rc;
     return check_cuda(cudaGetLastError(), "decode_combine_kernel launch");
 }
 
