@@ -33,16 +33,18 @@
 static long kv_head_of(long hq, long Hq, long Hkv) { return hq / (Hq / Hkv); }
 
 /*
- * One query row against n_keys keys.  Keys j with masked[j] (j >= n_vis when
- * the causal mask hides the tail) get score -inf before the softmax.
+ * One query row against n_keys keys.  Key j is visible when j < n_vis (the
+ * causal limit) and, with a sliding window, when j >= lo or j < sinks (the
+ * window's first key and the always-visible sink keys); hidden keys get score
+ * -inf before the softmax.  lo = 0, sinks = 0 means no window.
  */
-static void attend_row(const float *qrow, const float *k0, const float *v0,
-                       long key_stride, long n_keys, long n_vis, long d,
-                       double scale, double *s, double *orow, double *lse)
+static void attend_row_win(const float *qrow, const float *k0, const float *v0,
+                           long key_stride, long n_keys, long n_vis, long lo, long sinks,
+                           long d, double scale, double *s, double *orow, double *lse)
 {
     double m = -INFINITY;
     for (long j = 0; j < n_keys; ++j) {
-        if (j >= n_vis) { s[j] = -INFINITY; continue; }
+        if (j >= n_vis || (j < lo && j >= sinks)) { s[j] = -INFINITY; continue; }
         const float *kj = k0 + j * key_stride;
         double dot = 0.0;
         for (long c = 0; c < d; ++c) dot += (double)qrow[c] * (double)kj[c];
@@ -61,6 +63,13 @@ static void attend_row(const float *qrow, const float *k0, const float *v0,
     }
     for (long c = 0; c < d; ++c) orow[c] /= l;
     *lse = m + log(l);
+}
+
+static void attend_row(const float *qrow, const float *k0, const float *v0,
+                       long key_stride, long n_keys, long n_vis, long d,
+                       double scale, double *s, double *orow, double *lse)
+{
+    attend_row_win(qrow, k0, v0, key_stride, n_keys, n_vis, 0, 0, d, scale, s, orow, lse);
 }
 
 static int check_shape(long B, long Tq, long Tkv, long Hq, long Hkv, long d)
@@ -249,6 +258,72 @@ int oracle_decode_split(const float *q, const float *kc, const float *vc,
             if (lse) lse[r] = M + log(wsum);
         }
         free(part);
+        free(s);
+    }
+    return 0;
+}
+
+/*
+ * Causal forward with a sliding window of `window` keys (window >= 1) and
+ * `sinks` always-visible leading keys: row i (key position p = i + Tkv - Tq)
+ * sees key j iff j <= p and (j > p - window or j < sinks).  Course "Неделя 7.
+ * Внимание", step 3 ("Sliding window, attention sinks").  Layouts as
+ * oracle_attn_fwd.
+ */
+int oracle_attn_fwd_window(const float *q, const float *k, const float *v,
+                           double *o, double *lse,
+                           long B, long Tq, long Tkv, long Hq, long Hkv, long d,
+                           long window, long sinks, double scale, int nthreads)
+{
+    if (check_shape(B, Tq, Tkv, Hq, Hkv, d) || window < 1 || sinks < 0) return 1;
+    set_threads(nthreads);
+    long n_rows = B * Hq * Tq;
+    #pragma omp parallel
+    {
+        double *s = (double *)malloc(sizeof(double) * (size_t)(Tkv > 0 ? Tkv : 1));
+        #pragma omp for schedule(dynamic, 8)
+        for (long r = 0; r < n_rows; ++r) {
+            long i = r % Tq, bh = r / Tq, hq = bh % Hq, b = bh / Hq;
+            long kvh = kv_head_of(hq, Hq, Hkv);
+            long p = i + (Tkv - Tq);
+            double l_row;
+            attend_row_win(q + ((b * Tq + i) * Hq + hq) * d,
+                           k + (b * Tkv * Hkv + kvh) * d, v + (b * Tkv * Hkv + kvh) * d,
+                           Hkv * d, Tkv, visible_keys(i, Tq, Tkv, 1), p - window + 1, sinks,
+                           d, scale, s, o + ((b * Tq + i) * Hq + hq) * d, &l_row);
+            if (lse) lse[(b * Hq + hq) * Tq + i] = l_row;
+        }
+        free(s);
+    }
+    return 0;
+}
+
+/*
+ * Decode with a sliding window: the newest token of sequence b (position
+ * L - 1, L = seqlens[b]) sees cache rows j >= L - window plus rows j < sinks.
+ */
+int oracle_decode_window(const float *q, const float *kc, const float *vc,
+                         const int32_t *seqlens, double *o, double *lse,
+                         long B, long Hq, long Hkv, long d, long Lmax,
+                         long window, long sinks, double scale, int nthreads)
+{
+    if (check_shape(B, 1, Lmax, Hq, Hkv, d) || window < 1 || sinks < 0) return 1;
+    for (long b = 0; b < B; ++b)
+        if (seqlens[b] < 0 || seqlens[b] > Lmax) return 1;
+    set_threads(nthreads);
+    #pragma omp parallel
+    {
+        double *s = (double *)malloc(sizeof(double) * (size_t)(Lmax > 0 ? Lmax : 1));
+        #pragma omp for schedule(dynamic, 1)
+        for (long r = 0; r < B * Hq; ++r) {
+            long hq = r % Hq, b = r / Hq, kvh = kv_head_of(hq, Hq, Hkv);
+            long L = seqlens[b];
+            double l_row;
+            attend_row_win(q + r * d, kc + (b * Lmax * Hkv + kvh) * d,
+                           vc + (b * Lmax * Hkv + kvh) * d, Hkv * d, L, L, L - window, sinks,
+                           d, scale, s, o + r * d, &l_row);
+            if (lse) lse[r] = l_row;
+        }
         free(s);
     }
     return 0;

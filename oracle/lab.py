@@ -123,7 +123,7 @@ def expand_kv(folded, h):
     return out
 
 
-def attend(q, k, v, causal=False, scale=None):
+def attend(q, k, v, causal=False, scale=None, window=0, sinks=0):
     """Single-head attention of a query table against key/value tables.
 
     Lab step 4 ("1ヘッドのアテンションを作る"): for every query row, dot with every
@@ -136,8 +136,13 @@ def attend(q, k, v, causal=False, scale=None):
     bottom-right alignment, i.e. j > i when the lengths agree) and its score is
     -inf before the softmax.  A row with no visible key returns zeros.
     ``scale`` overrides 1/sqrt(head dim) (the same number when left as None).
+
+    ``window`` > 0 (with ``causal``) adds the sliding window of the course's
+    step 3 ("Sliding window, attention sinks"): query row i, at key position
+    p = i + (len(k) - len(q)), sees key j only if j > p - window; the first
+    ``sinks`` keys stay visible to every row that may see them (j <= p).
     """
-    probs = attention_probs(q, k, causal=causal, scale=scale)
+    probs = attention_probs(q, k, causal=causal, scale=scale, window=window, sinks=sinks)
     dim_v = len(v[0])
     out = []
     for p_row in probs:
@@ -151,7 +156,17 @@ def attend(q, k, v, causal=False, scale=None):
     return out
 
 
-def attention_probs(q, k, causal=False, scale=None):
+def visible(i, j, tq, tk, causal=False, window=0, sinks=0):
+    """Whether query row i may see key j (mask applied before the softmax)."""
+    p = i + (tk - tq)                       # the row's position among the keys
+    if causal and j > p:
+        return False
+    if window > 0 and j <= p - window and j >= sinks:
+        return False
+    return True
+
+
+def attention_probs(q, k, causal=False, scale=None, window=0, sinks=0):
     """The softmax weights ``attend`` uses: one row per query, one column per key."""
     dim = len(q[0])
     if scale is None:
@@ -161,7 +176,7 @@ def attention_probs(q, k, causal=False, scale=None):
     for i in range(tq):
         scores = []
         for j in range(tk):
-            if causal and j > i + (tk - tq):
+            if not visible(i, j, tq, tk, causal, window, sinks):
                 scores.append(-math.inf)
                 continue
             dot = 0.0

@@ -53,8 +53,13 @@ def _load():
                                   L, L, L, L, L, ctypes.c_double, ctypes.c_int]
     lib.oracle_decode_split.argtypes = [fp, fp, fp, ctypes.POINTER(ctypes.c_int32), dp, dp,
                                         L, L, L, L, L, ctypes.c_double, L, ctypes.c_int]
+    lib.oracle_attn_fwd_window.argtypes = [fp, fp, fp, dp, dp, L, L, L, L, L, L, L, L,
+                                           ctypes.c_double, ctypes.c_int]
+    lib.oracle_decode_window.argtypes = [fp, fp, fp, ctypes.POINTER(ctypes.c_int32), dp, dp,
+                                         L, L, L, L, L, L, L, ctypes.c_double, ctypes.c_int]
     for f in (lib.oracle_attn_fwd, lib.oracle_attn_fwd_rows, lib.oracle_decode,
-              lib.oracle_decode_split, lib.oracle_num_threads):
+              lib.oracle_decode_split, lib.oracle_num_threads, lib.oracle_attn_fwd_window,
+              lib.oracle_decode_window):
         f.restype = ctypes.c_int
     _lib = lib
     return lib
@@ -95,6 +100,42 @@ def attn_fwd(q, k, v, causal, scale=None, threads=0):
                                  int(bool(causal)), _default_scale(d, scale), threads)
     if rc != 0:
         raise ValueError("invalid shape for the oracle (Hq must be a multiple of Hkv)")
+    return o, lse
+
+
+def attn_fwd_window(q, k, v, window, sinks=0, scale=None, threads=0):
+    """Causal forward with a sliding window and sink keys -> (o, lse) as attn_fwd."""
+    q, k, v = _f32(q), _f32(k), _f32(v)
+    B, Tq, Hq, d = q.shape
+    _, Tkv, Hkv, _ = k.shape
+    o = np.empty((B, Tq, Hq, d), np.float64)
+    lse = np.empty((B, Hq, Tq), np.float64)
+    rc = _load().oracle_attn_fwd_window(_ptr(q, ctypes.c_float), _ptr(k, ctypes.c_float),
+                                        _ptr(v, ctypes.c_float), _ptr(o, ctypes.c_double),
+                                        _ptr(lse, ctypes.c_double), B, Tq, Tkv, Hq, Hkv, d,
+                                        int(window), int(sinks), _default_scale(d, scale), threads)
+    if rc != 0:
+        raise ValueError("invalid shape, window or sinks for the oracle")
+    return o, lse
+
+
+def decode_window(q, k_cache, v_cache, seqlens, window, sinks=0, scale=None, threads=0):
+    """Decode with a sliding window and sink keys -> (o [B,Hq,d], lse [B,Hq])."""
+    q, kc, vc = _f32(q), _f32(k_cache), _f32(v_cache)
+    if hasattr(seqlens, "detach"):
+        seqlens = seqlens.detach().cpu().numpy()
+    sl = np.ascontiguousarray(np.asarray(seqlens, dtype=np.int32))
+    B, Hq, d = q.shape
+    _, Lmax, Hkv, _ = kc.shape
+    o = np.empty((B, Hq, d), np.float64)
+    lse = np.empty((B, Hq), np.float64)
+    rc = _load().oracle_decode_window(_ptr(q, ctypes.c_float), _ptr(kc, ctypes.c_float),
+                                      _ptr(vc, ctypes.c_float), _ptr(sl, ctypes.c_int32),
+                                      _ptr(o, ctypes.c_double), _ptr(lse, ctypes.c_double),
+                                      B, Hq, Hkv, d, Lmax, int(window), int(sinks),
+                                      _default_scale(d, scale), threads)
+    if rc != 0:
+        raise ValueError("invalid shape, length, window or sinks for the oracle")
     return o, lse
 
 
