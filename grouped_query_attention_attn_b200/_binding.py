@@ -28,9 +28,12 @@ _F = ctypes.c_float
 _SIGNATURES = {
     "gqa_attn_fwd": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _P]),
     "gqa_attn_fwd_lse": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _P]),
+    "gqa_attn_fwd_window": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _F, _P]),
     "gqa_attn_fwd_f32": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _P]),
     "gqa_decode_workspace_size": (ctypes.c_size_t, [_I, _I, _I, _I, _I]),
     "gqa_decode": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _P, ctypes.c_size_t, _P]),
+    "gqa_decode_window": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _P,
+                               ctypes.c_size_t, _P]),
     "gqa_decode_static": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _P]),
     "gqa_fold_kv": (_I, [_P, _P, _I, _I, _I, _I, _I, _P]),
     "gqa_last_error": (ctypes.c_char_p, []),
@@ -63,6 +66,11 @@ def gqa_attn_fwd_lse(q, k, v, o, lse, B, Tq, Tkv, Hq, Hkv, d, causal, scale, str
     return lib().gqa_attn_fwd_lse(q, k, v, o, lse, B, Tq, Tkv, Hq, Hkv, d, causal, scale, stream)
 
 
+def gqa_attn_fwd_window(q, k, v, o, lse, B, Tq, Tkv, Hq, Hkv, d, window, sinks, scale, stream):
+    return lib().gqa_attn_fwd_window(q, k, v, o, lse, B, Tq, Tkv, Hq, Hkv, d, window, sinks,
+                                     scale, stream)
+
+
 def gqa_attn_fwd_f32(q, k, v, o, lse, B, Tq, Tkv, Hq, Hkv, d, causal, scale, stream):
     return lib().gqa_attn_fwd_f32(q, k, v, o, lse, B, Tq, Tkv, Hq, Hkv, d, causal, scale, stream)
 
@@ -75,6 +83,12 @@ def gqa_decode(q, k_cache, v_cache, seqlens, o, B, Hq, Hkv, d, Lmax, scale, work
                workspace_bytes, stream):
     return lib().gqa_decode(q, k_cache, v_cache, seqlens, o, B, Hq, Hkv, d, Lmax, scale,
                             workspace, workspace_bytes, stream)
+
+
+def gqa_decode_window(q, k_cache, v_cache, seqlens, o, B, Hq, Hkv, d, Lmax, window, sinks, scale,
+                      workspace, workspace_bytes, stream):
+    return lib().gqa_decode_window(q, k_cache, v_cache, seqlens, o, B, Hq, Hkv, d, Lmax, window,
+                                   sinks, scale, workspace, workspace_bytes, stream)
 
 
 def gqa_decode_static(q, k_cache, v_cache, seqlens, o, B, Hq, Hkv, d, Lmax, scale, stream):

@@ -49,12 +49,14 @@ def _shapes(q, k, v):
     return B, Tq, Tkv, Hq, Hkv, d
 
 
-def attn(q, k, v, causal=True, scale=None, out=None, return_lse=False):
+def attn(q, k, v, causal=True, scale=None, out=None, return_lse=False, window=None, sinks=0):
     """Grouped-query attention forward, bf16.
 
     q [B, Tq, Hq, d], k/v [B, Tkv, Hkv, d] (bf16, contiguous, on one GPU);
     query head h reads K/V head h // (Hq // Hkv).  Returns o [B, Tq, Hq, d]
-    (and lse [B, Hq, Tq] fp32 when ``return_lse``).
+    (and lse [B, Hq, Tq] fp32 when ``return_lse``).  ``window`` (an int >= 1)
+    selects causal sliding-window attention with ``sinks`` always-visible
+    leading keys.
     """
     for t, n in ((q, "q"), (k, "k"), (v, "v")):
         _need(t, n, torch.bfloat16, 4)
@@ -63,9 +65,16 @@ def attn(q, k, v, causal=True, scale=None, out=None, return_lse=False):
     o = torch.empty_like(q) if out is None else out
     _need(o, "out", torch.bfloat16, 4)
     lse = torch.empty((B, Hq, Tq), dtype=torch.float32, device=q.device) if return_lse else None
-    rc = _b.gqa_attn_fwd_lse(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
-                             lse.data_ptr() if lse is not None else None,
-                             B, Tq, Tkv, Hq, Hkv, d, int(bool(causal)), scale, _stream(q))
+    lp = lse.data_ptr() if lse is not None else None
+    if window is None:
+        rc = _b.gqa_attn_fwd_lse(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lp,
+                                 B, Tq, Tkv, Hq, Hkv, d, int(bool(causal)), scale, _stream(q))
+    else:
+        if not causal:
+            raise ValueError("a sliding window needs causal=True")
+        rc = _b.gqa_attn_fwd_window(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lp,
+                                    B, Tq, Tkv, Hq, Hkv, d, int(window), int(sinks), scale,
+                                    _stream(q))
     _check(rc, "gqa_attn_fwd")
     return (o, lse) if return_lse else o
 
@@ -89,7 +98,8 @@ def decode_workspace_size(B, Hq, Hkv, d, Lmax):
     return int(_b.gqa_decode_workspace_size(B, Hq, Hkv, d, Lmax))
 
 
-def decode(q, k_cache, v_cache, seqlens, scale=None, workspace=None, out=None):
+def decode(q, k_cache, v_cache, seqlens, scale=None, workspace=None, out=None, window=None,
+           sinks=0):
     """One query token per sequence against a bf16 KV cache.
 
     q [B, Hq, d], caches [B, Lmax, Hkv, d], seqlens int32 [B] on the device.
@@ -109,9 +119,15 @@ def decode(q, k_cache, v_cache, seqlens, scale=None, workspace=None, out=None):
     if workspace is None:
         workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
     o = torch.empty_like(q) if out is None else out
-    rc = _b.gqa_decode(q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(), seqlens.data_ptr(),
-                       o.data_ptr(), B, Hq, Hkv, d, Lmax, scale, workspace.data_ptr(),
-                       workspace.numel(), _stream(q))
+    if window is None:
+        rc = _b.gqa_decode(q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(),
+                           seqlens.data_ptr(), o.data_ptr(), B, Hq, Hkv, d, Lmax, scale,
+                           workspace.data_ptr(), workspace.numel(), _stream(q))
+    else:
+        rc = _b.gqa_decode_window(q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(),
+                                  seqlens.data_ptr(), o.data_ptr(), B, Hq, Hkv, d, Lmax,
+                                  int(window), int(sinks), scale, workspace.data_ptr(),
+                                  workspace.numel(), _stream(q))
     _check(rc, "gqa_decode")
     return o
 

@@ -65,7 +65,8 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v,
                     const __nv_bfloat16 *__restrict__ q, const int32_t *__restrict__ seqlens,
                     float *__restrict__ part_o, float *__restrict__ part_lse, int B, int Hq,
-                    int Hkv, int Lmax, int chunk, float scale_log2, int *status) {
+                    int Hkv, int Lmax, int chunk, int window, int sinks, float scale_log2,
+                    int *status) {
     using Lay = DecLayout<D, MB>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
@@ -87,6 +88,18 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tm_k,
     const int n_stages = (end - start + kDecBK - 1) / kDecBK;
     const int G = Hq / Hkv;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    // Sliding window: key j is visible iff j >= lo or j < sinks (and j < L).
+    const int lo = window > 0 ? L - window : 0;
+    const int n_sinks = window > 0 ? sinks : 0;
+    if (end <= lo && start >= n_sinks) {
+        // no visible key in this split: an empty partial (weight 0 in the merge)
+        const size_t row0 = (static_cast<size_t>(split) * B + b) * Hq + static_cast<size_t>(kvh) * G;
+        for (int idx = threadIdx.x; idx < G * D; idx += blockDim.x) {
+            part_o[row0 * D + idx] = 0.0f;
+            if (idx % D == 0) part_lse[row0 + idx / D] = -INFINITY;
+        }
+        return;
+    }
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kDecStages; ++s) {
@@ -198,7 +211,9 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tm_k,
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
                         const int kl = nb * 8 + 2 * tq + (e & 1);
-                        s[nb][e] = kl < n_valid ? sacc[mb][nb][e] * scale_log2 : -INFINITY;
+                        const int key = key0 + kl;
+                        const bool vis = kl < n_valid && (key >= lo || key < n_sinks);
+                        s[nb][e] = vis ? sacc[mb][nb][e] * scale_log2 : -INFINITY;
                         mx[e >> 1] = fmaxf(mx[e >> 1], s[nb][e]);
                     }
                 float alpha[2], m_use[2];
@@ -355,8 +370,8 @@ size_t decode_workspace_bytes(int B, int Hq, int Hkv, int d, int Lmax) {
 template <int D, int MB>
 static int launch_split(const CUtensorMap &tk, const CUtensorMap &tv, const void *q,
                         const int32_t *seqlens, float *part_o, float *part_lse, int B, int Hq,
-                        int Hkv, int Lmax, int chunk, float scale_log2, int *status,
-                        cudaStream_t stream) {
+                        int Hkv, int Lmax, int chunk, int window, int sinks, float scale_log2,
+                        int *status, cudaStream_t stream) {
     auto kern = decode_split_kernel<D, MB>;
     const int smem = DecLayout<D, MB>::kSmemBytes;
     if (int rc = check_cuda(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -365,13 +380,13 @@ static int launch_split(const CUtensorMap &tk, const CUtensorMap &tv, const void
     dim3 grid((Lmax + chunk - 1) / chunk, Hkv, B);
     kern<<<grid, kDecThreads, smem, stream>>>(tk, tv, static_cast<const __nv_bfloat16 *>(q),
                                               seqlens, part_o, part_lse, B, Hq, Hkv, Lmax, chunk,
-                                              scale_log2, status);
+                                              window, sinks, scale_log2, status);
     return check_cuda(cudaGetLastError(), "decode_split_kernel launch");
 }
 
 int launch_decode(const void *q, const void *k_cache, const void *v_cache,
                   const int32_t *seqlens, void *o, int B, int Hq, int Hkv, int d, int Lmax,
-                  float scale, void *workspace, cudaStream_t stream) {
+                  int window, int sinks, float scale, void *workspace, cudaStream_t stream) {
     if (B > 65535 || Hkv > 65535)
         return set_error(GQA_ERR_UNSUPPORTED, "decode: B and Hkv must be <= 65535");
     int *status = device_status_ptr();
@@ -391,14 +406,14 @@ int launch_decode(const void *q, const void *k_cache, const void *v_cache,
         int rc;
         if (d == 128)
             rc = G <= 16 ? launch_split<128, 1>(tk, tv, q, seqlens, part_o, part_lse, B, Hq, Hkv,
-                                                Lmax, chunk, scale_log2, status, stream)
+                                                Lmax, chunk, window, sinks, scale_log2, status, stream)
                          : launch_split<128, 2>(tk, tv, q, seqlens, part_o, part_lse, B, Hq, Hkv,
-                                                Lmax, chunk, scale_log2, status, stream);
+                                                Lmax, chunk, window, sinks, scale_log2, status, stream);
         else
             rc = G <= 16 ? launch_split<64, 1>(tk, tv, q, seqlens, part_o, part_lse, B, Hq, Hkv,
-                                               Lmax, chunk, scale_log2, status, stream)
+                                               Lmax, chunk, window, sinks, scale_log2, status, stream)
                          : launch_split<64, 2>(tk, tv, q, seqlens, part_o, part_lse, B, Hq, Hkv,
-                                               Lmax, chunk, scale_log2, status, stream);
+                                               Lmax, chunk, window, sinks, scale_log2, status, stream);
         if (rc) return rc;
     }
     // The combine kernel is a programmatic dependent launch: it is scheduled

@@ -152,10 +152,10 @@ extern "C" {
 
 const char *gqa_last_error(void) { return t_last_error; }
 
-int gqa_attn_fwd_lse(const void *q, const void *k, const void *v, void *o, float *lse,
-                     int B, int Tq, int Tkv, int Hq, int Hkv, int d, int causal, float scale,
-                     gqa_stream_t stream) {
-    t_last_error[0] = 0;
+// Shared by the plain and the sliding-window forward (window = 0: none).
+static int attn_fwd_bf16(const void *q, const void *k, const void *v, void *o, float *lse,
+                         int B, int Tq, int Tkv, int Hq, int Hkv, int d, int causal, int window,
+                         int sinks, float scale, gqa_stream_t stream) {
     if (int rc = check_fwd_common(B, Tq, Tkv, Hq, Hkv, d, causal, scale)) return rc;
     if (d != 64 && d != 128)
         return set_error(GQA_ERR_UNSUPPORTED, "head dim d=%d: the bf16 path supports 64 and 128", d);
@@ -170,7 +170,25 @@ int gqa_attn_fwd_lse(const void *q, const void *k, const void *v, void *o, float
     if (Tkv == 0) return launch_empty_rows(o, lse, 2, B, Tq, Hq, d, s);
     if (int rc = check_ptr(k, 16, "k")) return rc;
     if (int rc = check_ptr(v, 16, "v")) return rc;
-    return launch_prefill(q, k, v, o, lse, B, Tq, Tkv, Hq, Hkv, d, causal, scale, s);
+    return launch_prefill(q, k, v, o, lse, B, Tq, Tkv, Hq, Hkv, d, causal, window, sinks, scale,
+                          s);
+}
+
+int gqa_attn_fwd_lse(const void *q, const void *k, const void *v, void *o, float *lse,
+                     int B, int Tq, int Tkv, int Hq, int Hkv, int d, int causal, float scale,
+                     gqa_stream_t stream) {
+    t_last_error[0] = 0;
+    return attn_fwd_bf16(q, k, v, o, lse, B, Tq, Tkv, Hq, Hkv, d, causal, 0, 0, scale, stream);
+}
+
+int gqa_attn_fwd_window(const void *q, const void *k, const void *v, void *o, float *lse,
+                        int B, int Tq, int Tkv, int Hq, int Hkv, int d, int window, int sinks,
+                        float scale, gqa_stream_t stream) {
+    t_last_error[0] = 0;
+    if (window < 1 || sinks < 0)
+        return set_error(GQA_ERR_INVALID_ARG, "window=%d must be >= 1 and sinks=%d >= 0", window,
+                         sinks);
+    return attn_fwd_bf16(q, k, v, o, lse, B, Tq, Tkv, Hq, Hkv, d, 1, window, sinks, scale, stream);
 }
 
 int gqa_attn_fwd(const void *q, const void *k, const void *v, void *o, int B, int Tq, int Tkv,
@@ -201,10 +219,10 @@ size_t gqa_decode_workspace_size(int B, int Hq, int Hkv, int d, int Lmax) {
     return decode_workspace_bytes(B, Hq, Hkv, d, Lmax);
 }
 
-int gqa_decode(const void *q, const void *k_cache, const void *v_cache, const int32_t *seqlens,
-               void *o, int B, int Hq, int Hkv, int d, int Lmax, float scale, void *workspace,
-               size_t workspace_bytes, gqa_stream_t stream) {
-    t_last_error[0] = 0;
+static int decode_bf16(const void *q, const void *k_cache, const void *v_cache,
+                       const int32_t *seqlens, void *o, int B, int Hq, int Hkv, int d, int Lmax,
+                       int window, int sinks, float scale, void *workspace,
+                       size_t workspace_bytes, gqa_stream_t stream) {
     if (B < 0 || Lmax < 0) return set_error(GQA_ERR_INVALID_ARG, "B=%d, Lmax=%d must be >= 0", B, Lmax);
     if (int rc = check_heads(Hq, Hkv, d)) return rc;
     if (int rc = check_scale(scale)) return rc;
@@ -231,8 +249,28 @@ int gqa_decode(const void *q, const void *k_cache, const void *v_cache, const in
                              workspace_bytes, need);
     }
     if (int rc = require_sm100()) return rc;
-    return launch_decode(q, k_cache, v_cache, seqlens, o, B, Hq, Hkv, d, Lmax, scale, workspace,
-                         reinterpret_cast<cudaStream_t>(stream));
+    return launch_decode(q, k_cache, v_cache, seqlens, o, B, Hq, Hkv, d, Lmax, window, sinks,
+                         scale, workspace, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int gqa_decode(const void *q, const void *k_cache, const void *v_cache, const int32_t *seqlens,
+               void *o, int B, int Hq, int Hkv, int d, int Lmax, float scale, void *workspace,
+               size_t workspace_bytes, gqa_stream_t stream) {
+    t_last_error[0] = 0;
+    return decode_bf16(q, k_cache, v_cache, seqlens, o, B, Hq, Hkv, d, Lmax, 0, 0, scale,
+                       workspace, workspace_bytes, stream);
+}
+
+int gqa_decode_window(const void *q, const void *k_cache, const void *v_cache,
+                      const int32_t *seqlens, void *o, int B, int Hq, int Hkv, int d, int Lmax,
+                      int window, int sinks, float scale, void *workspace,
+                      size_t workspace_bytes, gqa_stream_t stream) {
+    t_last_error[0] = 0;
+    if (window < 1 || sinks < 0)
+        return set_error(GQA_ERR_INVALID_ARG, "window=%d must be >= 1 and sinks=%d >= 0", window,
+                         sinks);
+    return decode_bf16(q, k_cache, v_cache, seqlens, o, B, Hq, Hkv, d, Lmax, window, sinks, scale,
+                       workspace, workspace_bytes, stream);
 }
 
 int gqa_fold_kv(const void *in, void *out, int B, int T, int H, int g, int d,

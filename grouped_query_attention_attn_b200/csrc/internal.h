@@ -44,13 +44,14 @@ int launch_fold_kv(const void *in, void *out, int B, int T, int H, int g, int d,
 // Keys per decode split for these sizes (a multiple of the stage size).
 int decode_chunk(int B, int Hkv, int Lmax);
 size_t decode_workspace_bytes(int B, int Hq, int Hkv, int d, int Lmax);
+// window = 0: no sliding window (sinks ignored)
 int launch_decode(const void *q, const void *k_cache, const void *v_cache,
                   const int32_t *seqlens, void *o, int B, int Hq, int Hkv, int d, int Lmax,
-                  float scale, void *workspace, cudaStream_t stream);
+                  int window, int sinks, float scale, void *workspace, cudaStream_t stream);
 
 int launch_prefill(const void *q, const void *k, const void *v, void *o, float *lse,
-                   int B, int Tq, int Tkv, int Hq, int Hkv, int d, int causal, float scale,
-                   cudaStream_t stream);
+                   int B, int Tq, int Tkv, int Hq, int Hkv, int d, int causal, int window,
+                   int sinks, float scale, cudaStream_t stream);
 
 int selftest_wait_timeout(int timeout_us);
 

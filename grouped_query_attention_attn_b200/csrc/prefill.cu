@@ -25,6 +25,7 @@
 // Softmax warps rescale O_k by exp2(m_old - m_new) before the next PV, which
 // is safe because the commit that signals S_k(j) also covers PV_k(j-1).
 #include <cuda_bf16.h>
+#include <climits>
 
 #include "device.cuh"
 #include "internal.h"
@@ -62,6 +63,7 @@ struct PfParams {
     int B, Tq, Tkv, Hq, Hkv, G, P;   // P = positions per M tile
     int n_pairs;                      // M-tile pairs per (b, kvh)
     int causal;
+    int window, sinks;                // sliding window (0 = none) and sink keys
     float scale_log2;                 // scale * log2(e)
     __nv_bfloat16 *o;
     float *lse;
@@ -114,7 +116,18 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     const int last_pos = min(t0 + 2 * p.P, p.Tq) - 1;   // last real position in the pair
     int kv_end = p.Tkv;                                 // keys [0, kv_end) can be visible
     if (p.causal) kv_end = min(p.Tkv, last_pos + (p.Tkv - p.Tq) + 1);
-    const int n_kv = kv_end > 0 ? (kv_end + kPfBN - 1) / kPfBN : 0;
+    // KV tiles visited, in order: the sink tiles, then the window tiles (all
+    // tiles below kv_end when there is no window); tile_of(j) maps the
+    // visiting order to the tile index.
+    int n_sink_tiles = 0, first_tile = 0;
+    if (p.window > 0 && kv_end > 0) {
+        const int lo_min = t0 + (p.Tkv - p.Tq) - p.window + 1;   // window start, first row
+        n_sink_tiles = (min(p.sinks, kv_end) + kPfBN - 1) / kPfBN;
+        first_tile = max(n_sink_tiles, max(lo_min, 0) / kPfBN);
+    }
+    const int last_tile = kv_end > 0 ? (kv_end + kPfBN - 1) / kPfBN : 0;  // exclusive
+    const int n_kv = n_sink_tiles + max(0, last_tile - first_tile);
+    auto tile_of = [&](int j) { return j < n_sink_tiles ? j : first_tile + (j - n_sink_tiles); };
 
     if (threadIdx.x == 0) {
         mbar_init(&q_full, 1);
@@ -174,7 +187,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                     mbar_expect_tx(&k_full[st], Lay::kKTile);
                     for (int pn = 0; pn < Lay::kPanels; ++pn)
                         tma_load_4d(sK + st * Lay::kKTile + pn * Lay::kKPanel, &tm_k, &k_full[st],
-                                    pn * 64, kvh, j * kPfBN, b);
+                                    pn * 64, kvh, tile_of(j) * kPfBN, b);
                 }
                 __syncwarp();
                 issued = j + 1;
@@ -184,7 +197,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                     mbar_expect_tx(&v_full[st], Lay::kKTile);
                     for (int pn = 0; pn < Lay::kPanels; ++pn)
                         tma_load_4d(sV + st * Lay::kKTile + pn * Lay::kKPanel, &tm_v, &v_full[st],
-                                    pn * 64, kvh, j * kPfBN, b);
+                                    pn * 64, kvh, tile_of(j) * kPfBN, b);
                 }
                 __syncwarp();
             }
@@ -325,9 +338,12 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         const int pos = t0 + k * p.P + r / p.G;
         const int head = kvh * p.G + r % p.G;
         const bool row_real = (r < p.P * p.G) && (pos < p.Tq);
-        // last visible key of this row (keys past Tkv never count)
+        // visible keys of this row: key <= lim, and key >= lo or key < sinks
+        // (keys past Tkv never count; lo / sinks only with a sliding window)
         int lim = p.Tkv - 1;
         if (p.causal && row_real) lim = min(lim, pos + (p.Tkv - p.Tq));
+        const int lo = (p.window > 0 && row_real) ? pos + (p.Tkv - p.Tq) - p.window + 1 : INT_MIN;
+        const int n_sinks = p.window > 0 ? p.sinks : 0;
         // Online softmax with a lazily moved reference max: O and l stay scaled
         // by exp2(-m_ref) and m_ref only moves when a row's max exceeds it by
         // more than kRescaleLog2 (P then stays <= 2^kRescaleLog2).  Exact in
@@ -350,14 +366,18 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             tmem_ld32(lane_addr + colS, sr[0]);
             tmem_ld32(lane_addr + colS + 32, sr[1]);
             tmem_wait_ld();
-            const int cut = lim - j * kPfBN - 64 * h;   // my columns > cut are masked
-            const bool masked = __any_sync(0xffffffffu, cut < 63);
+            const int key0 = tile_of(j) * kPfBN + 64 * h;   // key of my first column
+            const bool masked = __any_sync(0xffffffffu, key0 + 63 > lim ||
+                                                            (key0 < lo && key0 + 63 >= n_sinks));
             if (masked) {
 #pragma unroll
                 for (int c = 0; c < 2; ++c)
 #pragma unroll
-                    for (int e = 0; e < 32; ++e)
-                        if (32 * c + e > cut) sr[c][e] = __float_as_uint(-INFINITY);
+                    for (int e = 0; e < 32; ++e) {
+                        const int key = key0 + 32 * c + e;
+                        if (key > lim || (key < lo && key >= n_sinks))
+                            sr[c][e] = __float_as_uint(-INFINITY);
+                    }
             }
             // row max of the raw scores (scale > 0 keeps the order), then the
             // other half's max through shared memory
@@ -485,9 +505,11 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
 
 template <int D>
 static int launch_prefill_d(const void *q, const void *k, const void *v, void *o, float *lse,
-                            int B, int Tq, int Tkv, int Hq, int Hkv, int causal, float scale,
-                            cudaStream_t stream) {
+                            int B, int Tq, int Tkv, int Hq, int Hkv, int causal, int window,
+                            int sinks, float scale, cudaStream_t stream) {
     PfParams prm;
+    prm.window = window;
+    prm.sinks = sinks;
     prm.B = B;
     prm.Tq = Tq;
     prm.Tkv = Tkv;
@@ -521,11 +543,13 @@ static int launch_prefill_d(const void *q, const void *k, const void *v, void *o
 }
 
 int launch_prefill(const void *q, const void *k, const void *v, void *o, float *lse, int B,
-                   int Tq, int Tkv, int Hq, int Hkv, int d, int causal, float scale,
-                   cudaStream_t stream) {
+                   int Tq, int Tkv, int Hq, int Hkv, int d, int causal, int window, int sinks,
+                   float scale, cudaStream_t stream) {
     if (d == 128)
-        return launch_prefill_d<128>(q, k, v, o, lse, B, Tq, Tkv, Hq, Hkv, causal, scale, stream);
-    return launch_prefill_d<64>(q, k, v, o, lse, B, Tq, Tkv, Hq, Hkv, causal, scale, stream);
+        return launch_prefill_d<128>(q, k, v, o, lse, B, Tq, Tkv, Hq, Hkv, causal, window, sinks,
+                                     scale, stream);
+    return launch_prefill_d<64>(q, k, v, o, lse, B, Tq, Tkv, Hq, Hkv, causal, window, sinks,
+                                scale, stream);
 }
 
 }  // namespace gqa

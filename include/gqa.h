@@ -79,6 +79,22 @@ int gqa_attn_fwd_lse(const void *q, const void *k, const void *v, void *o, float
                      int causal, float scale, gqa_stream_t stream);
 
 /*
+ * gqa_attn_fwd_window -- causal forward with a sliding window and attention
+ * sinks (course "Неделя 7. Внимание", step 3: the window bounds what a token
+ * sees -- and the cache -- to the most recent keys, while the first tokens,
+ * where the softmax parks its mass, stay visible).
+ *
+ * Row i (key position p = i + Tkv - Tq) sees key j iff j <= p and
+ * (j > p - window or j < sinks).  window >= 1 (window >= Tkv + Tq is plain
+ * causal attention), sinks >= 0; other arguments, layouts, lse (may be NULL)
+ * and errors as gqa_attn_fwd_lse.  Only the KV tiles a CTA's rows can see are
+ * read: the sink tiles and the tiles of the window.
+ */
+int gqa_attn_fwd_window(const void *q, const void *k, const void *v, void *o, float *lse,
+                        int B, int Tq, int Tkv, int Hq, int Hkv, int d,
+                        int window, int sinks, float scale, gqa_stream_t stream);
+
+/*
  * gqa_attn_fwd_f32 -- the same operation in fp32 end to end (fp32 FFMA,
  * no tensor cores).  Same layouts; fp32 tensors; any 1 <= d <= 256; pointers
  * 4-byte aligned; lse may be NULL.  A correctness path for fp32 callers, not
@@ -116,6 +132,19 @@ int gqa_decode(const void *q, const void *k_cache, const void *v_cache,
                const int32_t *seqlens, void *o,
                int B, int Hq, int Hkv, int d, int Lmax, float scale,
                void *workspace, size_t workspace_bytes, gqa_stream_t stream);
+
+/*
+ * gqa_decode_window -- gqa_decode with a sliding window and attention sinks
+ * (course step 3): the newest token of sequence b sees cache rows
+ * j >= seqlens[b] - window and rows j < sinks.  window >= 1, sinks >= 0;
+ * everything else (layouts, workspace and its size, errors) as gqa_decode.
+ * KV splits that hold no visible row read nothing.
+ */
+int gqa_decode_window(const void *q, const void *k_cache, const void *v_cache,
+                      const int32_t *seqlens, void *o,
+                      int B, int Hq, int Hkv, int d, int Lmax, int window, int sinks,
+                      float scale, void *workspace, size_t workspace_bytes,
+                      gqa_stream_t stream);
 
 /*
  * gqa_decode_static -- gqa_decode for callers that cannot allocate device

@@ -148,3 +148,14 @@ def test_product_package_never_imports_the_oracle():
                 text = open(os.path.join(dirpath, f)).read()
                 assert not re.search(r"^\s*(from|import)\s+oracle\b", text, re.M), f
                 assert "gqa_oracle" not in text and "liboracle" not in text, f
+
+
+def test_window_entry_points_reject_bad_window(gqa_lib):
+    for window, sinks in ((0, 0), (-3, 0), (4, -1)):
+        assert b.gqa_attn_fwd_window(FAKE, FAKE, FAKE, FAKE, NULL, 1, 8, 8, 4, 2, 128, window,
+                                     sinks, 0.088, NULL) == b.GQA_ERR_INVALID_ARG
+        assert b.gqa_decode_window(FAKE, FAKE, FAKE, FAKE, FAKE, 2, 4, 2, 128, 64, window, sinks,
+                                   0.088, FAKE, 1 << 20, NULL) == b.GQA_ERR_INVALID_ARG
+    # the usual shape checks still apply
+    assert b.gqa_attn_fwd_window(FAKE, FAKE, FAKE, FAKE, NULL, 1, 8, 8, 6, 4, 128, 4, 0, 0.088,
+                                 NULL) == b.GQA_ERR_INVALID_ARG
