@@ -258,3 +258,25 @@ def mults(n, d_model, h, g, head_dim):
     return {"proj_q": proj_q, "proj_k": proj_k, "proj_v": proj_v,
             "scores": scores, "weighted": weighted, "proj_out": proj_out,
             "total": total}
+
+
+def rope(x, positions, theta=10000.0):
+    """Rotary position embedding of one head's rows (course "Неделя 7. Внимание",
+    step 3): coordinate pair (2i, 2i+1) of the row at position m is rotated by
+    the angle m * theta_i, theta_i = theta ** (-2i / d).  Reading: adjacent
+    coordinates form a pair (the complex-number form of the page).
+    ``x``: rows of length d (even); ``positions``: one position per row."""
+    out = []
+    for row, m in zip(x, positions, strict=True):
+        d = len(row)
+        if d % 2:
+            raise ValueError("head dim must be even for RoPE")
+        r = list(row)
+        for i in range(d // 2):
+            ang = m * theta ** (-2.0 * i / d)
+            c, s = math.cos(ang), math.sin(ang)
+            a, b = row[2 * i], row[2 * i + 1]
+            r[2 * i] = a * c - b * s
+            r[2 * i + 1] = a * s + b * c
+        out.append(r)
+    return out

@@ -205,3 +205,35 @@ def fold_kv_tensor(kv, g):
             acc = acc + x[:, :, grp * size + m, :]        # float32 adds, head order
         out[:, :, grp, :] = acc / np.float32(size)
     return torch.from_numpy(out).to(torch.bfloat16)
+
+
+def rope_tensor(x, pos0, theta=10000.0):
+    """RoPE of a [B, T, H, d] tensor with row t at position pos0 + t, in double.
+
+    Course "Неделя 7. Внимание", step 3: pair (2i, 2i+1) rotated by
+    m * theta ** (-2i / d).  Returns a float64 numpy array."""
+    x = _f32(x).astype(np.float64)
+    B, T, H, d = x.shape
+    if d % 2:
+        raise ValueError("head dim must be even for RoPE")
+    m = (pos0 + np.arange(T, dtype=np.float64))[:, None]          # [T, 1]
+    inv = theta ** (-2.0 * np.arange(d // 2, dtype=np.float64) / d)  # [d/2]
+    ang = m * inv[None, :]                                          # [T, d/2]
+    c = np.cos(ang)[None, :, None, :]
+    s = np.sin(ang)[None, :, None, :]
+    a, b = x[..., 0::2], x[..., 1::2]
+    out = np.empty_like(x)
+    out[..., 0::2] = a * c - b * s
+    out[..., 1::2] = a * s + b * c
+    return out
+
+
+def rope_decode_q(q, seqlens, theta=10000.0):
+    """RoPE of decode queries [B, H, d]: sequence b's token sits at position seqlens[b] - 1."""
+    q = _f32(q).astype(np.float64)
+    if hasattr(seqlens, "detach"):
+        seqlens = seqlens.detach().cpu().numpy()
+    out = np.empty_like(q)
+    for b in range(q.shape[0]):
+        out[b] = rope_tensor(q[b][None, None], int(seqlens[b]) - 1, theta)[0, 0]
+    return out
