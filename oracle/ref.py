@@ -229,11 +229,13 @@ def rope_tensor(x, pos0, theta=10000.0):
 
 
 def rope_decode_q(q, seqlens, theta=10000.0):
-    """RoPE of decode queries [B, H, d]: sequence b's token sits at position seqlens[b] - 1."""
+    """RoPE of decode queries [B, H, d]: sequence b's token sits at position
+    max(seqlens[b] - 1, 0) (reading: with an empty cache the new token is the
+    first one, position 0)."""
     q = _f32(q).astype(np.float64)
     if hasattr(seqlens, "detach"):
         seqlens = seqlens.detach().cpu().numpy()
     out = np.empty_like(q)
     for b in range(q.shape[0]):
-        out[b] = rope_tensor(q[b][None, None], int(seqlens[b]) - 1, theta)[0, 0]
+        out[b] = rope_tensor(q[b][None, None], max(int(seqlens[b]) - 1, 0), theta)[0, 0]
     return out

@@ -55,13 +55,14 @@ def test_rope_tensor_matches_lab_rows():
 
 
 def test_rope_decode_q_positions():
-    q = rand((3, 2, 16), 6)
-    sl = torch.tensor([1, 10, 300], dtype=torch.int32)
+    q = rand((4, 2, 16), 6)
+    sl = torch.tensor([1, 10, 300, 0], dtype=torch.int32)
     got = ref.rope_decode_q(q, sl)
     for b in range(3):
         want = ref.rope_tensor(q[b][None, None], int(sl[b]) - 1)[0, 0]
         assert np.array_equal(got[b], want)
     assert np.array_equal(got[0], q[0].double().numpy())      # position 0: identity
+    assert np.array_equal(got[3], q[3].double().numpy())      # empty cache: position 0
 
 
 def test_rope_odd_dim_rejected():
