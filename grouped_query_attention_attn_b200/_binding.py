@@ -36,6 +36,8 @@ _SIGNATURES = {
                                ctypes.c_size_t, _P]),
     "gqa_decode_static": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _P]),
     "gqa_fold_kv": (_I, [_P, _P, _I, _I, _I, _I, _I, _P]),
+    "gqa_rope": (_I, [_P, _I, _I, _I, _I, _I, _F, _P]),
+    "gqa_rope_decode_q": (_I, [_P, _P, _I, _I, _I, _F, _P]),
     "gqa_last_error": (ctypes.c_char_p, []),
     "gqa_device_status": (_I, [_I]),
     "gqa_selftest_wait_timeout": (_I, [_I]),
@@ -99,6 +101,14 @@ def gqa_decode_static(q, k_cache, v_cache, seqlens, o, B, Hq, Hkv, d, Lmax, scal
 
 def gqa_fold_kv(inp, out, B, T, H, g, d, stream):
     return lib().gqa_fold_kv(inp, out, B, T, H, g, d, stream)
+
+
+def gqa_rope(x, B, T, H, d, pos0, theta, stream):
+    return lib().gqa_rope(x, B, T, H, d, pos0, theta, stream)
+
+
+def gqa_rope_decode_q(q, seqlens, B, H, d, theta, stream):
+    return lib().gqa_rope_decode_q(q, seqlens, B, H, d, theta, stream)
 
 
 def gqa_last_error():

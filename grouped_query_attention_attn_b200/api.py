@@ -142,6 +142,25 @@ def fold_kv(kv, g):
     return out
 
 
+def rope_(x, pos0=0, theta=10000.0):
+    """Rotary position embedding of a bf16 [B, T, H, d] q or k tensor, in place
+    (row t at position pos0 + t).  Returns x."""
+    _need(x, "x", torch.bfloat16, 4)
+    B, T, H, d = x.shape
+    _check(_b.gqa_rope(x.data_ptr(), B, T, H, d, int(pos0), float(theta), _stream(x)), "gqa_rope")
+    return x
+
+
+def rope_decode_q_(q, seqlens, theta=10000.0):
+    """RoPE of bf16 decode queries [B, H, d] in place, sequence b at position seqlens[b] - 1."""
+    _need(q, "q", torch.bfloat16, 3)
+    _need(seqlens, "seqlens", torch.int32, 1)
+    B, H, d = q.shape
+    _check(_b.gqa_rope_decode_q(q.data_ptr(), seqlens.data_ptr(), B, H, d, float(theta),
+                                _stream(q)), "gqa_rope_decode_q")
+    return q
+
+
 def device_status(reset=True):
     """Synchronise, then raise if a kernel recorded an error (e.g. a wait timeout)."""
     _check(_b.gqa_device_status(int(bool(reset))), "gqa_device_status")

@@ -42,6 +42,8 @@ int set_error(int code, const char *fmt, ...) {
     return code;
 }
 
+void clear_error() { t_last_error[0] = 0; }
+
 int check_cuda(cudaError_t e, const char *what) {
     if (e == cudaSuccess) return GQA_OK;
     return set_error(GQA_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));

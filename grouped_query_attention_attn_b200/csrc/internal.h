@@ -13,6 +13,9 @@ namespace gqa {
 // Record a message for gqa_last_error() on this host thread; returns `code`.
 int set_error(int code, const char *fmt, ...);
 
+// Clear that message (every entry point starts with it).
+void clear_error();
+
 // Map a CUDA runtime error to GQA_ERR_CUDA with a message; GQA_OK on success.
 int check_cuda(cudaError_t e, const char *what);
 

@@ -122,7 +122,7 @@ size_t gqa_decode_workspace_size(int B, int Hq, int Hkv, int d, int Lmax);
  *   o        [B, Hq, d] bf16 (written; a sequence of length 0 gets zeros)
  *   workspace: device scratch of at least gqa_decode_workspace_size(...)
  *   bytes, 256-byte aligned; its contents on entry do not matter.
- *   d in {64, 128}; Hq % Hkv == 0; G = Hq/Hkv <= 64.
+ *   d in {64, 128}; Hq % Hkv == 0; G = Hq/Hkv <= 32 (else UNSUPPORTED).
  * Each split of the KV length is streamed from HBM once for all G query heads
  * of its group, and the splits are merged with the log-sum-exp identity by a
  * second kernel on the same stream.  A seqlens[b] above Lmax is clamped to
@@ -177,6 +177,29 @@ int gqa_decode_window(const void *q, const void *k_cache, const void *v_cache,
 int gqa_decode_static(const void *q, const void *k_cache, const void *v_cache,
                       const int32_t *seqlens, void *o,
                       int B, int Hq, int Hkv, int d, int Lmax, float scale,
+                      gqa_stream_t stream);
+
+/*
+ * gqa_rope -- rotary position embedding, in place (course "Неделя 7.
+ * Внимание", step 3): coordinate pair (2i, 2i+1) of the row at position m is
+ * rotated by m * theta^(-2i/d).  Apply it to q and to k (never to v) before
+ * attention; the scores then depend on position differences only.
+ *   x [B, T, H, d] bf16, rewritten in place; row t sits at position pos0 + t
+ *   (for causal prefill with Tq != Tkv: q uses pos0 + Tkv - Tq, k uses pos0).
+ *   d a multiple of 8 in [8, 256]; theta > 0 (10000 is usual); x 16-byte
+ *   aligned.  Angles are reduced in double, then fp32 sine / cosine; the
+ *   result is rounded to bf16 (nearest even).  Reading of the page: adjacent
+ *   coordinates form a pair.
+ */
+int gqa_rope(void *x, int B, int T, int H, int d, int pos0, float theta, gqa_stream_t stream);
+
+/*
+ * gqa_rope_decode_q -- gqa_rope of decode queries q [B, H, d] (bf16, in place):
+ * sequence b's new token sits at position max(seqlens[b] - 1, 0) (seqlens:
+ * device int32 [B]; an empty cache makes it the first token).  The cached keys are expected to be rotated already, each at
+ * its own position when it was appended.
+ */
+int gqa_rope_decode_q(void *q, const int32_t *seqlens, int B, int H, int d, float theta,
                       gqa_stream_t stream);
 
 /*

@@ -159,3 +159,11 @@ def test_window_entry_points_reject_bad_window(gqa_lib):
     # the usual shape checks still apply
     assert b.gqa_attn_fwd_window(FAKE, FAKE, FAKE, FAKE, NULL, 1, 8, 8, 6, 4, 128, 4, 0, 0.088,
                                  NULL) == b.GQA_ERR_INVALID_ARG
+
+
+def test_rope_rejects(gqa_lib):
+    assert b.gqa_rope(FAKE, 1, 4, 2, 12, 0, 10000.0, NULL) == b.GQA_ERR_INVALID_ARG   # d % 8
+    assert b.gqa_rope(FAKE, 1, 4, 2, 128, 0, 0.0, NULL) == b.GQA_ERR_INVALID_ARG      # theta
+    assert b.gqa_rope(FAKE + 8, 1, 4, 2, 128, 0, 10000.0, NULL) == b.GQA_ERR_INVALID_ARG
+    assert b.gqa_rope(NULL, 0, 4, 2, 128, 0, 10000.0, NULL) == b.GQA_OK              # empty
+    assert b.gqa_rope_decode_q(FAKE, NULL, 2, 2, 128, 10000.0, NULL) == b.GQA_ERR_INVALID_ARG
