@@ -239,3 +239,47 @@ def rope_decode_q(q, seqlens, theta=10000.0):
     for b in range(q.shape[0]):
         out[b] = rope_tensor(q[b][None, None], max(int(seqlens[b]) - 1, 0), theta)[0, 0]
     return out
+
+
+def attn_bwd(q, k, v, do, causal, scale=None, window=0, sinks=0):
+    """Gradients of the attention output with respect to q, k and v, in float64.
+
+    The forward is the plain definition, written with torch CPU ops: K and V
+    expanded to the query heads by repeat_interleave (K3 notes, "GVA",
+    "Forward: repeat_interleave"), scores scaled by ``scale``, masked with -inf
+    before the softmax, weighted sum of V.  torch autograd supplies the chain
+    rule, so the expanded heads' gradients are summed back into each shared K/V
+    head ("Backward: view + sum": the gradient of a copy is a sum, not a mean).
+    Returns (dq [B,Tq,Hq,d], dk, dv [B,Tkv,Hkv,d]) as float64 numpy arrays.
+    """
+    import torch
+    qd = torch.from_numpy(_f32(q).astype(np.float64)).requires_grad_(True)
+    kd = torch.from_numpy(_f32(k).astype(np.float64)).requires_grad_(True)
+    vd = torch.from_numpy(_f32(v).astype(np.float64)).requires_grad_(True)
+    dod = torch.from_numpy(_f32(do).astype(np.float64))
+    B, Tq, Hq, d = qd.shape
+    Tkv, Hkv = kd.shape[1], kd.shape[2]
+    if Hq % Hkv != 0:
+        raise ValueError("Hq must be a multiple of Hkv")
+    G = Hq // Hkv
+    sc = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    ke = kd.repeat_interleave(G, dim=2)                     # [B, Tkv, Hq, d]
+    ve = vd.repeat_interleave(G, dim=2)
+    s = torch.einsum("bihc,bjhc->bhij", qd, ke) * sc
+    i = torch.arange(Tq)[:, None]
+    j = torch.arange(Tkv)[None, :]
+    p_pos = i + (Tkv - Tq)
+    vis = torch.ones(Tq, Tkv, dtype=torch.bool)
+    if causal:
+        vis &= j <= p_pos
+        if window > 0:
+            vis &= (j > p_pos - window) | (j < sinks)
+    s = s.masked_fill(~vis, float("-inf"))
+    m = s.amax(dim=-1, keepdim=True)
+    m = torch.where(torch.isfinite(m), m, torch.zeros_like(m))   # rows with no key
+    e = torch.exp(s - m)
+    den = e.sum(dim=-1, keepdim=True)
+    p = e / torch.where(den > 0, den, torch.ones_like(den))
+    o = torch.einsum("bhij,bjhc->bihc", p, ve)
+    o.backward(dod)
+    return qd.grad.numpy(), kd.grad.numpy(), vd.grad.numpy()
