@@ -36,6 +36,9 @@ _SIGNATURES = {
                                ctypes.c_size_t, _P]),
     "gqa_decode_static": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _P]),
     "gqa_fold_kv": (_I, [_P, _P, _I, _I, _I, _I, _I, _P]),
+    "gqa_attn_bwd_workspace_size": (ctypes.c_size_t, [_I, _I, _I]),
+    "gqa_attn_bwd": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _I,
+                          _F, _P, ctypes.c_size_t, _P]),
     "gqa_rope": (_I, [_P, _I, _I, _I, _I, _I, _F, _P]),
     "gqa_rope_decode_q": (_I, [_P, _P, _I, _I, _I, _F, _P]),
     "gqa_last_error": (ctypes.c_char_p, []),
@@ -101,6 +104,16 @@ def gqa_decode_static(q, k_cache, v_cache, seqlens, o, B, Hq, Hkv, d, Lmax, scal
 
 def gqa_fold_kv(inp, out, B, T, H, g, d, stream):
     return lib().gqa_fold_kv(inp, out, B, T, H, g, d, stream)
+
+
+def gqa_attn_bwd_workspace_size(B, Tq, Hq):
+    return lib().gqa_attn_bwd_workspace_size(B, Tq, Hq)
+
+
+def gqa_attn_bwd(q, k, v, o, dout, lse, dq, dk, dv, B, Tq, Tkv, Hq, Hkv, d, causal, window, sinks,
+                 scale, workspace, workspace_bytes, stream):
+    return lib().gqa_attn_bwd(q, k, v, o, dout, lse, dq, dk, dv, B, Tq, Tkv, Hq, Hkv, d, causal,
+                              window, sinks, scale, workspace, workspace_bytes, stream)
 
 
 def gqa_rope(x, B, T, H, d, pos0, theta, stream):

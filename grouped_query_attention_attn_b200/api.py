@@ -142,6 +142,33 @@ def fold_kv(kv, g):
     return out
 
 
+def attn_bwd(q, k, v, o, lse, dout, causal=True, scale=None, window=None, sinks=0,
+             workspace=None):
+    """Gradients (dq, dk, dv) of attn(q, k, v) for the upstream gradient dout.
+
+    o and lse are the forward's outputs (attn(..., return_lse=True)).  dk / dv
+    of a K/V head are summed over the G query heads that share it.
+    """
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (o, "o"), (dout, "dout")):
+        _need(t, n, torch.bfloat16, 4)
+    _need(lse, "lse", torch.float32, 3)
+    B, Tq, Tkv, Hq, Hkv, d = _shapes(q, k, v)
+    if tuple(o.shape) != tuple(q.shape) or tuple(dout.shape) != tuple(q.shape):
+        raise ValueError("o and dout must have q's shape")
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    need = int(_b.gqa_attn_bwd_workspace_size(B, Tq, Hq))
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    rc = _b.gqa_attn_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), dout.data_ptr(),
+                         lse.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(),
+                         B, Tq, Tkv, Hq, Hkv, d, int(bool(causal)),
+                         0 if window is None else int(window), int(sinks), scale,
+                         workspace.data_ptr(), workspace.numel(), _stream(q))
+    _check(rc, "gqa_attn_bwd")
+    return dq, dk, dv
+
+
 def rope_(x, pos0=0, theta=10000.0):
     """Rotary position embedding of a bf16 [B, T, H, d] q or k tensor, in place
     (row t at position pos0 + t).  Returns x."""

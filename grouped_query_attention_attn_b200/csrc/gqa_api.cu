@@ -275,6 +275,53 @@ int gqa_decode_window(const void *q, const void *k_cache, const void *v_cache,
                        workspace, workspace_bytes, stream);
 }
 
+size_t gqa_attn_bwd_workspace_size(int B, int Tq, int Hq) {
+    if (B < 0 || Tq < 0 || Hq < 1) return 0;
+    return bwd_workspace_bytes(B, Tq, Hq);
+}
+
+int gqa_attn_bwd(const void *q, const void *k, const void *v, const void *o, const void *dout,
+                 const float *lse, void *dq, void *dk, void *dv, int B, int Tq, int Tkv, int Hq,
+                 int Hkv, int d, int causal, int window, int sinks, float scale, void *workspace,
+                 size_t workspace_bytes, gqa_stream_t stream) {
+    t_last_error[0] = 0;
+    if (int rc = check_fwd_common(B, Tq, Tkv, Hq, Hkv, d, causal, scale)) return rc;
+    if (d != 64 && d != 128)
+        return set_error(GQA_ERR_UNSUPPORTED, "head dim d=%d: the backward supports 64 and 128", d);
+    if (window < 0 || sinks < 0 || (window > 0 && !causal))
+        return set_error(GQA_ERR_INVALID_ARG,
+                         "window=%d, sinks=%d must be >= 0 (a window needs causal=1)", window, sinks);
+    if (B == 0 || (Tq == 0 && Tkv == 0)) return GQA_OK;
+    // query-side tensors are needed when Tq > 0, key-side ones when Tkv > 0
+    const struct { const void *p; const char *n; bool kv_side; } ptrs[] = {
+        {q, "q", false}, {o, "o", false}, {dout, "dout", false}, {dq, "dq", false},
+        {k, "k", true},  {v, "v", true},  {dk, "dk", true},      {dv, "dv", true}};
+    for (const auto &e : ptrs)
+        if (e.kv_side ? Tkv > 0 : Tq > 0)
+            if (int rc = check_ptr(e.p, 16, e.n)) return rc;
+    if (Tq > 0 && !lse) return set_error(GQA_ERR_INVALID_ARG, "lse is NULL");
+    if (lse && !aligned(lse, 4)) return set_error(GQA_ERR_INVALID_ARG, "lse is not 4-byte aligned");
+    const size_t need = bwd_workspace_bytes(B, Tq, Hq);
+    if (need > 0) {
+        if (!workspace) return set_error(GQA_ERR_WORKSPACE, "workspace is NULL (%zu bytes needed)", need);
+        if (!aligned(workspace, 256))
+            return set_error(GQA_ERR_WORKSPACE, "workspace is not 256-byte aligned");
+        if (workspace_bytes < need)
+            return set_error(GQA_ERR_WORKSPACE, "workspace has %zu bytes, %zu needed",
+                             workspace_bytes, need);
+    }
+    if (int rc = require_sm100()) return rc;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (Tq == 0) {
+        // no query sees any key: the K / V gradients are zero
+        const size_t bytes = static_cast<size_t>(B) * Tkv * Hkv * d * 2;
+        if (int rc = check_cuda(cudaMemsetAsync(dk, 0, bytes, s), "cudaMemsetAsync(dk)")) return rc;
+        return check_cuda(cudaMemsetAsync(dv, 0, bytes, s), "cudaMemsetAsync(dv)");
+    }
+    return launch_bwd(q, k, v, o, dout, lse, dq, dk, dv, B, Tq, Tkv, Hq, Hkv, d, causal, window,
+                      sinks, scale, workspace, s);
+}
+
 int gqa_fold_kv(const void *in, void *out, int B, int T, int H, int g, int d,
                 gqa_stream_t stream) {
     t_last_error[0] = 0;

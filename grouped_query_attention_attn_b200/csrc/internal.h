@@ -56,6 +56,12 @@ int launch_prefill(const void *q, const void *k, const void *v, void *o, float *
                    int B, int Tq, int Tkv, int Hq, int Hkv, int d, int causal, int window,
                    int sinks, float scale, cudaStream_t stream);
 
+size_t bwd_workspace_bytes(int B, int Tq, int Hq);
+int launch_bwd(const void *q, const void *k, const void *v, const void *o, const void *dout,
+               const float *lse, void *dq, void *dk, void *dv, int B, int Tq, int Tkv, int Hq,
+               int Hkv, int d, int causal, int window, int sinks, float scale, void *workspace,
+               cudaStream_t stream);
+
 int selftest_wait_timeout(int timeout_us);
 
 }  // namespace gqa

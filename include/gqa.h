@@ -180,6 +180,36 @@ int gqa_decode_static(const void *q, const void *k_cache, const void *v_cache,
                       gqa_stream_t stream);
 
 /*
+ * gqa_attn_bwd_workspace_size -- bytes of device scratch gqa_attn_bwd needs
+ * (one fp32 row statistic per query row: B * Hq * Tq floats, rounded up to
+ * 256).  0 for invalid sizes.  Pure host function.
+ */
+size_t gqa_attn_bwd_workspace_size(int B, int Tq, int Hq);
+
+/*
+ * gqa_attn_bwd -- gradients of the forward (gqa_attn_fwd_lse or, with
+ * window > 0, gqa_attn_fwd_window) with respect to q, k and v.
+ *
+ *   q, o, dout [B, Tq, Hq, d] bf16 (o and lse from the forward; dout = dL/do)
+ *   k, v       [B, Tkv, Hkv, d] bf16
+ *   lse        [B, Hq, Tq] fp32 from the forward
+ *   dq [B, Tq, Hq, d], dk, dv [B, Tkv, Hkv, d] bf16 (written)
+ *   causal, window (0 = none, else needs causal), sinks, scale: as the forward.
+ * The gradient of a K/V head shared by G query heads is the sum of the G
+ * heads' gradients (K3 notes "GVA", "Backward: view + sum": a copy's
+ * backward is a sum, not a mean); dq carries the chain-rule factor `scale`
+ * (same notes, "scale 的处理").  P is recomputed from lse; fp32 accumulation.
+ * workspace: >= gqa_attn_bwd_workspace_size(B, Tq, Hq) bytes, 256-byte
+ * aligned, contents on entry irrelevant.  d in {64, 128}.  Errors as the
+ * forward plus GQA_ERR_WORKSPACE.
+ */
+int gqa_attn_bwd(const void *q, const void *k, const void *v, const void *o, const void *dout,
+                 const float *lse, void *dq, void *dk, void *dv,
+                 int B, int Tq, int Tkv, int Hq, int Hkv, int d,
+                 int causal, int window, int sinks, float scale,
+                 void *workspace, size_t workspace_bytes, gqa_stream_t stream);
+
+/*
  * gqa_rope -- rotary position embedding, in place (course "Неделя 7.
  * Внимание", step 3): coordinate pair (2i, 2i+1) of the row at position m is
  * rotated by m * theta^(-2i/d).  Apply it to q and to k (never to v) before

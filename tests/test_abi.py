@@ -167,3 +167,21 @@ def test_rope_rejects(gqa_lib):
     assert b.gqa_rope(FAKE + 8, 1, 4, 2, 128, 0, 10000.0, NULL) == b.GQA_ERR_INVALID_ARG
     assert b.gqa_rope(NULL, 0, 4, 2, 128, 0, 10000.0, NULL) == b.GQA_OK              # empty
     assert b.gqa_rope_decode_q(FAKE, NULL, 2, 2, 128, 10000.0, NULL) == b.GQA_ERR_INVALID_ARG
+
+
+def test_backward_rejects(gqa_lib):
+    def bwd(**kw):
+        a = dict(B=1, Tq=8, Tkv=8, Hq=4, Hkv=2, d=128, causal=1, window=0, sinks=0, ws=FAKE,
+                 ws_bytes=1 << 20, lse=FAKE)
+        a.update(kw)
+        return b.gqa_attn_bwd(FAKE, FAKE, FAKE, FAKE, FAKE, a["lse"], FAKE, FAKE, FAKE, a["B"],
+                              a["Tq"], a["Tkv"], a["Hq"], a["Hkv"], a["d"], a["causal"],
+                              a["window"], a["sinks"], 0.088, a["ws"], a["ws_bytes"], NULL)
+    assert bwd(Hkv=3) == b.GQA_ERR_INVALID_ARG
+    assert bwd(d=96) == b.GQA_ERR_UNSUPPORTED
+    assert bwd(window=4, causal=0) == b.GQA_ERR_INVALID_ARG
+    assert bwd(lse=NULL) == b.GQA_ERR_INVALID_ARG
+    assert bwd(ws=NULL) == b.GQA_ERR_WORKSPACE
+    assert bwd(ws_bytes=16) == b.GQA_ERR_WORKSPACE
+    assert bwd(B=0) == b.GQA_OK
+    assert b.gqa_attn_bwd_workspace_size(2, 100, 8) >= 2 * 100 * 8 * 4

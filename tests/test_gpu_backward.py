@@ -1,0 +1,67 @@
+"""Backward kernels (dq, dk, dv) against the float64 autograd oracle.
+
+Tolerance: the kernels round P and dS to bf16 before the tensor-core products
+(2^-9 relative each) and write bf16 gradients; gradients grow with the number
+of rows summed, so the bound is relative to the tensor's largest magnitude:
+max |gpu - ref| <= 2e-2 * max(1, max |ref|).
+"""
+
+import numpy as np
+import pytest
+import torch
+
+import grouped_query_attention_attn_b200 as gqa
+from grouped_query_attention_attn_b200 import workloads
+from oracle import ref
+
+pytestmark = pytest.mark.gpu
+
+
+def rel_err(gpu, want):
+    g = gpu.float().cpu().numpy().astype(np.float64)
+    assert np.all(np.isfinite(g))
+    return float(np.max(np.abs(g - want))) / max(1.0, float(np.max(np.abs(want))))
+
+
+@pytest.mark.parametrize("B,Tq,Tkv,Hq,Hkv,d,causal,window,sinks", [
+    (1, 128, 128, 4, 1, 128, True, 0, 0),
+    (2, 200, 200, 8, 2, 128, True, 0, 0),       # ragged tails, G = 4
+    (1, 150, 150, 8, 8, 64, False, 0, 0),       # MHA, non-causal, d = 64
+    (1, 100, 260, 6, 2, 128, True, 0, 0),       # Tq < Tkv
+    (1, 260, 100, 4, 2, 128, True, 0, 0),       # Tq > Tkv: rows with no key
+    (1, 300, 300, 8, 2, 128, True, 64, 3),      # sliding window with sinks
+    (1, 96, 96, 32, 1, 128, True, 0, 0),        # MQA
+])
+def test_backward_matches_oracle(gqa_lib, B, Tq, Tkv, Hq, Hkv, d, causal, window, sinks):
+    q, k, v = workloads.prefill_inputs(B, Tq, Hq, Hkv, d, Tkv=Tkv, seeds=(Tq, Tkv + 1, Hq + d))
+    dout = workloads.randn((B, Tq, Hq, d), 77)
+    qc, kc, vc = q.cuda(), k.cuda(), v.cuda()
+    if window:
+        o, lse = gqa.attn(qc, kc, vc, causal=True, return_lse=True, window=window, sinks=sinks)
+    else:
+        o, lse = gqa.attn(qc, kc, vc, causal=causal, return_lse=True)
+    dq, dk, dv = gqa.attn_bwd(qc, kc, vc, o, lse, dout.cuda(), causal=causal,
+                              window=window or None, sinks=sinks)
+    gqa.device_status()
+    rq, rk, rv = ref.attn_bwd(q, k, v, dout, causal, window=window, sinks=sinks)
+    assert rel_err(dq, rq) <= 2e-2
+    assert rel_err(dk, rk) <= 2e-2
+    assert rel_err(dv, rv) <= 2e-2
+
+
+def test_backward_shared_head_sum(gqa_lib):
+    # GQA gradients equal the expanded-MHA gradients summed over each group
+    B, T, Hq, Hkv, d = 1, 256, 8, 2, 128
+    G = Hq // Hkv
+    q, k, v = workloads.prefill_inputs(B, T, Hq, Hkv, d, seeds=(5, 6, 7))
+    dout = workloads.randn((B, T, Hq, d), 8).cuda()
+    qc, kc, vc = q.cuda(), k.cuda(), v.cuda()
+    o, lse = gqa.attn(qc, kc, vc, causal=True, return_lse=True)
+    dq, dk, dv = gqa.attn_bwd(qc, kc, vc, o, lse, dout)
+    ke, ve = kc.repeat_interleave(G, 2).contiguous(), vc.repeat_interleave(G, 2).contiguous()
+    oe, lsee = gqa.attn(qc, ke, ve, causal=True, return_lse=True)
+    dqe, dke, dve = gqa.attn_bwd(qc, ke, ve, oe, lsee, dout)
+    sk = dke.float().view(B, T, Hkv, G, d).sum(3)
+    sv = dve.float().view(B, T, Hkv, G, d).sum(3)
+    assert float((dk.float() - sk).abs().max()) <= 2e-2 * max(1.0, float(sk.abs().max()))
+    assert float((dv.float() - sv).abs().max()) <= 2e-2 * max(1.0, float(sv.abs().max()))
