@@ -225,6 +225,101 @@ def run_reference(args, world, rank):
 
 # ------------------------------------------------------------- GPU path --
 
+def visible_pairs(Tq, Tkv, causal=True, window=0, sinks=0):
+    """Exact number of (query, key) pairs the mask leaves visible."""
+    import numpy as np
+    p = np.arange(Tq, dtype=np.int64) + (Tkv - Tq)
+    if not causal:
+        return Tq * Tkv
+    n = np.clip(p + 1, 0, Tkv)
+    if window > 0:
+        lo = np.maximum(p - window + 1, 0)
+        n = np.clip(np.minimum(p + 1, window), 0, Tkv) + np.minimum(sinks, lo)
+    return int(n.sum())
+
+
+def time_median(fn, flush, stream, reps):
+    """Median CUDA-event time (ms) of fn() with L2 flushed before each launch."""
+    for _ in range(3):
+        fn()
+    ts = []
+    for _ in range(reps):
+        flush.zero_()
+        s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s0.record(stream)
+        fn()
+        s1.record(stream)
+        torch.cuda.synchronize()
+        ts.append(s0.elapsed_time(s1))
+    return statistics.median(ts)
+
+
+def measure_next_rows(dev, stream, flush, peaks, peak_kind, reps):
+    """Throughput of the rows built after the hot path (each on its own workload)."""
+    import grouped_query_attention_attn_b200 as gqa
+    from grouped_query_attention_attn_b200 import workloads
+
+    def tensor_row(flops, ms, cfg):
+        a = flops / (ms / 1e3) / 1e12
+        return {"value": a, "unit": "TFLOP/s", "ms": ms, "config": cfg,
+                "roofline": {"bound": "tensor", "achieved": a, "peak": peaks["bf16_tflops"],
+                             "unit": "TFLOP/s", "frac": a / peaks["bf16_tflops"],
+                             "peak_kind": f"{peak_kind} bf16 burst", "flops_per_launch": flops}}
+
+    def hbm_row(nbytes, ms, cfg):
+        a = nbytes / (ms / 1e3) / 1e9
+        return {"value": a, "unit": "GB/s", "ms": ms, "config": cfg,
+                "roofline": {"bound": "hbm", "achieved": a, "peak": peaks["hbm_gbs"],
+                             "unit": "GB/s", "frac": a / peaks["hbm_gbs"],
+                             "peak_kind": f"{peak_kind} copy", "bytes_per_launch": nbytes}}
+
+    out = {}
+    # sliding window + sinks prefill (Mistral-like window over a long prompt)
+    cw = dict(B=1, Hq=32, Hkv=8, T=16384, d=128, window=4096, sinks=4)
+    q, k, v = (t.to(dev) for t in workloads.prefill_inputs(1, cw["T"], cw["Hq"], cw["Hkv"], 128,
+                                                          seeds=(11, 12, 13)))
+    o = torch.empty_like(q)
+    ms = time_median(lambda: gqa.attn(q, k, v, causal=True, out=o, window=cw["window"],
+                                      sinks=cw["sinks"]), flush, stream, reps)
+    flops = 4 * cw["Hq"] * 128 * visible_pairs(cw["T"], cw["T"], True, cw["window"], cw["sinks"])
+    out["prefill_window"] = tensor_row(flops, ms, cw)
+    del q, k, v, o
+    # backward on the headline prefill workload (5 algorithmic matmuls)
+    c = PREFILL
+    q, k, v = (t.to(dev) for t in workloads.prefill_inputs(1, c["T"], c["Hq"], c["Hkv"], 128))
+    do = workloads.randn((1, c["T"], c["Hq"], 128), 77).to(dev)
+    o, lse = gqa.attn(q, k, v, causal=True, return_lse=True)
+    ws = torch.empty(int(gqa._binding.gqa_attn_bwd_workspace_size(1, c["T"], c["Hq"])),
+                     dtype=torch.uint8, device=dev)
+    ms = time_median(lambda: gqa.attn_bwd(q, k, v, o, lse, do, workspace=ws), flush, stream, reps)
+    out["backward"] = tensor_row(10 * c["Hq"] * 128 * visible_pairs(c["T"], c["T"]), ms,
+                                 dict(c, kernels="rowdot + dkdv + dq (mma.sync)"))
+    # RoPE of q and k of the same workload, in place (read + write)
+    ms = time_median(lambda: gqa.rope_qk_(q, k, 0), flush, stream, reps)
+    out["rope_qk"] = hbm_row(2 * (q.numel() + k.numel()) * 2, ms, dict(c, theta=10000.0))
+    del q, k, v, o, lse, do, ws
+    # MHA -> GQA fold of the head-sharing sweep's K (32 -> 8 heads)
+    kv = workloads.randn((4, 2048, 32, 128), 2).to(dev)
+    ms = time_median(lambda: gqa.fold_kv(kv, 8), flush, stream, reps)
+    out["fold_kv"] = hbm_row(kv.numel() * 2 + kv.numel() // 4 * 2, ms,
+                             dict(B=4, T=2048, H=32, g=8, d=128))
+    del kv
+    # sliding-window decode on the batched-decode workload
+    dc = DECODE
+    dq_, kc, vc, sl = workloads.decode_inputs(dc["B"], dc["Hq"], dc["Hkv"], dc["d"], dc["Lmin"],
+                                              dc["Lmax"])
+    W, S = 2048, 4
+    rows = sum(min(int(L), W) + min(S, max(0, int(L) - W)) for L in sl)
+    nbytes = rows * dc["Hkv"] * dc["d"] * 4 + 2 * dc["B"] * dc["Hq"] * dc["d"] * 2
+    dq_, kc, vc, sl = dq_.to(dev), kc.to(dev), vc.to(dev), sl.to(dev)
+    ws = torch.empty(gqa.decode_workspace_size(dc["B"], dc["Hq"], dc["Hkv"], dc["d"], dc["Lmax"]),
+                     dtype=torch.uint8, device=dev)
+    ms = time_median(lambda: gqa.decode(dq_, kc, vc, sl, workspace=ws, window=W, sinks=S), flush,
+                     stream, reps)
+    out["decode_window"] = hbm_row(nbytes, ms, dict(dc, window=W, sinks=S))
+    return out
+
+
 def run_ours(args, world, rank, local):
     import grouped_query_attention_attn_b200 as gqa
     from grouped_query_attention_attn_b200 import workloads
@@ -368,6 +463,10 @@ def run_ours(args, world, rank, local):
         dec = {"value": world * d_bytes * K / (dec_ms / 1e3) / 1e9, "unit": "GB/s",
                "roofline": dec_roof}
 
+    nxt = None
+    if args.only is None and not args.no_next:
+        nxt = measure_next_rows(dev, stream, flush, peaks, peak_kind, args.next_reps)
+
     if rank == 0:
         line = {
             "metric": METRIC, "value": value if do_pre else (dec or {}).get("value"),
@@ -386,6 +485,7 @@ def run_ours(args, world, rank, local):
             "gpu_launches": K * ((1 if do_pre else 0) + (2 if do_dec else 0)),
             "wall_s_timed_region": wall,
             "cpu_baseline": cpu,
+            "next_rows": nxt,
         }
         print(json.dumps(line), flush=True)
     if world > 1:
@@ -407,6 +507,9 @@ def main():
                     help="time one kernel family only (profiling runs)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--no-next", action="store_true",
+                    help="skip the measurements of the rows beyond the hot path")
+    ap.add_argument("--next-reps", type=int, default=20)
     args = ap.parse_args()
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")

@@ -9,4 +9,4 @@ fallback: a missing or unloadable library raises.
 """
 
 from .api import (attn, attn_bwd, attn_f32, decode, decode_workspace_size, device_status, fold_kv,  # noqa: F401
-                  rope_, rope_decode_q_)
+                  rope_, rope_decode_q_, rope_qk_)

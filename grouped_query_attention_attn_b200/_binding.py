@@ -40,6 +40,7 @@ _SIGNATURES = {
     "gqa_attn_bwd": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _I,
                           _F, _P, ctypes.c_size_t, _P]),
     "gqa_rope": (_I, [_P, _I, _I, _I, _I, _I, _F, _P]),
+    "gqa_rope_qk": (_I, [_P, _P, _I, _I, _I, _I, _I, _I, _F, _P]),
     "gqa_rope_decode_q": (_I, [_P, _P, _I, _I, _I, _F, _P]),
     "gqa_last_error": (ctypes.c_char_p, []),
     "gqa_device_status": (_I, [_I]),
@@ -118,6 +119,10 @@ def gqa_attn_bwd(q, k, v, o, dout, lse, dq, dk, dv, B, Tq, Tkv, Hq, Hkv, d, caus
 
 def gqa_rope(x, B, T, H, d, pos0, theta, stream):
     return lib().gqa_rope(x, B, T, H, d, pos0, theta, stream)
+
+
+def gqa_rope_qk(q, k, B, T, Hq, Hkv, d, pos0, theta, stream):
+    return lib().gqa_rope_qk(q, k, B, T, Hq, Hkv, d, pos0, theta, stream)
 
 
 def gqa_rope_decode_q(q, seqlens, B, H, d, theta, stream):

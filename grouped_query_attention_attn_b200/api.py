@@ -178,6 +178,19 @@ def rope_(x, pos0=0, theta=10000.0):
     return x
 
 
+def rope_qk_(q, k, pos0=0, theta=10000.0):
+    """RoPE of bf16 q [B, T, Hq, d] and k [B, T, Hkv, d] in place, in one launch
+    (row t of both at position pos0 + t).  Returns (q, k)."""
+    _need(q, "q", torch.bfloat16, 4)
+    _need(k, "k", torch.bfloat16, 4)
+    B, T, Hq, d = q.shape
+    if k.shape[0] != B or k.shape[1] != T or k.shape[3] != d:
+        raise ValueError(f"k shape {tuple(k.shape)} does not match q {tuple(q.shape)}")
+    _check(_b.gqa_rope_qk(q.data_ptr(), k.data_ptr(), B, T, Hq, k.shape[2], d, int(pos0),
+                          float(theta), _stream(q)), "gqa_rope_qk")
+    return q, k
+
+
 def rope_decode_q_(q, seqlens, theta=10000.0):
     """RoPE of bf16 decode queries [B, H, d] in place, sequence b at position seqlens[b] - 1."""
     _need(q, "q", torch.bfloat16, 3)

@@ -1,10 +1,17 @@
-// rope.cu -- rotary position embedding of q or k, in place, bf16.
+// rope.cu -- rotary position embedding of q and k, in place, bf16.
 //
 // Course "Неделя 7. Внимание", step 3: coordinate pair (2i, 2i+1) of the row at
 // position m is rotated by the angle m * theta_i, theta_i = theta^(-2i/d); only q
-// and k rotate.  HBM-bound: each thread moves 16-byte vectors (4 pairs).  The
-// angle m * theta_i reaches ~10^4 rad at long context, so it is formed and
-// reduced modulo 2 pi in double before the fp32 sine and cosine.
+// and k rotate.  HBM-bound (one read and one write of each element), so the
+// arithmetic is arranged to stay far below the memory time:
+//   * thread (c8, slot) of a block owns 16-byte column c8 (pairs 4 c8 .. 4 c8 + 3)
+//     of one token, computes those four sine / cosine pairs once and applies them
+//     to that column of every head of q and of k: one sincos per head row of
+//     eight pairs, no integer division in the loop;
+//   * the angle m * theta_i reaches ~10^4 rad at long context, so the number of
+//     turns m * theta_i / (2 pi) is formed and reduced to [-1/2, 1/2] in double,
+//     then sincospif gives the fp32 sine and cosine of 2 pi times that fraction;
+//   * loads are issued in batches of kBatch head rows before any store.
 #include <cuda_bf16.h>
 
 #include "device.cuh"
@@ -13,65 +20,93 @@
 namespace gqa {
 
 constexpr int kRopeMaxHalf = 128;    // d <= 256
+constexpr int kRopeThreads = 256;
+constexpr int kRopeBatch = 8;
 
-// x viewed as [B, T, H, d]; row (b, t) sits at position pos0 + t, or at
-// seqlens[b] - 1 when seqlens is given (decode queries, T = 1).
-__global__ void __launch_bounds__(256)
-rope_kernel(uint4 *__restrict__ x, size_t n_vec, int T, int H, int d, int pos0,
-            const int32_t *__restrict__ seqlens, double log_theta) {
-    __shared__ double inv_freq[kRopeMaxHalf];
-    for (int i = threadIdx.x; i < d / 2; i += blockDim.x)
-        inv_freq[i] = exp(-2.0 * i / d * log_theta);
-    __syncthreads();
-    const int d8 = d / 8;
-    const double two_pi = 6.283185307179586476925286766559;
-    const size_t stride = static_cast<size_t>(gridDim.x) * blockDim.x;
-    for (size_t v = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; v < n_vec;
-         v += stride) {
-        const int c8 = static_cast<int>(v % d8);
-        const size_t row = v / d8;                 // (b * T + t) * H + h
-        const size_t bt = row / H;
-        const int t = static_cast<int>(bt % T);
-        const int b = static_cast<int>(bt / T);
-        const int m = seqlens ? max(seqlens[b] - 1, 0) : pos0 + t;
-        uint4 w = x[v];
-        uint32_t *wp = reinterpret_cast<uint32_t *>(&w);
+__device__ __forceinline__ uint32_t rotate_pair(uint32_t w, float cs, float sn) {
+    const float2 a = bf16x2_to_float2(w);
+    return pack_bf16x2(a.x * cs - a.y * sn, a.x * sn + a.y * cs);
+}
+
+// Rotates column c8 of H head rows starting at row (head-row units of d8 vectors).
+__device__ __forceinline__ void rope_rows(uint4 *__restrict__ row0, int H, int d8,
+                                          const float (&cs)[4], const float (&sn)[4]) {
+    for (int h0 = 0; h0 < H; h0 += kRopeBatch) {
+        uint4 w[kRopeBatch];
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            const int i = c8 * 4 + e;              // pair index
-            const double ang = static_cast<double>(m) * inv_freq[i];
-            const double red = ang - two_pi * rint(ang / two_pi);
-            float sn, cs;
-            sincosf(static_cast<float>(red), &sn, &cs);
-            const float2 a = bf16x2_to_float2(wp[e]);
-            wp[e] = pack_bf16x2(a.x * cs - a.y * sn, a.x * sn + a.y * cs);
+        for (int j = 0; j < kRopeBatch; ++j)
+            if (h0 + j < H) w[j] = row0[static_cast<size_t>(h0 + j) * d8];
+#pragma unroll
+        for (int j = 0; j < kRopeBatch; ++j) {
+            if (h0 + j < H) {
+                w[j].x = rotate_pair(w[j].x, cs[0], sn[0]);
+                w[j].y = rotate_pair(w[j].y, cs[1], sn[1]);
+                w[j].z = rotate_pair(w[j].z, cs[2], sn[2]);
+                w[j].w = rotate_pair(w[j].w, cs[3], sn[3]);
+                row0[static_cast<size_t>(h0 + j) * d8] = w[j];
+            }
         }
-        x[v] = w;
     }
 }
 
-static int launch_rope(void *x, int B, int T, int H, int d, int pos0, const int32_t *seqlens,
-                       float theta, cudaStream_t stream) {
-    const size_t n_vec = static_cast<size_t>(B) * T * H * (d / 8);
-    int blocks = static_cast<int>((n_vec + 255) / 256);
-    if (blocks > 148 * 16) blocks = 148 * 16;
-    rope_kernel<<<blocks, 256, 0, stream>>>(static_cast<uint4 *>(x), n_vec, T, H, d, pos0, seqlens,
-                                            log(static_cast<double>(theta)));
+// x0 [n_tok, H0, d], x1 [n_tok, H1, d] (x1 may be absent, H1 = 0); token tok =
+// b * T + t sits at position pos0 + t, or at max(seqlens[b] - 1, 0) when seqlens
+// is given (decode queries, T = 1).  blockDim = (d8, slots): one token per slot.
+__global__ void __launch_bounds__(kRopeThreads)
+rope_kernel(uint4 *__restrict__ x0, int H0, uint4 *__restrict__ x1, int H1, int n_tok, int T,
+            int pos0, const int32_t *__restrict__ seqlens, double log_theta) {
+    __shared__ double turns[kRopeMaxHalf];         // theta_i / (2 pi)
+    const int d8 = blockDim.x, half = 4 * d8;
+    const int tid = threadIdx.y * d8 + threadIdx.x;
+    for (int i = tid; i < half; i += d8 * blockDim.y)
+        turns[i] = exp(-static_cast<double>(i) / half * log_theta) *
+                   0.15915494309189533576888376337251;
+    __syncthreads();
+    const int tok = blockIdx.x * blockDim.y + threadIdx.y;
+    if (tok >= n_tok) return;
+    const int c8 = threadIdx.x;
+    const int b = tok / T;
+    const int m = seqlens ? max(seqlens[b] - 1, 0) : pos0 + (tok - b * T);
+    float cs[4], sn[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+        const double t = static_cast<double>(m) * turns[c8 * 4 + e];
+        const float fr = static_cast<float>(t - rint(t));    // in [-1/2, 1/2]
+        sincospif(2.0f * fr, &sn[e], &cs[e]);
+    }
+    rope_rows(x0 + static_cast<size_t>(tok) * H0 * d8 + c8, H0, d8, cs, sn);
+    if (x1) rope_rows(x1 + static_cast<size_t>(tok) * H1 * d8 + c8, H1, d8, cs, sn);
+}
+
+static int launch_rope(void *x0, int H0, void *x1, int H1, int B, int T, int d, int pos0,
+                       const int32_t *seqlens, float theta, cudaStream_t stream) {
+    const int d8 = d / 8;
+    const int slots = kRopeThreads / d8;
+    const long long n_tok = static_cast<long long>(B) * T;
+    const long long blocks = (n_tok + slots - 1) / slots;
+    rope_kernel<<<static_cast<unsigned>(blocks), dim3(d8, slots), 0, stream>>>(
+        static_cast<uint4 *>(x0), H0, static_cast<uint4 *>(x1), H1, static_cast<int>(n_tok), T,
+        pos0, seqlens, log(static_cast<double>(theta)));
     return check_cuda(cudaGetLastError(), "rope_kernel launch");
 }
 
-static int check_rope_args(const void *x, int B, int T, int H, int d, float theta) {
+static int check_rope_args(const void *x, const char *name, int B, int T, int H, int d,
+                           float theta) {
     if (B < 0 || T < 0 || H < 1)
-        return set_error(GQA_ERR_INVALID_ARG, "B=%d, T=%d must be >= 0 and H=%d >= 1", B, T, H);
+        return set_error(GQA_ERR_INVALID_ARG, "B=%d, T=%d must be >= 0 and %s heads=%d >= 1", B,
+                         T, name, H);
+    if (static_cast<long long>(B) * T > 0x7fffffffLL)
+        return set_error(GQA_ERR_INVALID_ARG, "B*T=%lld tokens exceeds 2^31 - 1",
+                         static_cast<long long>(B) * T);
     if (d < 8 || d % 8 != 0 || d > 2 * kRopeMaxHalf)
         return set_error(GQA_ERR_INVALID_ARG, "head dim d=%d must be a multiple of 8 in [8, 256]",
                          d);
     if (!(theta > 0.0f) || !isfinite(theta))
         return set_error(GQA_ERR_INVALID_ARG, "theta=%g must be finite and > 0", (double)theta);
     if (B > 0 && T > 0) {
-        if (!x) return set_error(GQA_ERR_INVALID_ARG, "x is NULL");
+        if (!x) return set_error(GQA_ERR_INVALID_ARG, "%s is NULL", name);
         if (reinterpret_cast<uintptr_t>(x) % 16)
-            return set_error(GQA_ERR_INVALID_ARG, "x is not 16-byte aligned");
+            return set_error(GQA_ERR_INVALID_ARG, "%s is not 16-byte aligned", name);
     }
     return GQA_OK;
 }
@@ -83,19 +118,33 @@ using namespace gqa;
 extern "C" int gqa_rope(void *x, int B, int T, int H, int d, int pos0, float theta,
                         gqa_stream_t stream) {
     clear_error();
-    if (int rc = check_rope_args(x, B, T, H, d, theta)) return rc;
+    if (int rc = check_rope_args(x, "x", B, T, H, d, theta)) return rc;
     if (B == 0 || T == 0) return GQA_OK;
     if (int rc = require_sm100()) return rc;
-    return launch_rope(x, B, T, H, d, pos0, nullptr, theta, reinterpret_cast<cudaStream_t>(stream));
+    return launch_rope(x, H, nullptr, 0, B, T, d, pos0, nullptr, theta,
+                       reinterpret_cast<cudaStream_t>(stream));
+}
+
+extern "C" int gqa_rope_qk(void *q, void *k, int B, int T, int Hq, int Hkv, int d, int pos0,
+                           float theta, gqa_stream_t stream) {
+    clear_error();
+    if (int rc = check_rope_args(q, "q", B, T, Hq, d, theta)) return rc;
+    if (int rc = check_rope_args(k, "k", B, T, Hkv, d, theta)) return rc;
+    if (B == 0 || T == 0) return GQA_OK;
+    if (q == k) return set_error(GQA_ERR_INVALID_ARG, "q and k are the same buffer");
+    if (int rc = require_sm100()) return rc;
+    return launch_rope(q, Hq, k, Hkv, B, T, d, pos0, nullptr, theta,
+                       reinterpret_cast<cudaStream_t>(stream));
 }
 
 extern "C" int gqa_rope_decode_q(void *q, const int32_t *seqlens, int B, int H, int d, float theta,
                                  gqa_stream_t stream) {
     clear_error();
-    if (int rc = check_rope_args(q, B, 1, H, d, theta)) return rc;
+    if (int rc = check_rope_args(q, "q", B, 1, H, d, theta)) return rc;
     if (B == 0) return GQA_OK;
     if (!seqlens || reinterpret_cast<uintptr_t>(seqlens) % 4)
         return set_error(GQA_ERR_INVALID_ARG, "seqlens is NULL or misaligned");
     if (int rc = require_sm100()) return rc;
-    return launch_rope(q, B, 1, H, d, 0, seqlens, theta, reinterpret_cast<cudaStream_t>(stream));
+    return launch_rope(q, H, nullptr, 0, B, 1, d, 0, seqlens, theta,
+                       reinterpret_cast<cudaStream_t>(stream));
 }

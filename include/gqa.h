@@ -224,6 +224,16 @@ int gqa_attn_bwd(const void *q, const void *k, const void *v, const void *o, con
 int gqa_rope(void *x, int B, int T, int H, int d, int pos0, float theta, gqa_stream_t stream);
 
 /*
+ * gqa_rope_qk -- gqa_rope of q [B, T, Hq, d] and k [B, T, Hkv, d] in one launch
+ * (self-attention prefill: row t of both at position pos0 + t).  Each angle is
+ * evaluated once per token and column and applied to all Hq + Hkv heads.
+ * Same argument rules as gqa_rope for each tensor; q and k must be distinct
+ * buffers (GQA_ERR_INVALID_ARG otherwise).
+ */
+int gqa_rope_qk(void *q, void *k, int B, int T, int Hq, int Hkv, int d, int pos0, float theta,
+                gqa_stream_t stream);
+
+/*
  * gqa_rope_decode_q -- gqa_rope of decode queries q [B, H, d] (bf16, in place):
  * sequence b's new token sits at position max(seqlens[b] - 1, 0) (seqlens:
  * device int32 [B]; an empty cache makes it the first token).  The cached keys are expected to be rotated already, each at

@@ -167,6 +167,11 @@ def test_rope_rejects(gqa_lib):
     assert b.gqa_rope(FAKE + 8, 1, 4, 2, 128, 0, 10000.0, NULL) == b.GQA_ERR_INVALID_ARG
     assert b.gqa_rope(NULL, 0, 4, 2, 128, 0, 10000.0, NULL) == b.GQA_OK              # empty
     assert b.gqa_rope_decode_q(FAKE, NULL, 2, 2, 128, 10000.0, NULL) == b.GQA_ERR_INVALID_ARG
+    assert b.gqa_rope_qk(FAKE, FAKE, 1, 4, 4, 2, 128, 0, 10000.0, NULL) == b.GQA_ERR_INVALID_ARG
+    assert b.gqa_rope_qk(FAKE, NULL, 1, 4, 4, 2, 128, 0, 10000.0, NULL) == b.GQA_ERR_INVALID_ARG
+    assert b.gqa_rope_qk(FAKE, FAKE + 16, 1, 4, 4, 0, 128, 0, 10000.0, NULL) == \
+        b.GQA_ERR_INVALID_ARG                                                           # Hkv
+    assert b.gqa_rope_qk(NULL, NULL, 1, 0, 4, 2, 128, 0, 10000.0, NULL) == b.GQA_OK    # empty
 
 
 def test_backward_rejects(gqa_lib):

@@ -31,6 +31,21 @@ def test_rope_matches_oracle(gqa_lib, B, T, H, d, pos0, theta):
     assert (got.cpu() == bf16_round(want)).float().mean() > 0.99
 
 
+@pytest.mark.parametrize("B,T,Hq,Hkv,d,pos0", [(2, 77, 8, 2, 128, 0), (1, 300, 32, 8, 128, 9000),
+                                              (3, 5, 3, 1, 24, 11)])
+def test_rope_qk_matches_oracle(gqa_lib, B, T, Hq, Hkv, d, pos0):
+    q = workloads.randn((B, T, Hq, d), 40 + T)
+    k = workloads.randn((B, T, Hkv, d), 41 + T)
+    gq, gk = gqa.rope_qk_(q.cuda(), k.cuda(), pos0)
+    for got, x in ((gq, q), (gk, k)):
+        want = ref.rope_tensor(x, pos0, 10000.0)
+        rel = np.abs(got.float().cpu().numpy() - want) / np.maximum(np.abs(want), 1e-30)
+        assert np.max(np.where(np.abs(want) > 1e-3, rel, 0.0)) <= 2.0 ** -8
+    # one launch over q and k gives the same bits as two separate rotations
+    assert torch.equal(gq.cpu(), gqa.rope_(q.cuda(), pos0).cpu())
+    assert torch.equal(gk.cpu(), gqa.rope_(k.cuda(), pos0).cpu())
+
+
 def test_rope_position_zero_is_identity(gqa_lib):
     x = workloads.randn((1, 1, 4, 128), 3)
     assert torch.equal(gqa.rope_(x.cuda(), 0).cpu(), x)
