@@ -100,6 +100,12 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tm_k,
         }
         return;
     }
+    // Stages holding no visible key are not loaded: the sink stages [0, t_s)
+    // and the window stages [t_w, n_stages) of the split, in that order.
+    int t_s = min(n_stages, max(0, (n_sinks - start + kDecBK - 1) / kDecBK));
+    int t_w = min(n_stages, max(0, (lo - start) / kDecBK));
+    if (t_s >= t_w) t_s = t_w = 0;                  // the two runs meet: every stage
+    const int n_iter = t_s + n_stages - t_w;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kDecStages; ++s) {
@@ -115,14 +121,14 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tm_k,
         if (lane == 0) {
             tma_prefetch_desc(&tm_k);
             tma_prefetch_desc(&tm_v);
-            for (int t = 0; t < n_stages; ++t) {
+            for (int t = 0; t < n_iter; ++t) {
                 const int st = t % kDecStages;
                 const uint32_t ph = (t / kDecStages) & 1;
                 if (!mbar_wait(&empty_bar[st], ph ^ 1, &abort_flag, status)) break;
                 uint8_t *kt = smem + st * Lay::kStageBytes;
                 uint8_t *vt = kt + Lay::kTileBytes;
                 mbar_expect_tx(&full_bar[st], Lay::kStageBytes);
-                const int j0 = start + t * kDecBK;
+                const int j0 = start + (t < t_s ? t : t_w + t - t_s) * kDecBK;
 #pragma unroll
                 for (int p = 0; p < Lay::kPanels; ++p) {
                     tma_load_4d(kt + p * Lay::kPanelBytes, &tm_k, &full_bar[st], p * 64, kvh, j0, b);
@@ -161,14 +167,15 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tm_k,
         l_run[mb][0] = l_run[mb][1] = 0.0f;
     }
 
-    for (int t = 0; t < n_stages; ++t) {
+    for (int t = 0; t < n_iter; ++t) {
         const int st = t % kDecStages;
         const uint32_t ph = (t / kDecStages) & 1;
         // warp-uniform outcome: ldmatrix and mma.sync below are warp-collective
         if (!__all_sync(0xffffffffu, mbar_wait(&full_bar[st], ph, &abort_flag, status))) break;
         uint8_t *kt = smem + st * Lay::kStageBytes;
         uint8_t *vt = kt + Lay::kTileBytes;
-        const int key0 = start + t * kDecBK + warp * 16;  // first key of this warp's slice
+        const int stage = t < t_s ? t : t_w + t - t_s;
+        const int key0 = start + stage * kDecBK + warp * 16;  // first key of this warp's slice
         const int n_valid = end - key0;                   // keys of the slice inside the split
         const bool partial = n_valid > 0 && n_valid < 16;
         if (partial) {

@@ -63,6 +63,23 @@ int require_sm100() {
     return GQA_OK;
 }
 
+int sm_count(int *n) {
+    static int cache[64] = {};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return check_cuda(e, "cudaGetDevice");
+    if (dev < 0 || dev >= 64) return set_error(GQA_ERR_UNSUPPORTED, "device index %d", dev);
+    if (!cache[dev]) {
+        int v = 0;
+        if (int rc = check_cuda(cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev),
+                                "cudaDeviceGetAttribute(SM count)"))
+            return rc;
+        cache[dev] = v;
+    }
+    *n = cache[dev];
+    return GQA_OK;
+}
+
 using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
                                    const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
                                    const cuuint32_t *, CUtensorMapInterleave,

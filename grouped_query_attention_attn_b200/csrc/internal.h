@@ -21,6 +21,8 @@ int check_cuda(cudaError_t e, const char *what);
 
 // GQA_OK when the current device is an sm_100 part, else GQA_ERR_UNSUPPORTED.
 int require_sm100();
+// Number of SMs of the current device (cached per device).
+int sm_count(int *n);
 
 // Device address of the library's status word on the current device
 // (looked up once per device); nullptr with a message set on failure.

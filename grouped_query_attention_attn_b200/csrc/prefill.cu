@@ -26,6 +26,7 @@
 // is safe because the commit that signals S_k(j) also covers PV_k(j-1).
 #include <cuda_bf16.h>
 #include <climits>
+#include <cstdlib>
 
 #include "device.cuh"
 #include "internal.h"
@@ -90,6 +91,54 @@ __device__ __forceinline__ void softmax_chunk(const uint32_t (&s)[32], float2 cc
     }
 }
 
+// One work unit: a (batch, KV head) and two adjacent M tiles (256 rows), with
+// the KV tiles its rows can see.
+struct PfUnit {
+    int b, kvh, t0;             // t0: first position of M tile 0
+    int n_kv;                   // KV tiles visited
+    int n_sink_tiles, first_tile;
+    // KV tiles are visited in order: the sink tiles, then the window tiles
+    // (every tile below the causal limit when there is no window).
+    __device__ __forceinline__ int tile(int j) const {
+        return j < n_sink_tiles ? j : first_tile + (j - n_sink_tiles);
+    }
+};
+
+// The i-th unit of this CTA.  Units are ranked by decreasing causal work
+// (the last position pairs first); round i hands ranks [i g, (i + 1) g) to
+// the g CTAs, in reverse order on odd rounds, which balances the rounds'
+// decreasing costs across CTAs.  Returns false past the last unit.
+__device__ __forceinline__ bool pf_unit(const PfParams &p, int i, PfUnit &u) {
+    const int g = gridDim.x, c = blockIdx.x;
+    const long long rank = static_cast<long long>(i) * g + ((i & 1) ? g - 1 - c : c);
+    const int bhs = p.B * p.Hkv;
+    if (rank >= static_cast<long long>(p.n_pairs) * bhs) return false;
+    const int r = static_cast<int>(rank);
+    const int bh = r % bhs;
+    const int pair = p.n_pairs - 1 - r / bhs;
+    u.b = bh / p.Hkv;
+    u.kvh = bh % p.Hkv;
+    u.t0 = pair * 2 * p.P;
+    const int last_pos = min(u.t0 + 2 * p.P, p.Tq) - 1;    // last real position in the pair
+    int kv_end = p.Tkv;                                      // keys [0, kv_end) can be visible
+    if (p.causal) kv_end = min(p.Tkv, last_pos + (p.Tkv - p.Tq) + 1);
+    u.n_sink_tiles = 0;
+    u.first_tile = 0;
+    if (p.window > 0 && kv_end > 0) {
+        const int lo_min = u.t0 + (p.Tkv - p.Tq) - p.window + 1;   // window start, first row
+        u.n_sink_tiles = (min(p.sinks, kv_end) + kPfBN - 1) / kPfBN;
+        u.first_tile = max(u.n_sink_tiles, max(lo_min, 0) / kPfBN);
+    }
+    const int last_tile = kv_end > 0 ? (kv_end + kPfBN - 1) / kPfBN : 0;   // exclusive
+    u.n_kv = u.n_sink_tiles + max(0, last_tile - u.first_tile);
+    return true;
+}
+
+// Persistent kernel: one CTA per SM walks its units; the roles below stream
+// across unit boundaries, so the next unit's Q load and first MMAs overlap
+// the current unit's epilogue.  Iteration counters run over all units of the
+// CTA (ring stages and barrier phases), unit counters over units with at
+// least one KV tile.
 template <int D>
 __global__ void __launch_bounds__(kPfThreads, 1)
 prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -98,39 +147,18 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-    __shared__ uint64_t q_full, k_full[kPfStages], k_empty[kPfStages], v_full[kPfStages],
-        v_empty[kPfStages], s_full[2], p_full[2], o_done[2], mma_drain;
+    __shared__ uint64_t q_full[2], q_empty[2], k_full[kPfStages], k_empty[kPfStages],
+        v_full[kPfStages], v_empty[kPfStages], s_full[2], p_full[2], o_done[2], o_free[2],
+        mma_drain;
     __shared__ uint32_t tmem_base_sh;
     // row-max / l exchange between the two warps that share rows:
-    // [phase parity][tile][half][row]
+    // [exchange parity][tile][half][row]
     __shared__ float xchg[2][2][2][kPfBM];
     __shared__ int abort_flag;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-    // ---- work unit: longest causal tiles first ----
-    const int bh = blockIdx.x % (p.B * p.Hkv);
-    const int pair = p.n_pairs - 1 - blockIdx.x / (p.B * p.Hkv);
-    const int b = bh / p.Hkv, kvh = bh % p.Hkv;
-    const int t0 = pair * 2 * p.P;                      // first position of M tile 0
-    const int last_pos = min(t0 + 2 * p.P, p.Tq) - 1;   // last real position in the pair
-    int kv_end = p.Tkv;                                 // keys [0, kv_end) can be visible
-    if (p.causal) kv_end = min(p.Tkv, last_pos + (p.Tkv - p.Tq) + 1);
-    // KV tiles visited, in order: the sink tiles, then the window tiles (all
-    // tiles below kv_end when there is no window); tile_of(j) maps the
-    // visiting order to the tile index.
-    int n_sink_tiles = 0, first_tile = 0;
-    if (p.window > 0 && kv_end > 0) {
-        const int lo_min = t0 + (p.Tkv - p.Tq) - p.window + 1;   // window start, first row
-        n_sink_tiles = (min(p.sinks, kv_end) + kPfBN - 1) / kPfBN;
-        first_tile = max(n_sink_tiles, max(lo_min, 0) / kPfBN);
-    }
-    const int last_tile = kv_end > 0 ? (kv_end + kPfBN - 1) / kPfBN : 0;  // exclusive
-    const int n_kv = n_sink_tiles + max(0, last_tile - first_tile);
-    auto tile_of = [&](int j) { return j < n_sink_tiles ? j : first_tile + (j - n_sink_tiles); };
-
     if (threadIdx.x == 0) {
-        mbar_init(&q_full, 1);
         for (int s = 0; s < kPfStages; ++s) {
             mbar_init(&k_full[s], 1);
             mbar_init(&k_empty[s], 1);
@@ -138,9 +166,12 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             mbar_init(&v_empty[s], 1);
         }
         for (int k = 0; k < 2; ++k) {
+            mbar_init(&q_full[k], 1);
+            mbar_init(&q_empty[k], 1);
             mbar_init(&s_full[k], 1);
             mbar_init(&p_full[k], 8);   // every softmax warp of the tile
             mbar_init(&o_done[k], 1);
+            mbar_init(&o_free[k], 8);
         }
         mbar_init(&mma_drain, 1);
         abort_flag = 0;
@@ -163,154 +194,188 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         // ------------------------------------------------ TMA producer ----
         // The whole warp runs the schedule (barrier waits stay warp-uniform);
         // one elected lane issues the copies.
-        if (n_kv > 0) {
-            const bool leader = elect_one();
-            if (leader) {
-                tma_prefetch_desc(&tm_q);
-                tma_prefetch_desc(&tm_k);
-                tma_prefetch_desc(&tm_v);
-                const int q_box_bytes = 64 * p.G * p.P * 2;
-                mbar_expect_tx(&q_full, 2 * Lay::kPanels * q_box_bytes);
-                for (int mt = 0; mt < 2; ++mt)
+        const bool leader = elect_one();
+        if (leader) {
+            tma_prefetch_desc(&tm_q);
+            tma_prefetch_desc(&tm_k);
+            tma_prefetch_desc(&tm_v);
+        }
+        const uint32_t q_box_bytes = 64u * p.G * p.P * 2u;
+        int gi = 0, ui = 0;         // iterations issued, active units started
+        bool ok = true;
+        PfUnit u;
+        for (int i = 0; ok && pf_unit(p, i, u); ++i) {
+            if (u.n_kv == 0) continue;
+            for (int k = 0; k < 2; ++k) {           // Q tile k, once S_k of the last unit is done
+                if (ui > 0 && !(ok = __all_sync(0xffffffffu, mbar_wait(&q_empty[k], (ui - 1) & 1,
+                                                                        &abort_flag, p.status))))
+                    break;
+                if (leader) {
+                    mbar_expect_tx(&q_full[k], Lay::kPanels * q_box_bytes);
                     for (int pn = 0; pn < Lay::kPanels; ++pn)
-                        tma_load_4d(sQ + mt * Lay::kQTile + pn * Lay::kQPanel, &tm_q, &q_full,
-                                    pn * 64, kvh * p.G, t0 + mt * p.P, b);
+                        tma_load_4d(sQ + k * Lay::kQTile + pn * Lay::kQPanel, &tm_q, &q_full[k],
+                                    pn * 64, u.kvh * p.G, u.t0 + k * p.P, u.b);
+                }
+                __syncwarp();
             }
-            __syncwarp();
-            int issued = 0;
-            for (int j = 0; j < n_kv; ++j) {
-                const int st = j % kPfStages;
-                const uint32_t ph = (j / kPfStages) & 1;
-                if (!__all_sync(0xffffffffu, mbar_wait(&k_empty[st], ph ^ 1, &abort_flag, p.status)))
+            ++ui;
+            for (int j = 0; ok && j < u.n_kv; ++j) {
+                const int st = gi % kPfStages;
+                const uint32_t ph = (gi / kPfStages) & 1;
+                const int row = u.tile(j) * kPfBN;
+                if (!(ok = __all_sync(0xffffffffu,
+                                      mbar_wait(&k_empty[st], ph ^ 1, &abort_flag, p.status))))
                     break;
                 if (leader) {
                     mbar_expect_tx(&k_full[st], Lay::kKTile);
                     for (int pn = 0; pn < Lay::kPanels; ++pn)
                         tma_load_4d(sK + st * Lay::kKTile + pn * Lay::kKPanel, &tm_k, &k_full[st],
-                                    pn * 64, kvh, tile_of(j) * kPfBN, b);
+                                    pn * 64, u.kvh, row, u.b);
                 }
                 __syncwarp();
-                issued = j + 1;
-                if (!__all_sync(0xffffffffu, mbar_wait(&v_empty[st], ph ^ 1, &abort_flag, p.status)))
+                if (!(ok = __all_sync(0xffffffffu,
+                                      mbar_wait(&v_empty[st], ph ^ 1, &abort_flag, p.status)))) {
+                    ++gi;                           // K of this iteration is in flight
                     break;
+                }
                 if (leader) {
                     mbar_expect_tx(&v_full[st], Lay::kKTile);
                     for (int pn = 0; pn < Lay::kPanels; ++pn)
                         tma_load_4d(sV + st * Lay::kKTile + pn * Lay::kKPanel, &tm_v, &v_full[st],
-                                    pn * 64, kvh, tile_of(j) * kPfBN, b);
+                                    pn * 64, u.kvh, row, u.b);
                 }
                 __syncwarp();
+                ++gi;
             }
-            if (abort_flag) {
-                // let copies already in flight land before the block exits
-                for (int j = max(0, issued - kPfStages); j < issued; ++j) {
-                    const int st = j % kPfStages;
-                    const uint32_t ph = (j / kPfStages) & 1;
-                    mbar_wait(&k_full[st], ph, &abort_flag, p.status, 1000000ull);
-                    mbar_wait(&v_full[st], ph, &abort_flag, p.status, 1000000ull);
-                }
+        }
+        if (!ok) {
+            // let copies that may be in flight land before the block exits
+            for (int g = max(0, gi - kPfStages); g < gi; ++g) {
+                const int st = g % kPfStages;
+                const uint32_t ph = (g / kPfStages) & 1;
+                mbar_wait(&k_full[st], ph, &abort_flag, p.status, 1000000ull);
+                mbar_wait(&v_full[st], ph, &abort_flag, p.status, 1000000ull);
             }
+            if (ui > 0)
+                for (int k = 0; k < 2; ++k)
+                    mbar_wait(&q_full[k], (ui - 1) & 1, &abort_flag, p.status, 1000000ull);
         }
     } else if (warp == 1) {
         // ------------------------------------------------- MMA issuer ----
         // The whole warp follows the schedule; one elected lane issues every
         // tcgen05.mma and tcgen05.commit (a commit tracks its own thread's MMAs).
-        if (n_kv > 0) {
-            const bool leader = elect_one();
-            constexpr uint32_t idesc_s = umma_idesc_bf16(kPfBM, kPfBN, 0, 0);
-            constexpr uint32_t idesc_o = umma_idesc_bf16(kPfBM, D, 0, 1);
-            const uint32_t sQa = smem_u32(sQ), sKa = smem_u32(sK), sVa = smem_u32(sV);
-            bool ok = __all_sync(0xffffffffu, mbar_wait(&q_full, 0, &abort_flag, p.status));
+        // Step g issues PV_0(g-1), S_0(g), PV_1(g-1), S_1(g) over the flattened
+        // iterations of all units, so the two tiles keep alternating on the
+        // tensor pipe across unit boundaries.
+        const bool leader = elect_one();
+        constexpr uint32_t idesc_s = umma_idesc_bf16(kPfBM, kPfBN, 0, 0);
+        constexpr uint32_t idesc_o = umma_idesc_bf16(kPfBM, D, 0, 1);
+        const uint32_t sQa = smem_u32(sQ), sKa = smem_u32(sK), sVa = smem_u32(sV);
+        // Descriptors are built once; stepping along K only moves the start
+        // address field (low bits, 16-byte units): +32 B per 16 elements
+        // inside a 64-column panel of Q / K, +2048 B per 16 keys of V.
+        static_assert(kPfStages == 2, "descriptor selects assume a 2-deep ring");
+        const uint64_t dq0 = umma_smem_desc(sQa, 16, 1024);
+        const uint64_t dq1 = umma_smem_desc(sQa + Lay::kQTile, 16, 1024);
+        const uint64_t dk0 = umma_smem_desc(sKa, 16, 1024);
+        const uint64_t dk1 = umma_smem_desc(sKa + Lay::kKTile, 16, 1024);
+        const uint64_t dv0 = umma_smem_desc(sVa, Lay::kKPanel, 1024);
+        const uint64_t dv1 = umma_smem_desc(sVa + Lay::kKTile, Lay::kKPanel, 1024);
+        // S_k = Q_k K_st^T : K-major A and B, 16 elements of d per instruction
+        auto issue_s = [&](int k, int st) {
+            const uint32_t ts = tmem + (k ? Lay::kColS1 : Lay::kColS0);
+            const uint64_t a = k ? dq1 : dq0, bk = st ? dk1 : dk0;
+            if (leader) {
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint32_t off = ((kk >> 2) * Lay::kQPanel + (kk & 3) * 32) >> 4;
+                    umma_ss(ts, a + off, bk + off, idesc_s, kk > 0);
+                }
+            }
+            __syncwarp();
+        };
+        // O_k (+)= P_k V_st : P from tensor memory, V MN-major (d contiguous)
+        auto issue_pv = [&](int k, int st, bool acc) {
+            const uint32_t ts = tmem + (k ? Lay::kColS1 : Lay::kColS0);
+            const uint32_t to = tmem + (k ? Lay::kColO1 : Lay::kColO0);
+            const uint64_t bv = st ? dv1 : dv0;
+            if (leader) {
+#pragma unroll
+                for (int kk = 0; kk < kPfBN / 16; ++kk)
+                    umma_ts(to, ts + kk * 8, bv + kk * (2048 >> 4), idesc_o,
+                            (acc || kk > 0) ? 1u : 0u);
+            }
+            __syncwarp();
+        };
+        auto commit = [&](uint64_t *bar) {
+            if (leader) tc_commit(bar);
+            __syncwarp();
+        };
+        auto wait_all = [&](uint64_t *bar, uint32_t parity) {
+            return __all_sync(0xffffffffu, mbar_wait(bar, parity, &abort_flag, p.status));
+        };
+        // PV_k of the previous step: its P, and for a unit's first PV (which
+        // overwrites O_k) the previous unit's epilogue read of O_k.
+        int pv_st = 0, pv_j = 0, pv_n = 0, pv_ui = 0, pv_gi = 0;
+        bool pv_pending = false;
+        auto pv_step = [&](int k) {
+            if (!wait_all(&p_full[k], pv_gi & 1)) return false;
+            if (pv_j == 0 && pv_ui > 0 && !wait_all(&o_free[k], (pv_ui - 1) & 1)) return false;
             tc_fence_after();
-            // Descriptors are built once; stepping along K only moves the start
-            // address field (low bits, 16-byte units): +32 B per 16 elements
-            // inside a 64-column panel of Q / K, +2048 B per 16 keys of V.
-            static_assert(kPfStages == 2, "descriptor selects assume a 2-deep ring");
-            const uint64_t dq0 = umma_smem_desc(sQa, 16, 1024);
-            const uint64_t dq1 = umma_smem_desc(sQa + Lay::kQTile, 16, 1024);
-            const uint64_t dk0 = umma_smem_desc(sKa, 16, 1024);
-            const uint64_t dk1 = umma_smem_desc(sKa + Lay::kKTile, 16, 1024);
-            const uint64_t dv0 = umma_smem_desc(sVa, Lay::kKPanel, 1024);
-            const uint64_t dv1 = umma_smem_desc(sVa + Lay::kKTile, Lay::kKPanel, 1024);
-            // S_k = Q_k K_st^T : K-major A and B, 16 elements of d per instruction
-            auto issue_s = [&](int k, int st) {
-                const uint32_t ts = tmem + (k ? Lay::kColS1 : Lay::kColS0);
-                const uint64_t a = k ? dq1 : dq0, bk = st ? dk1 : dk0;
-                if (leader) {
-#pragma unroll
-                    for (int kk = 0; kk < D / 16; ++kk) {
-                        const uint32_t off = ((kk >> 2) * Lay::kQPanel + (kk & 3) * 32) >> 4;
-                        umma_ss(ts, a + off, bk + off, idesc_s, kk > 0);
-                    }
-                }
-                __syncwarp();
-            };
-            // O_k (+)= P_k V_st : P from tensor memory, V MN-major (d contiguous)
-            auto issue_pv = [&](int k, int st, bool acc) {
-                const uint32_t ts = tmem + (k ? Lay::kColS1 : Lay::kColS0);
-                const uint32_t to = tmem + (k ? Lay::kColO1 : Lay::kColO0);
-                const uint64_t bv = st ? dv1 : dv0;
-                if (leader) {
-#pragma unroll
-                    for (int kk = 0; kk < kPfBN / 16; ++kk)
-                        umma_ts(to, ts + kk * 8, bv + kk * (2048 >> 4), idesc_o,
-                                (acc || kk > 0) ? 1u : 0u);
-                }
-                __syncwarp();
-            };
-            auto commit = [&](uint64_t *bar) {
-                if (leader) tc_commit(bar);
-                __syncwarp();
-            };
-            auto wait_all = [&](uint64_t *bar, uint32_t parity) {
-                return __all_sync(0xffffffffu, mbar_wait(bar, parity, &abort_flag, p.status));
-            };
-            for (int j = 0; ok && j < n_kv; ++j) {
-                const int st = j % kPfStages;
-                const uint32_t ph = (j / kPfStages) & 1;
-                const int sp = (j + kPfStages - 1) % kPfStages;          // stage of tile j-1
-                const uint32_t php = ((j - 1) / kPfStages) & 1;
+            issue_pv(k, pv_st, pv_j > 0);
+            if (pv_j == pv_n - 1) commit(&o_done[k]);
+            return true;
+        };
+        int gi = 0, ui = 0;
+        bool ok = true;
+        PfUnit u;
+        for (int i = 0; ok && pf_unit(p, i, u); ++i) {
+            if (u.n_kv == 0) continue;
+            for (int j = 0; j < u.n_kv; ++j) {
+                const int st = gi % kPfStages;
+                const uint32_t ph = (gi / kPfStages) & 1;
                 if (!(ok = wait_all(&k_full[st], ph))) break;
-                tc_fence_after();
-                if (j > 0) {
-                    if (!(ok = wait_all(&v_full[sp], php))) break;
-                    if (!(ok = wait_all(&p_full[0], (j - 1) & 1))) break;
-                    tc_fence_after();
-                    issue_pv(0, sp, j > 1);
+                if (pv_pending && !(ok = wait_all(&v_full[pv_st], (pv_gi / kPfStages) & 1))) break;
+                if (pv_pending && !(ok = pv_step(0))) break;
+                // at a unit boundary the last PV_1 goes first: it must not wait
+                // for the new unit's Q tiles
+                if (pv_pending && j == 0) {
+                    if (!(ok = pv_step(1))) break;
+                    commit(&v_empty[pv_st]);
+                    pv_pending = false;
                 }
+                if (j == 0 && !(ok = wait_all(&q_full[0], ui & 1))) break;
+                tc_fence_after();
                 issue_s(0, st);
                 commit(&s_full[0]);
-                if (j > 0) {
-                    if (!(ok = wait_all(&p_full[1], (j - 1) & 1))) break;
-                    tc_fence_after();
-                    issue_pv(1, sp, j > 1);
-                    commit(&v_empty[sp]);
+                if (j == u.n_kv - 1) commit(&q_empty[0]);
+                if (pv_pending) {
+                    if (!(ok = pv_step(1))) break;
+                    commit(&v_empty[pv_st]);
                 }
+                if (j == 0 && !(ok = wait_all(&q_full[1], ui & 1))) break;
+                tc_fence_after();
                 issue_s(1, st);
                 commit(&s_full[1]);
                 commit(&k_empty[st]);
+                if (j == u.n_kv - 1) commit(&q_empty[1]);
+                pv_st = st;
+                pv_j = j;
+                pv_n = u.n_kv;
+                pv_ui = ui;
+                pv_gi = gi;
+                pv_pending = true;
+                ++gi;
             }
-            if (ok) {
-                const int sl = (n_kv - 1) % kPfStages;
-                const uint32_t phl = ((n_kv - 1) / kPfStages) & 1;
-                ok = wait_all(&v_full[sl], phl) && wait_all(&p_full[0], (n_kv - 1) & 1);
-                if (ok) {
-                    tc_fence_after();
-                    issue_pv(0, sl, n_kv > 1);
-                    commit(&o_done[0]);
-                    ok = wait_all(&p_full[1], (n_kv - 1) & 1);
-                }
-                if (ok) {
-                    tc_fence_after();
-                    issue_pv(1, sl, n_kv > 1);
-                    commit(&o_done[1]);
-                    commit(&v_empty[sl]);
-                }
-            }
-            // every MMA this warp issued has finished before tensor memory is freed
-            commit(&mma_drain);
-            mbar_wait(&mma_drain, 0, &abort_flag, p.status, 1000000000ull);
+            ++ui;
         }
+        if (ok && pv_pending) {
+            ok = wait_all(&v_full[pv_st], (pv_gi / kPfStages) & 1) && pv_step(0) && pv_step(1);
+            if (ok) commit(&v_empty[pv_st]);
+        }
+        // every MMA this warp issued has finished before tensor memory is freed
+        commit(&mma_drain);
+        mbar_wait(&mma_drain, 0, &abort_flag, p.status, 1000000000ull);
     } else if (warp >= 4) {
         // -------------------------------------------- softmax + epilogue ----
         // Two threads per row: warps 4-11 serve M tile 0, warps 12-19 M tile 1;
@@ -326,172 +391,201 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         const uint32_t colO = (k ? Lay::kColO1 : Lay::kColO0) + (D / 2) * h;
         const int bar_id = 1 + k * 4 + g4;              // the two warps sharing these rows
         // Publish a value for my row and take the other half's.  Both warps of
-        // the pair reach every exchange (the loop's continue / abort decision is
-        // taken jointly from the exchanged values), so the hardware barrier
-        // always completes.  Slots alternate by phase so a fast warp cannot
-        // overwrite a value its partner has not read yet.
-        auto exchange = [&](float mine, uint32_t ph, float &other) {
-            xchg[ph][k][h][r] = mine;
+        // the pair make the same sequence of exchanges (every continue / abort
+        // decision is taken jointly from exchanged values), so the hardware
+        // barrier always completes.  Slots alternate by exchange so a fast
+        // warp cannot overwrite a value its partner has not read yet.
+        int xc = 0;
+        auto exchange = [&](float mine, float &other) {
+            const int slot = xc & 1;
+            ++xc;
+            xchg[slot][k][h][r] = mine;
             named_barrier_sync(bar_id, 64);
-            other = xchg[ph][k][h ^ 1][r];
+            other = xchg[slot][k][h ^ 1][r];
         };
-        const int pos = t0 + k * p.P + r / p.G;
-        const int head = kvh * p.G + r % p.G;
-        const bool row_real = (r < p.P * p.G) && (pos < p.Tq);
-        // visible keys of this row: key <= lim, and key >= lo or key < sinks
-        // (keys past Tkv never count; lo / sinks only with a sliding window)
-        int lim = p.Tkv - 1;
-        if (p.causal && row_real) lim = min(lim, pos + (p.Tkv - p.Tq));
-        const int lo = (p.window > 0 && row_real) ? pos + (p.Tkv - p.Tq) - p.window + 1 : INT_MIN;
-        const int n_sinks = p.window > 0 ? p.sinks : 0;
-        // Online softmax with a lazily moved reference max: O and l stay scaled
-        // by exp2(-m_ref) and m_ref only moves when a row's max exceeds it by
-        // more than kRescaleLog2 (P then stays <= 2^kRescaleLog2).  Exact in
-        // real arithmetic: the epilogue divides by l taken at the same m_ref.
-        // Both halves of a row see the same row max, so they take identical
-        // m_ref / alpha decisions; each keeps the partial l of its columns.
-        float m_ref = -INFINITY, l_run = 0.0f;
+        const float kAbortMark = __int_as_float(0x7fc00001);   // a NaN no max can produce
+        auto is_abort = [](float x) { return __float_as_int(x) == 0x7fc00001; };
         const float c2 = p.scale_log2;
+        const int n_sinks = p.window > 0 ? p.sinks : 0;
+        int gi = 0, ui = 0;
         bool ok = true;
-        for (int j = 0; j < n_kv; ++j) {
-            // warp-uniform outcome: the tensor-memory accesses below are .sync.aligned
-            ok = __all_sync(0xffffffffu, mbar_wait(&s_full[k], j & 1, &abort_flag, p.status));
-            if (!ok) {
-                float dummy;
-                exchange(__int_as_float(0x7fc00001), j & 1, dummy);   // tell the partner
-                break;
+        PfUnit u;
+        for (int i = 0; ok && pf_unit(p, i, u); ++i) {
+            const int pos = u.t0 + k * p.P + r / p.G;
+            const int head = u.kvh * p.G + r % p.G;
+            const bool row_real = (r < p.P * p.G) && (pos < p.Tq);
+            __nv_bfloat16 *dst =
+                p.o + ((static_cast<size_t>(u.b) * p.Tq + pos) * p.Hq + head) * D + (D / 2) * h;
+            float *lse_dst = p.lse ? p.lse + (static_cast<size_t>(u.b) * p.Hq + head) * p.Tq + pos
+                                   : nullptr;
+            if (u.n_kv == 0) {
+                // no visible key for any row of the unit: o = 0, lse = -inf
+                if (row_real) {
+#pragma unroll
+                    for (int e = 0; e < D / 16; ++e)
+                        reinterpret_cast<uint4 *>(dst)[e] = make_uint4(0u, 0u, 0u, 0u);
+                    if (lse_dst && h == 0) *lse_dst = -INFINITY;
+                }
+                continue;
             }
-            tc_fence_after();
-            uint32_t sr[2][32];
-            tmem_ld32(lane_addr + colS, sr[0]);
-            tmem_ld32(lane_addr + colS + 32, sr[1]);
-            tmem_wait_ld();
-            const int key0 = tile_of(j) * kPfBN + 64 * h;   // key of my first column
-            const bool masked = __any_sync(0xffffffffu, key0 + 63 > lim ||
-                                                            (key0 < lo && key0 + 63 >= n_sinks));
-            if (masked) {
+            // visible keys of this row: key <= lim, and key >= lo or key < sinks
+            // (keys past Tkv never count; lo / sinks only with a sliding window)
+            int lim = p.Tkv - 1;
+            if (p.causal && row_real) lim = min(lim, pos + (p.Tkv - p.Tq));
+            const int lo =
+                (p.window > 0 && row_real) ? pos + (p.Tkv - p.Tq) - p.window + 1 : INT_MIN;
+            // Online softmax with a lazily moved reference max: O and l stay
+            // scaled by exp2(-m_ref) and m_ref only moves when a row's max
+            // exceeds it by more than kRescaleLog2 (P then stays <=
+            // 2^kRescaleLog2).  Exact in real arithmetic: the epilogue divides
+            // by l taken at the same m_ref.  Both halves of a row see the same
+            // row max, so they take identical m_ref / alpha decisions; each
+            // keeps the partial l of its columns.
+            float m_ref = -INFINITY, l_run = 0.0f;
+            for (int j = 0; j < u.n_kv; ++j, ++gi) {
+                // warp-uniform outcome: the tensor-memory accesses below are .sync.aligned
+                ok = __all_sync(0xffffffffu, mbar_wait(&s_full[k], gi & 1, &abort_flag, p.status));
+                if (!ok) {
+                    float dummy;
+                    exchange(kAbortMark, dummy);    // tell the partner
+                    break;
+                }
+                tc_fence_after();
+                uint32_t sr[2][32];
+                tmem_ld32(lane_addr + colS, sr[0]);
+                tmem_ld32(lane_addr + colS + 32, sr[1]);
+                tmem_wait_ld();
+                const int key0 = u.tile(j) * kPfBN + 64 * h;   // key of my first column
+                const bool masked = __any_sync(
+                    0xffffffffu, key0 + 63 > lim || (key0 < lo && key0 + 63 >= n_sinks));
+                if (masked) {
 #pragma unroll
-                for (int c = 0; c < 2; ++c)
+                    for (int c = 0; c < 2; ++c)
 #pragma unroll
-                    for (int e = 0; e < 32; ++e) {
-                        const int key = key0 + 32 * c + e;
-                        if (key > lim || (key < lo && key >= n_sinks))
-                            sr[c][e] = __float_as_uint(-INFINITY);
+                        for (int e = 0; e < 32; ++e) {
+                            const int key = key0 + 32 * c + e;
+                            if (key > lim || (key < lo && key >= n_sinks))
+                                sr[c][e] = __float_as_uint(-INFINITY);
+                        }
+                }
+                // row max of the raw scores (scale > 0 keeps the order), then
+                // the other half's max through shared memory
+                float mx4[4];
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {            // 4 independent chains of 16 scores
+                    const uint32_t *v = &sr[c >> 1][(c & 1) * 16];
+                    float m = __uint_as_float(v[0]);
+#pragma unroll
+                    for (int e = 1; e < 15; e += 2)
+                        m = max3f(m, __uint_as_float(v[e]), __uint_as_float(v[e + 1]));
+                    mx4[c] = fmaxf(m, __uint_as_float(v[15]));
+                }
+                const float mx_mine = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
+                float mx_other;
+                tc_fence_before();                      // my S loads precede the other half's P stores
+                exchange(mx_mine, mx_other);
+                tc_fence_after();
+                if (__any_sync(0xffffffffu, is_abort(mx_other))) {
+                    ok = false;
+                    break;
+                }
+                const float mxs = fmaxf(mx_mine, mx_other) * c2;
+                const bool move = mxs > m_ref + kRescaleLog2;  // always true on the first key seen
+                float alpha = 1.0f;
+                if (move) {
+                    alpha = fast_exp2(m_ref - mxs);     // 0 when nothing was seen before
+                    m_ref = mxs;
+                }
+                const float m_use = (m_ref == -INFINITY) ? 0.0f : m_ref;
+                const float2 cc = make_float2(c2, c2), nm = make_float2(-m_use, -m_use);
+                float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+                // P = exp2(s * scale * log2e - m_ref), truncated to bf16; P
+                // overwrites the first 64 columns of S (this half: packed
+                // columns 32h..32h+31).  l sums exactly the bf16 weights the PV
+                // product uses, so O / l is a convex combination of V rows.
+                // Tiles with masked (-inf) scores use the MUFU exp only; full
+                // tiles send part of the pairs to the FMA-pipe polynomial.
+                if (masked) {
+#pragma unroll
+                    for (int c = 0; c < 2; ++c) {
+                        uint32_t pk[16];
+                        softmax_chunk<false>(sr[c], cc, nm, pk, acc);
+                        tmem_st16(lane_addr + colP + 16 * c, pk);
                     }
-            }
-            // row max of the raw scores (scale > 0 keeps the order), then the
-            // other half's max through shared memory
-            float mx4[4];
+                } else {
 #pragma unroll
-            for (int c = 0; c < 4; ++c) {                // 4 independent chains of 16 scores
-                const uint32_t *v = &sr[c >> 1][(c & 1) * 16];
-                float m = __uint_as_float(v[0]);
+                    for (int c = 0; c < 2; ++c) {
+                        uint32_t pk[16];
+                        softmax_chunk<true>(sr[c], cc, nm, pk, acc);
+                        tmem_st16(lane_addr + colP + 16 * c, pk);
+                    }
+                }
+                l_run = l_run * alpha + ((acc[0] + acc[1]) + (acc[2] + acc[3]));
+                // O holds tiles < j at the old reference: rescale rows whose reference moved
+                if (j > 0 && __any_sync(0xffffffffu, move)) {
+                    const float2 a2 = make_float2(alpha, alpha);
 #pragma unroll
-                for (int e = 1; e < 15; e += 2)
-                    m = max3f(m, __uint_as_float(v[e]), __uint_as_float(v[e + 1]));
-                mx4[c] = fmaxf(m, __uint_as_float(v[15]));
+                    for (int c = 0; c < D / 64; ++c) {
+                        uint32_t orr[32];
+                        tmem_ld32(lane_addr + colO + 32 * c, orr);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int e = 0; e < 32; e += 2) {
+                            const float2 v2 = mul2(make_float2(__uint_as_float(orr[e]),
+                                                               __uint_as_float(orr[e + 1])), a2);
+                            orr[e] = __float_as_uint(v2.x);
+                            orr[e + 1] = __float_as_uint(v2.y);
+                        }
+                        tmem_st32(lane_addr + colO + 32 * c, orr);
+                    }
+                }
+                tmem_wait_st();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&p_full[k]);
             }
-            float mx2[2] = {fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3])};
-            const float mx_mine = fmaxf(mx2[0], mx2[1]);
-            float mx_other;
-            tc_fence_before();                          // my S loads precede the other half's P stores
-            exchange(mx_mine, j & 1, mx_other);
-            tc_fence_after();
-            // the partner's abort marker (a NaN payload no max can produce)
-            if (__any_sync(0xffffffffu, __float_as_int(mx_other) == 0x7fc00001)) {
+            if (!ok) break;
+            // ---- epilogue: O / l -> bf16, lse (each half writes its d/2 columns) ----
+            // O_k is read out of tensor memory, then released to the next
+            // unit's first PV before the conversion and the global stores.
+            const bool done = __all_sync(0xffffffffu,
+                                         mbar_wait(&o_done[k], ui & 1, &abort_flag, p.status));
+            float l_other;
+            exchange(done ? l_run : kAbortMark, l_other);
+            if (!done || __any_sync(0xffffffffu, is_abort(l_other))) {
                 ok = false;
                 break;
             }
-            const float mxs = fmaxf(mx_mine, mx_other) * c2;
-            const bool move = mxs > m_ref + kRescaleLog2;  // always true on the first key seen
-            float alpha = 1.0f;
-            if (move) {
-                alpha = fast_exp2(m_ref - mxs);         // 0 when nothing was seen before
-                m_ref = mxs;
-            }
-            const float m_use = (m_ref == -INFINITY) ? 0.0f : m_ref;
-            const float2 cc = make_float2(c2, c2), nm = make_float2(-m_use, -m_use);
-            float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-            // P = exp2(s * scale * log2e - m_ref), truncated to bf16; P overwrites
-            // the first 64 columns of S (this half: packed columns 32h..32h+31).
-            // l sums exactly the bf16 weights the PV product uses, so O / l is
-            // a convex combination of V rows.  Tiles with masked (-inf) scores
-            // use the MUFU exp only; full tiles send part of the pairs to the
-            // FMA-pipe polynomial.
-            if (masked) {
+            tc_fence_after();
+            uint32_t orr[D / 64][32];
 #pragma unroll
-                for (int c = 0; c < 2; ++c) {
-                    uint32_t pk[16];
-                    softmax_chunk<false>(sr[c], cc, nm, pk, acc);
-                    tmem_st16(lane_addr + colP + 16 * c, pk);
-                }
-            } else {
-#pragma unroll
-                for (int c = 0; c < 2; ++c) {
-                    uint32_t pk[16];
-                    softmax_chunk<true>(sr[c], cc, nm, pk, acc);
-                    tmem_st16(lane_addr + colP + 16 * c, pk);
-                }
-            }
-            l_run = l_run * alpha + ((acc[0] + acc[1]) + (acc[2] + acc[3]));
-            // O holds tiles < j at the old reference: rescale rows whose reference moved
-            if (j > 0 && __any_sync(0xffffffffu, move)) {
-                const float2 a2 = make_float2(alpha, alpha);
-#pragma unroll
-                for (int c = 0; c < D / 64; ++c) {
-                    uint32_t orr[32];
-                    tmem_ld32(lane_addr + colO + 32 * c, orr);
-                    tmem_wait_ld();
-#pragma unroll
-                    for (int e = 0; e < 32; e += 2) {
-                        const float2 v2 = mul2(make_float2(__uint_as_float(orr[e]),
-                                                           __uint_as_float(orr[e + 1])), a2);
-                        orr[e] = __float_as_uint(v2.x);
-                        orr[e + 1] = __float_as_uint(v2.y);
-                    }
-                    tmem_st32(lane_addr + colO + 32 * c, orr);
-                }
-            }
-            tmem_wait_st();
+            for (int c = 0; c < D / 64; ++c) tmem_ld32(lane_addr + colO + 32 * c, orr[c]);
+            tmem_wait_ld();
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&p_full[k]);
-        }
-        // ---- epilogue: O / l -> bf16, lse (each half writes its d/2 columns) ----
-        float l_other = 0.0f;
-        if (ok) exchange(l_run, n_kv & 1, l_other);
-        const float l_row = l_run + l_other;
-        if (ok && n_kv > 0)
-            ok = __all_sync(0xffffffffu, mbar_wait(&o_done[k], 0, &abort_flag, p.status));
-        tc_fence_after();
-        const float inv_l = (l_row > 0.0f) ? 1.0f / l_row : 0.0f;
-        __nv_bfloat16 *dst =
-            p.o + ((static_cast<size_t>(b) * p.Tq + pos) * p.Hq + head) * D + (D / 2) * h;
-#pragma unroll
-        for (int c = 0; c < D / 64; ++c) {
-            uint32_t orr[32];
-            if (ok && n_kv > 0) {
-                tmem_ld32(lane_addr + colO + 32 * c, orr);
-                tmem_wait_ld();
-            } else {
-#pragma unroll
-                for (int e = 0; e < 32; ++e) orr[e] = 0u;
-            }
-            uint32_t pk[16];
-#pragma unroll
-            for (int e = 0; e < 16; ++e)
-                pk[e] = pack_bf16x2(__uint_as_float(orr[2 * e]) * inv_l,
-                                    __uint_as_float(orr[2 * e + 1]) * inv_l);
+            if (lane == 0) mbar_arrive(&o_free[k]);
+            ++ui;
+            const float l_row = l_run + l_other;
+            const float inv_l = (l_row > 0.0f) ? 1.0f / l_row : 0.0f;
             if (row_real) {
-                uint4 *d4 = reinterpret_cast<uint4 *>(dst + 32 * c);
 #pragma unroll
-                for (int e = 0; e < 4; ++e)
-                    d4[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
+                for (int c = 0; c < D / 64; ++c) {
+                    uint4 *d4 = reinterpret_cast<uint4 *>(dst + 32 * c);
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const uint32_t *v = &orr[c][8 * e];
+                        d4[e] = make_uint4(
+                            pack_bf16x2(__uint_as_float(v[0]) * inv_l, __uint_as_float(v[1]) * inv_l),
+                            pack_bf16x2(__uint_as_float(v[2]) * inv_l, __uint_as_float(v[3]) * inv_l),
+                            pack_bf16x2(__uint_as_float(v[4]) * inv_l, __uint_as_float(v[5]) * inv_l),
+                            pack_bf16x2(__uint_as_float(v[6]) * inv_l, __uint_as_float(v[7]) * inv_l));
+                    }
+                }
+                if (lse_dst && h == 0)
+                    *lse_dst = (l_row > 0.0f) ? (m_ref + __log2f(l_row)) * 0.69314718055994531f
+                                              : -INFINITY;
             }
         }
-        if (p.lse && row_real && h == 0)
-            p.lse[(static_cast<size_t>(b) * p.Hq + head) * p.Tq + pos] =
-                (l_row > 0.0f) ? (m_ref + __log2f(l_row)) * 0.69314718055994531f : -INFINITY;
     }
 
     tc_fence_before();
@@ -525,8 +619,16 @@ static int launch_prefill_d(const void *q, const void *k, const void *v, void *o
     prm.lse = lse;
     prm.status = device_status_ptr();
     if (!prm.status) return GQA_ERR_CUDA;
-    const long long blocks = static_cast<long long>(prm.n_pairs) * B * Hkv;
-    if (blocks > 0x7fffffffLL) return set_error(GQA_ERR_UNSUPPORTED, "prefill grid too large");
+    const long long units = static_cast<long long>(prm.n_pairs) * B * Hkv;
+    if (units > 0x7fffffffLL) return set_error(GQA_ERR_UNSUPPORTED, "prefill grid too large");
+    int n_sm = 0;
+    if (int rc = sm_count(&n_sm)) return rc;
+    long long blocks = units < n_sm ? units : n_sm;   // persistent: one CTA per SM
+    // GQA_PREFILL_MAX_CTAS caps the grid (tests use it to put many units on each CTA)
+    if (const char *cap = getenv("GQA_PREFILL_MAX_CTAS")) {
+        const long long m = atoll(cap);
+        if (m > 0 && m < blocks) blocks = m;
+    }
 
     CUtensorMap tq, tk, tv;
     if (int rc = encode_tmap_bf16_4d(&tq, q, D, Hq, Tq, B, 64, prm.G, prm.P, 1, 1)) return rc;

@@ -142,3 +142,40 @@ def test_head_sharing_sweep_t2048(gqa_lib, Hkv):
 def test_long_context_t32768(gqa_lib):
     q, k, v = workloads.prefill_inputs(1, 32768, 64, 8, 128, qk_std=8.0)
     check_sampled(q, k, v, True, 2048, 5)
+
+
+PERSISTENT_CASES = [
+    # B, Tq, Tkv, Hq, Hkv, d, causal, window, sinks
+    (2, 300, 300, 8, 2, 128, True, 0, 0),
+    (1, 300, 100, 8, 2, 128, True, 0, 0),      # units with no visible key between others
+    (3, 200, 200, 8, 8, 128, False, 0, 0),
+    (1, 700, 700, 8, 2, 128, True, 200, 4),    # window + sinks
+    (1, 520, 520, 32, 1, 64, True, 0, 0),
+]
+
+
+@pytest.mark.parametrize("ctas", [1, 3])
+@pytest.mark.parametrize("B,Tq,Tkv,Hq,Hkv,d,causal,window,sinks", PERSISTENT_CASES)
+def test_persistent_units_per_cta(gqa_lib, monkeypatch, ctas, B, Tq, Tkv, Hq, Hkv, d, causal,
+                                  window, sinks):
+    # a capped grid makes every CTA walk many units: the Q reloads, the O
+    # hand-over between units and the barrier phases across unit boundaries
+    monkeypatch.setenv("GQA_PREFILL_MAX_CTAS", str(ctas))
+    q, k, v = workloads.prefill_inputs(B, Tq, Hq, Hkv, d, Tkv=Tkv, seeds=(Tq + 5, Tkv + 6, ctas))
+    if window:
+        o_ref, lse_ref = ref.attn_fwd_window(q, k, v, window, sinks)
+    else:
+        o_ref, lse_ref = ref.attn_fwd(q, k, v, causal)
+    o, lse = gqa.attn(q.cuda(), k.cuda(), v.cuda(), causal=causal, return_lse=True,
+                      window=window or None, sinks=sinks)
+    gqa.device_status()
+    assert max_abs(o, o_ref) <= BF16_TOL
+    l = lse.cpu().numpy().astype(np.float64)
+    fin = np.isfinite(lse_ref)
+    assert np.array_equal(np.isneginf(l), ~fin)
+    assert np.max(np.abs(l[fin] - lse_ref[fin]), initial=0.0) <= BF16_TOL
+    # the same bits as the full grid: the schedule does not change the arithmetic
+    monkeypatch.delenv("GQA_PREFILL_MAX_CTAS")
+    o_full = gqa.attn(q.cuda(), k.cuda(), v.cuda(), causal=causal, window=window or None,
+                      sinks=sinks)
+    assert torch.equal(o.cpu(), o_full.cpu())
