@@ -8,5 +8,5 @@ streams only.  The library is loaded on first use and there is no CPU
 fallback: a missing or unloadable library raises.
 """
 
-from .api import (attn, attn_bwd, attn_f32, decode, decode_workspace_size, device_status, fold_kv,  # noqa: F401
-                  rope_, rope_decode_q_, rope_qk_)
+from .api import (attn, attn_bwd, attn_f32, attn_host, decode, decode_workspace_size, device_status, fold_kv,  # noqa: F401
+                  host_staging, rope_, rope_decode_q_, rope_qk_)

@@ -28,6 +28,8 @@ _F = ctypes.c_float
 _SIGNATURES = {
     "gqa_attn_fwd": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _P]),
     "gqa_attn_fwd_lse": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _P]),
+    "gqa_attn_fwd_host": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _P,
+                               _P]),
     "gqa_attn_fwd_window": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _F, _P]),
     "gqa_attn_fwd_f32": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _P]),
     "gqa_decode_workspace_size": (ctypes.c_size_t, [_I, _I, _I, _I, _I]),
@@ -119,6 +121,12 @@ def gqa_attn_bwd(q, k, v, o, dout, lse, dq, dk, dv, B, Tq, Tkv, Hq, Hkv, d, caus
 
 def gqa_rope(x, B, T, H, d, pos0, theta, stream):
     return lib().gqa_rope(x, B, T, H, d, pos0, theta, stream)
+
+
+def gqa_attn_fwd_host(q_host, k_host, v_host, o_host, q_dev, k_dev, v_dev, o_dev, B, Tq, Tkv, Hq,
+                      Hkv, d, causal, scale, stream, done_event):
+    return lib().gqa_attn_fwd_host(q_host, k_host, v_host, o_host, q_dev, k_dev, v_dev, o_dev, B,
+                                   Tq, Tkv, Hq, Hkv, d, causal, scale, stream, done_event)
 
 
 def gqa_rope_qk(q, k, B, T, Hq, Hkv, d, pos0, theta, stream):

@@ -79,6 +79,59 @@ def attn(q, k, v, causal=True, scale=None, out=None, return_lse=False, window=No
     return (o, lse) if return_lse else o
 
 
+def _need_host(t, name, ndim):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.is_cuda:
+        raise ValueError(f"{name} must be a host (CPU) tensor")
+    if t.dtype != torch.bfloat16:
+        raise ValueError(f"{name} must be torch.bfloat16, got {t.dtype}")
+    if t.dim() != ndim or not t.is_contiguous():
+        raise ValueError(f"{name} must be a contiguous {ndim}-d tensor, got {tuple(t.shape)}")
+
+
+def host_staging(q, k, device=None):
+    """Device staging buffers (q, k, v, o) for ``attn_host`` on host tensors shaped like q, k."""
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else device
+    return (torch.empty(q.shape, dtype=torch.bfloat16, device=dev),
+            torch.empty(k.shape, dtype=torch.bfloat16, device=dev),
+            torch.empty(k.shape, dtype=torch.bfloat16, device=dev),
+            torch.empty(q.shape, dtype=torch.bfloat16, device=dev))
+
+
+def attn_host(q, k, v, out=None, causal=True, scale=None, staging=None, done=None):
+    """``attn`` on host (CPU, preferably pinned) bf16 tensors: the copies up and down
+    run in the library, overlapped with the attention chunk by chunk.  ``staging``
+    is a (q, k, v, o) tuple of device buffers (``host_staging``).  The call is
+    asynchronous on the staging device's current stream and returns ``out``: valid
+    once that stream has reached this point, or, with ``done`` (a torch.cuda.Event),
+    once ``done`` has completed (the stream is then not held for the copies down, so
+    consecutive calls overlap).  The host tensors must stay alive and unchanged until
+    then: the copies run after this function returns."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _need_host(t, n, 4)
+    B, Tq, Tkv, Hq, Hkv, d = _shapes(q, k, v)
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    o = torch.empty(q.shape, dtype=torch.bfloat16, pin_memory=q.is_pinned()) if out is None else out
+    _need_host(o, "out", 4)
+    if tuple(o.shape) != tuple(q.shape):
+        raise ValueError(f"out shape {tuple(o.shape)} != q shape {tuple(q.shape)}")
+    st = host_staging(q, k) if staging is None else staging
+    for t, ref, n in zip(st, (q, k, k, q), ("q_dev", "k_dev", "v_dev", "o_dev")):
+        _need(t, n, torch.bfloat16, 4)
+        if tuple(t.shape) != tuple(ref.shape):
+            raise ValueError(f"{n} shape {tuple(t.shape)} != {tuple(ref.shape)}")
+    ev = None
+    if done is not None:
+        done.record(torch.cuda.current_stream(st[0].device))   # makes sure the event exists
+        ev = done.cuda_event
+    rc = _b.gqa_attn_fwd_host(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
+                              *(t.data_ptr() for t in st), B, Tq, Tkv, Hq, Hkv, d,
+                              int(bool(causal)), scale, _stream(st[0]), ev)
+    _check(rc, "gqa_attn_fwd_host")
+    return o
+
+
 def attn_f32(q, k, v, causal=True, scale=None, return_lse=False):
     """The same operation in fp32 (FP32 pipe); q/k/v fp32 in the same layouts."""
     for t, n in ((q, "q"), (k, "k"), (v, "v")):

@@ -102,11 +102,11 @@ static EncodeTiledFn encode_fn() {
 
 int encode_tmap_bf16_4d(CUtensorMap *map, const void *base, uint64_t n0, uint64_t n1,
                         uint64_t n2, uint64_t n3, uint32_t b0, uint32_t b1, uint32_t b2,
-                        uint32_t b3, int swizzle128) {
+                        uint32_t b3, int swizzle128, uint64_t n2_pitch) {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return set_error(GQA_ERR_CUDA, "cuTensorMapEncodeTiled is not available");
     cuuint64_t dims[4] = {n0, n1, n2, n3};
-    cuuint64_t strides[3] = {n0 * 2, n0 * n1 * 2, n0 * n1 * n2 * 2};
+    cuuint64_t strides[3] = {n0 * 2, n0 * n1 * 2, n0 * n1 * (n2_pitch ? n2_pitch : n2) * 2};
     cuuint32_t box[4] = {b0, b1, b2, b3};
     cuuint32_t estr[4] = {1, 1, 1, 1};
     CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(base), dims,
@@ -191,6 +191,34 @@ static int attn_fwd_bf16(const void *q, const void *k, const void *v, void *o, f
     if (int rc = check_ptr(v, 16, "v")) return rc;
     return launch_prefill(q, k, v, o, lse, B, Tq, Tkv, Hq, Hkv, d, causal, window, sinks, scale,
                           s);
+}
+
+int gqa_attn_fwd_host(const void *q_host, const void *k_host, const void *v_host, void *o_host,
+                      void *q_dev, void *k_dev, void *v_dev, void *o_dev, int B, int Tq, int Tkv,
+                      int Hq, int Hkv, int d, int causal, float scale, gqa_stream_t stream,
+                      void *done_event) {
+    t_last_error[0] = 0;
+    if (int rc = check_fwd_common(B, Tq, Tkv, Hq, Hkv, d, causal, scale)) return rc;
+    if (d != 64 && d != 128)
+        return set_error(GQA_ERR_UNSUPPORTED, "head dim d=%d: the bf16 path supports 64 and 128", d);
+    if (Hq / Hkv > 128)
+        return set_error(GQA_ERR_UNSUPPORTED, "group size Hq/Hkv=%d exceeds 128", Hq / Hkv);
+    if (B == 0 || Tq == 0) return GQA_OK;
+    if (int rc = check_ptr(q_host, 2, "q_host")) return rc;
+    if (int rc = check_ptr(o_host, 2, "o_host")) return rc;
+    if (int rc = check_ptr(q_dev, 16, "q_dev")) return rc;
+    if (int rc = check_ptr(o_dev, 16, "o_dev")) return rc;
+    if (Tkv > 0) {
+        if (int rc = check_ptr(k_host, 2, "k_host")) return rc;
+        if (int rc = check_ptr(v_host, 2, "v_host")) return rc;
+        if (int rc = check_ptr(k_dev, 16, "k_dev")) return rc;
+        if (int rc = check_ptr(v_dev, 16, "v_dev")) return rc;
+    }
+    if (int rc = require_sm100()) return rc;
+    return launch_fwd_host_pipeline(q_host, k_host, v_host, o_host, q_dev, k_dev, v_dev, o_dev, B,
+                                    Tq, Tkv, Hq, Hkv, d, causal, scale,
+                                    reinterpret_cast<cudaStream_t>(stream),
+                                    static_cast<cudaEvent_t>(done_event));
 }
 
 int gqa_attn_fwd_lse(const void *q, const void *k, const void *v, void *o, float *lse,

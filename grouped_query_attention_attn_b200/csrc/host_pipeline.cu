@@ -1,0 +1,151 @@
+// host_pipeline.cu -- attention forward on host-resident q / k / v / o.
+//
+// The host <-> device copies are the long pole (PCIe moves ~50 GB/s, the
+// prefill kernel reads the same bytes at several TB/s), so the query
+// positions are cut into chunks and three queues overlap: chunk c's q rows and
+// the k / v rows it newly needs go up on one copy stream while chunk c - 1's
+// attention runs on the caller's stream and chunk c - 2's o comes down on a
+// second copy stream.  With a causal mask chunk c needs keys [0, last row of
+// c + Tkv - Tq], so k / v travel in the same chunks as q.  Each chunk's
+// attention is the prefill kernel on views of the staging buffers (bottom-right
+// alignment makes a chunk of rows against its key prefix exactly the same
+// computation as in the whole problem).  With a completion event the caller's
+// stream is not held for the copies down, so the next call's copies up start
+// when this call's attention is done and overlap this call's copies down.
+#include <mutex>
+
+#include "internal.h"
+
+namespace gqa {
+
+namespace {
+
+constexpr int kMaxChunks = 16;
+constexpr int kMaxDevices = 64;
+
+// Copy streams and events, created once per device and reused by every call
+// (the enqueue sequence below runs under a lock, so calls from several host
+// threads cannot interleave their event records).
+struct PipeRes {
+    cudaStream_t up = nullptr, down = nullptr;
+    cudaEvent_t ev[2 * kMaxChunks + 2] = {};
+    bool ready = false;
+};
+
+std::mutex g_pipe_mu;
+PipeRes g_pipe[kMaxDevices];
+
+int pipe_res(int dev, PipeRes **out) {
+    PipeRes &r = g_pipe[dev];
+    if (!r.ready) {
+        if (int rc = check_cuda(cudaStreamCreateWithFlags(&r.up, cudaStreamNonBlocking),
+                                "cudaStreamCreateWithFlags"))
+            return rc;
+        if (int rc = check_cuda(cudaStreamCreateWithFlags(&r.down, cudaStreamNonBlocking),
+                                "cudaStreamCreateWithFlags"))
+            return rc;
+        for (cudaEvent_t &e : r.ev)
+            if (int rc = check_cuda(cudaEventCreateWithFlags(&e, cudaEventDisableTiming),
+                                    "cudaEventCreateWithFlags"))
+                return rc;
+        r.ready = true;
+    }
+    *out = &r;
+    return GQA_OK;
+}
+
+// rows [r0, r1) of every batch of a [B, T, H, d] bf16 tensor: B strided blocks
+int copy_rows(void *dst, const void *src, int B, int T, int H, int d, int r0, int r1,
+              cudaMemcpyKind kind, cudaStream_t s) {
+    if (r1 <= r0 || B == 0) return GQA_OK;
+    const size_t row = static_cast<size_t>(H) * d * 2;
+    const size_t off = static_cast<size_t>(r0) * row;
+    return check_cuda(cudaMemcpy2DAsync(static_cast<uint8_t *>(dst) + off, T * row,
+                                        static_cast<const uint8_t *>(src) + off, T * row,
+                                        (r1 - r0) * row, B, kind, s),
+                      "cudaMemcpy2DAsync");
+}
+
+}  // namespace
+
+int launch_fwd_host_pipeline(const void *q_host, const void *k_host, const void *v_host,
+                             void *o_host, void *q_dev, void *k_dev, void *v_dev, void *o_dev,
+                             int B, int Tq, int Tkv, int Hq, int Hkv, int d, int causal,
+                             float scale, cudaStream_t stream, cudaEvent_t done) {
+    int dev = 0;
+    if (int rc = check_cuda(cudaGetDevice(&dev), "cudaGetDevice")) return rc;
+    if (dev < 0 || dev >= kMaxDevices) return set_error(GQA_ERR_UNSUPPORTED, "device %d", dev);
+    std::lock_guard<std::mutex> lock(g_pipe_mu);
+    PipeRes *r = nullptr;
+    if (int rc = pipe_res(dev, &r)) return rc;
+
+    // chunks of at least 256 rows, at most kMaxChunks of them
+    int rows = (Tq + 7) / 8;
+    if (rows < 256) rows = 256;
+    if ((Tq + rows - 1) / rows > kMaxChunks) rows = (Tq + kMaxChunks - 1) / kMaxChunks;
+    const int n_chunks = (Tq + rows - 1) / rows;
+    const size_t qrow = static_cast<size_t>(Hq) * d * 2;
+
+    // ev_done marks the end of the last call's copies down on this device (an
+    // event never recorded yet is complete)
+    cudaEvent_t ev_start = r->ev[2 * kMaxChunks], ev_done = r->ev[2 * kMaxChunks + 1];
+    // the staging buffers may still be read by earlier work on the caller's stream
+    if (int rc = check_cuda(cudaEventRecord(ev_start, stream), "cudaEventRecord")) return rc;
+    if (int rc = check_cuda(cudaStreamWaitEvent(r->up, ev_start, 0), "cudaStreamWaitEvent"))
+        return rc;
+    // and o_dev may still be on its way down from the previous call
+    if (int rc = check_cuda(cudaStreamWaitEvent(stream, ev_done, 0), "cudaStreamWaitEvent"))
+        return rc;
+    int kv_have = 0;
+    for (int c = 0; c < n_chunks; ++c) {
+        const int a = c * rows, b = a + rows < Tq ? a + rows : Tq;
+        int kv_need = Tkv;
+        if (causal) {
+            kv_need = b + (Tkv - Tq);
+            kv_need = kv_need < 0 ? 0 : (kv_need > Tkv ? Tkv : kv_need);
+        }
+        cudaEvent_t ev_in = r->ev[2 * c], ev_out = r->ev[2 * c + 1];
+        // ---- up: the rows this chunk adds ----
+        if (kv_need > kv_have) {
+            if (int rc = copy_rows(k_dev, k_host, B, Tkv, Hkv, d, kv_have, kv_need,
+                                   cudaMemcpyHostToDevice, r->up))
+                return rc;
+            if (int rc = copy_rows(v_dev, v_host, B, Tkv, Hkv, d, kv_have, kv_need,
+                                   cudaMemcpyHostToDevice, r->up))
+                return rc;
+            kv_have = kv_need;
+        }
+        if (int rc = copy_rows(q_dev, q_host, B, Tq, Hq, d, a, b, cudaMemcpyHostToDevice, r->up))
+            return rc;
+        if (int rc = check_cuda(cudaEventRecord(ev_in, r->up), "cudaEventRecord")) return rc;
+        // ---- compute on the caller's stream ----
+        if (int rc = check_cuda(cudaStreamWaitEvent(stream, ev_in, 0), "cudaStreamWaitEvent"))
+            return rc;
+        uint8_t *o_view = static_cast<uint8_t *>(o_dev) + a * qrow;
+        if (kv_need == 0) {
+            // rows that see no key: o = 0
+            if (int rc = check_cuda(cudaMemset2DAsync(o_view, Tq * qrow, 0, (b - a) * qrow, B,
+                                                      stream),
+                                    "cudaMemset2DAsync"))
+                return rc;
+        } else {
+            if (int rc = launch_prefill(static_cast<const uint8_t *>(q_dev) + a * qrow, k_dev,
+                                        v_dev, o_view, nullptr, B, b - a, kv_need, Hq, Hkv, d,
+                                        causal, 0, 0, scale, stream, Tq, Tkv))
+                return rc;
+        }
+        if (int rc = check_cuda(cudaEventRecord(ev_out, stream), "cudaEventRecord")) return rc;
+        // ---- down: this chunk's o ----
+        if (int rc = check_cuda(cudaStreamWaitEvent(r->down, ev_out, 0), "cudaStreamWaitEvent"))
+            return rc;
+        if (int rc = copy_rows(o_host, o_dev, B, Tq, Hq, d, a, b, cudaMemcpyDeviceToHost, r->down))
+            return rc;
+    }
+    // every key row went up with some chunk (the last one needs all of them)
+    if (int rc = check_cuda(cudaEventRecord(ev_done, r->down), "cudaEventRecord")) return rc;
+    if (done) return check_cuda(cudaEventRecord(done, r->down), "cudaEventRecord");
+    // without a completion event the caller's stream completes once o is back
+    return check_cuda(cudaStreamWaitEvent(stream, ev_done, 0), "cudaStreamWaitEvent");
+}
+
+}  // namespace gqa

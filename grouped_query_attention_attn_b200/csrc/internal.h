@@ -28,12 +28,15 @@ int sm_count(int *n);
 // (looked up once per device); nullptr with a message set on failure.
 int *device_status_ptr();
 
-// 4-D bf16 tensor map over a [n3][n2][n1][n0] contiguous array (n0 innermost),
-// box (b0, b1, b2, b3), 128-byte swizzle when swizzle128 != 0, zero fill out
-// of bounds.  Returns GQA_OK or GQA_ERR_CUDA.
+// 4-D bf16 tensor map over a [n3][n2][n1][n0] array (n0 innermost, the first
+// three dimensions contiguous), box (b0, b1, b2, b3), 128-byte swizzle when
+// swizzle128 != 0, zero fill out of bounds.  Consecutive n3 indices lie
+// n2_pitch rows of n1 * n0 elements apart (n2_pitch = 0: n2, i.e. contiguous),
+// so a window of rows of a longer tensor can be mapped.  Returns GQA_OK or
+// GQA_ERR_CUDA.
 int encode_tmap_bf16_4d(CUtensorMap *map, const void *base, uint64_t n0, uint64_t n1,
                         uint64_t n2, uint64_t n3, uint32_t b0, uint32_t b1, uint32_t b2,
-                        uint32_t b3, int swizzle128);
+                        uint32_t b3, int swizzle128, uint64_t n2_pitch = 0);
 
 // ---- launchers (arguments already validated by the C-ABI layer) ----------
 int launch_fwd_f32(const float *q, const float *k, const float *v, float *o, float *lse,
@@ -54,9 +57,19 @@ int launch_decode(const void *q, const void *k_cache, const void *v_cache,
                   const int32_t *seqlens, void *o, int B, int Hq, int Hkv, int d, int Lmax,
                   int window, int sinks, float scale, void *workspace, cudaStream_t stream);
 
+// q / o are views of Tq rows of [B, tq_pitch, Hq, d] buffers and k / v of Tkv rows
+// of [B, tkv_pitch, Hkv, d] buffers (pitch 0: the view is the whole tensor).
 int launch_prefill(const void *q, const void *k, const void *v, void *o, float *lse,
                    int B, int Tq, int Tkv, int Hq, int Hkv, int d, int causal, int window,
-                   int sinks, float scale, cudaStream_t stream);
+                   int sinks, float scale, cudaStream_t stream, int tq_pitch = 0,
+                   int tkv_pitch = 0);
+
+// Forward on host-resident tensors through device staging buffers, with the
+// copies pipelined against the attention in chunks of query rows.
+int launch_fwd_host_pipeline(const void *q_host, const void *k_host, const void *v_host,
+                             void *o_host, void *q_dev, void *k_dev, void *v_dev, void *o_dev,
+                             int B, int Tq, int Tkv, int Hq, int Hkv, int d, int causal,
+                             float scale, cudaStream_t stream, cudaEvent_t done);
 
 size_t bwd_workspace_bytes(int B, int Tq, int Hq);
 int launch_bwd(const void *q, const void *k, const void *v, const void *o, const void *dout,

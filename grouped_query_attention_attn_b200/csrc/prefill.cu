@@ -62,6 +62,7 @@ struct PfLayout {
 
 struct PfParams {
     int B, Tq, Tkv, Hq, Hkv, G, P;   // P = positions per M tile
+    int tq_pitch;                     // rows between batches of o (>= Tq)
     int n_pairs;                      // M-tile pairs per (b, kvh)
     int causal;
     int window, sinks;                // sliding window (0 = none) and sink keys
@@ -415,7 +416,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             const int head = u.kvh * p.G + r % p.G;
             const bool row_real = (r < p.P * p.G) && (pos < p.Tq);
             __nv_bfloat16 *dst =
-                p.o + ((static_cast<size_t>(u.b) * p.Tq + pos) * p.Hq + head) * D + (D / 2) * h;
+                p.o + ((static_cast<size_t>(u.b) * p.tq_pitch + pos) * p.Hq + head) * D + (D / 2) * h;
             float *lse_dst = p.lse ? p.lse + (static_cast<size_t>(u.b) * p.Hq + head) * p.Tq + pos
                                    : nullptr;
             if (u.n_kv == 0) {
@@ -600,8 +601,10 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
 template <int D>
 static int launch_prefill_d(const void *q, const void *k, const void *v, void *o, float *lse,
                             int B, int Tq, int Tkv, int Hq, int Hkv, int causal, int window,
-                            int sinks, float scale, cudaStream_t stream) {
+                            int sinks, float scale, cudaStream_t stream, int tq_pitch,
+                            int tkv_pitch) {
     PfParams prm;
+    prm.tq_pitch = tq_pitch > 0 ? tq_pitch : Tq;
     prm.window = window;
     prm.sinks = sinks;
     prm.B = B;
@@ -631,9 +634,13 @@ static int launch_prefill_d(const void *q, const void *k, const void *v, void *o
     }
 
     CUtensorMap tq, tk, tv;
-    if (int rc = encode_tmap_bf16_4d(&tq, q, D, Hq, Tq, B, 64, prm.G, prm.P, 1, 1)) return rc;
-    if (int rc = encode_tmap_bf16_4d(&tk, k, D, Hkv, Tkv, B, 64, 1, kPfBN, 1, 1)) return rc;
-    if (int rc = encode_tmap_bf16_4d(&tv, v, D, Hkv, Tkv, B, 64, 1, kPfBN, 1, 1)) return rc;
+    const uint64_t kv_pitch = tkv_pitch > 0 ? tkv_pitch : Tkv;
+    if (int rc = encode_tmap_bf16_4d(&tq, q, D, Hq, Tq, B, 64, prm.G, prm.P, 1, 1, prm.tq_pitch))
+        return rc;
+    if (int rc = encode_tmap_bf16_4d(&tk, k, D, Hkv, Tkv, B, 64, 1, kPfBN, 1, 1, kv_pitch))
+        return rc;
+    if (int rc = encode_tmap_bf16_4d(&tv, v, D, Hkv, Tkv, B, 64, 1, kPfBN, 1, 1, kv_pitch))
+        return rc;
 
     auto kern = prefill_kernel<D>;
     const int smem = PfLayout<D>::kSmemBytes;
@@ -646,12 +653,12 @@ static int launch_prefill_d(const void *q, const void *k, const void *v, void *o
 
 int launch_prefill(const void *q, const void *k, const void *v, void *o, float *lse, int B,
                    int Tq, int Tkv, int Hq, int Hkv, int d, int causal, int window, int sinks,
-                   float scale, cudaStream_t stream) {
+                   float scale, cudaStream_t stream, int tq_pitch, int tkv_pitch) {
     if (d == 128)
         return launch_prefill_d<128>(q, k, v, o, lse, B, Tq, Tkv, Hq, Hkv, causal, window, sinks,
-                                     scale, stream);
+                                     scale, stream, tq_pitch, tkv_pitch);
     return launch_prefill_d<64>(q, k, v, o, lse, B, Tq, Tkv, Hq, Hkv, causal, window, sinks,
-                                scale, stream);
+                                scale, stream, tq_pitch, tkv_pitch);
 }
 
 }  // namespace gqa

@@ -79,6 +79,34 @@ int gqa_attn_fwd_lse(const void *q, const void *k, const void *v, void *o, float
                      int causal, float scale, gqa_stream_t stream);
 
 /*
+ * gqa_attn_fwd_host -- gqa_attn_fwd for host-resident tensors (same operation,
+ * layouts and arguments; no lse).  q_host, k_host, v_host are read and o_host
+ * written (pinned host memory for the copies to run asynchronously; pageable
+ * memory works, slower); q_dev, k_dev, v_dev, o_dev are caller-owned device
+ * staging buffers of the full tensor sizes (16-byte aligned), overwritten.
+ * The query rows are cut into at most 16 chunks of >= 256 rows; chunk c's q
+ * rows and the k / v rows it newly needs (with the causal mask, keys up to
+ * its last row + Tkv - Tq) are copied up on a library-owned copy stream
+ * while chunk c - 1's attention runs on `stream` and chunk c - 2's o is
+ * copied down on a second library-owned stream.  Asynchronous: with
+ * done_event == NULL, o_host is complete when the work enqueued on `stream` so
+ * far is; otherwise done_event (a cudaEvent_t created by the caller) is
+ * recorded when o_host is complete and `stream` is not held for the copies
+ * down, so a following call's copies up overlap them.  A call orders its
+ * copies up after the work on `stream` at the time of the call and its first
+ * attention chunk after the previous call's copies down (on this device).
+ * The host buffers must stay allocated and unchanged until the call completes.
+ * The copy streams and their events are created once per device on first use
+ * and kept (no device memory is allocated); concurrent calls from several
+ * host threads are serialised while they enqueue.  Errors as
+ * gqa_attn_fwd_lse, plus GQA_ERR_CUDA for a failed copy.
+ */
+int gqa_attn_fwd_host(const void *q_host, const void *k_host, const void *v_host, void *o_host,
+                      void *q_dev, void *k_dev, void *v_dev, void *o_dev, int B, int Tq, int Tkv,
+                      int Hq, int Hkv, int d, int causal, float scale, gqa_stream_t stream,
+                      void *done_event);
+
+/*
  * gqa_attn_fwd_window -- causal forward with a sliding window and attention
  * sinks (course "Неделя 7. Внимание", step 3: the window bounds what a token
  * sees -- and the cache -- to the most recent keys, while the first tokens,

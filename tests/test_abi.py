@@ -161,6 +161,20 @@ def test_window_entry_points_reject_bad_window(gqa_lib):
                                  NULL) == b.GQA_ERR_INVALID_ARG
 
 
+def test_host_forward_rejects(gqa_lib):
+    args = (1, 64, 64, 4, 2, 128, 1, 0.088, NULL, NULL)
+    assert b.gqa_attn_fwd_host(NULL, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, *args) == \
+        b.GQA_ERR_INVALID_ARG                                                   # q_host
+    assert b.gqa_attn_fwd_host(FAKE, FAKE, FAKE, FAKE, FAKE + 8, FAKE, FAKE, FAKE, *args) == \
+        b.GQA_ERR_INVALID_ARG                                                   # q_dev alignment
+    assert b.gqa_attn_fwd_host(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE,
+                               1, 64, 64, 4, 3, 128, 1, 0.088, NULL, NULL) == b.GQA_ERR_INVALID_ARG
+    assert b.gqa_attn_fwd_host(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE,
+                               1, 64, 64, 4, 2, 96, 1, 0.088, NULL, NULL) == b.GQA_ERR_UNSUPPORTED
+    assert b.gqa_attn_fwd_host(NULL, NULL, NULL, NULL, NULL, NULL, NULL, NULL,
+                               1, 0, 64, 4, 2, 128, 1, 0.088, NULL, NULL) == b.GQA_OK  # empty
+
+
 def test_rope_rejects(gqa_lib):
     assert b.gqa_rope(FAKE, 1, 4, 2, 12, 0, 10000.0, NULL) == b.GQA_ERR_INVALID_ARG   # d % 8
     assert b.gqa_rope(FAKE, 1, 4, 2, 128, 0, 0.0, NULL) == b.GQA_ERR_INVALID_ARG      # theta
