@@ -34,6 +34,10 @@ __device__ __forceinline__ void cp_async16(uint32_t dst, const void *src, bool v
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;"
                  ::"r"(dst), "l"(src), "r"(valid ? 16 : 0) : "memory");
 }
+__device__ __forceinline__ void cp_async4(uint32_t dst, const void *src, bool valid) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;"
+                 ::"r"(dst), "l"(src), "r"(valid ? 4 : 0) : "memory");
+}
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 template <int N>
 __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
@@ -50,6 +54,16 @@ struct Vis {
         return true;
     }
 };
+
+// Every (query, key) pair of rows [i0, i0 + ni) x keys [j0, j0 + nj) visible?
+__device__ __forceinline__ bool block_visible(const Vis &v, int i0, int ni, int j0, int nj) {
+    if (i0 + ni > v.Tq || j0 + nj > v.Tkv) return false;
+    const int p0 = i0 + (v.Tkv - v.Tq);                 // key position of the first row
+    if (v.causal && j0 + nj - 1 > p0) return false;
+    // window: the last row's window must still reach key j0 (sinks aside)
+    if (v.window > 0 && j0 <= p0 + ni - 1 - v.window && j0 + nj > v.sinks) return false;
+    return true;
+}
 
 // ------------------------------------------------------------- rowdot ---
 __global__ void __launch_bounds__(256)
@@ -104,9 +118,14 @@ dkdv_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict
     __nv_bfloat16 *sV = sK + kKvTile * P;
     __nv_bfloat16 *sQ = sV + kKvTile * P;                // [2][kQBlk][P]
     __nv_bfloat16 *sO = sQ + 2 * kQBlk * P;              // dO, [2][kQBlk][P]
+    float *sL = reinterpret_cast<float *>(sO + 2 * kQBlk * P);   // lse, [2][kQBlk]
+    float *sD = sL + 2 * kQBlk;                                  // D,   [2][kQBlk]
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int gq = lane >> 2, tq = lane & 3;
-    const int kb = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z;
+    // key tiles in decreasing causal work (the first tiles see the most queries)
+    const int bhs = Hkv * B;
+    const int lin = blockIdx.x;
+    const int kb = lin / bhs, kvh = lin % Hkv, b = (lin / Hkv) % B;
     const int G = Hq / Hkv;
     const int k0 = kb * kKvTile;
     const float c2 = scale * 1.4426950408889634f;
@@ -126,11 +145,20 @@ dkdv_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict
     const uint32_t aK = smem_u32(sK), aV = smem_u32(sV), aQ = smem_u32(sQ), aO = smem_u32(sO);
     load_tile<D>(aK, k + (static_cast<size_t>(b) * Tkv * Hkv + kvh) * D, kstride, k0, kKvTile, Tkv);
     load_tile<D>(aV, v + (static_cast<size_t>(b) * Tkv * Hkv + kvh) * D, kstride, k0, kKvTile, Tkv);
+    const uint32_t aL = smem_u32(sL), aD = smem_u32(sD);
     auto issue_item = [&](int it) {
         const int g = it / n_qb, qb = qb0 + it % n_qb, buf = it & 1;
         const size_t base = (static_cast<size_t>(b) * Tq * Hq + kvh * G + g) * D;
         load_tile<D>(aQ + buf * kQBlk * P * 2, q + base, qstride, qb * kQBlk, kQBlk, Tq);
         load_tile<D>(aO + buf * kQBlk * P * 2, dout + base, qstride, qb * kQBlk, kQBlk, Tq);
+        // the block's softmax statistics: lse and D of its kQBlk query rows
+        const int t = threadIdx.x;
+        if (t < 2 * kQBlk) {
+            const int r = t % kQBlk, qi = qb * kQBlk + r;
+            const size_t li = (static_cast<size_t>(b) * Hq + kvh * G + g) * Tq + min(qi, Tq - 1);
+            cp_async4((t < kQBlk ? aL : aD) + (buf * kQBlk + r) * 4,
+                      (t < kQBlk ? lse : Dsum) + li, qi < Tq);
+        }
     };
     if (n_items > 0) issue_item(0);
     cp_async_commit();
@@ -147,8 +175,7 @@ dkdv_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict
         cp_async_commit();
         cp_async_wait<1>();
         __syncthreads();
-        const int g = it / n_qb, qb = qb0 + it % n_qb, buf = it & 1;
-        const int hq = kvh * G + g;
+        const int qb = qb0 + it % n_qb, buf = it & 1;
         const uint32_t bQ = aQ + buf * kQBlk * P * 2, bO = aO + buf * kQBlk * P * 2;
         // S^T (16 keys x 32 queries) and dP^T = V dO^T
         float st[4][4], dpt[4][4];
@@ -174,7 +201,10 @@ dkdv_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict
                 mma_16816(dpt[2 * np + 1], va, obf[2], obf[3]);
             }
         }
-        // P^T and dS^T, packed as A fragments over the 32 queries (2 k-steps)
+        // P^T and dS^T, packed as A fragments over the 32 queries (2 k-steps).
+        // Blocks inside the visible region skip the per-element test.
+        const bool full = block_visible(vis, qb * kQBlk, kQBlk, k0, kKvTile);
+        const float *bL = sL + buf * kQBlk, *bD = sD + buf * kQBlk;
         uint32_t pa[2][4], sa[2][4];
 #pragma unroll
         for (int n = 0; n < 4; ++n) {
@@ -182,12 +212,11 @@ dkdv_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
                 const int key = k0 + krow + gq + ((e >> 1) << 3);
-                const int qi = qb * kQBlk + n * 8 + 2 * tq + (e & 1);
+                const int ql = n * 8 + 2 * tq + (e & 1);
                 float pr = 0.0f, dsv = 0.0f;
-                if (vis(qi, key)) {
-                    const size_t li = (static_cast<size_t>(b) * Hq + hq) * Tq + qi;
-                    pr = fast_exp2(st[n][e] * c2 - lse[li] * 1.4426950408889634f);
-                    dsv = pr * (dpt[n][e] - Dsum[li]);
+                if (full || vis(qb * kQBlk + ql, key)) {
+                    pr = fast_exp2(fmaf(st[n][e], c2, -bL[ql] * 1.4426950408889634f));
+                    dsv = pr * (dpt[n][e] - bD[ql]);
                 }
                 pv[e] = pr;
                 sv[e] = dsv;
@@ -250,7 +279,10 @@ dq_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict__
     __nv_bfloat16 *sV = sK + 2 * kKBlk * P;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int gq = lane >> 2, tq = lane & 3;
-    const int qt = blockIdx.x, hq = blockIdx.y, b = blockIdx.z;
+    // query tiles in decreasing causal work (the last tiles see the most keys)
+    const int bhs = Hq * B, n_qt = (Tq + kQTile - 1) / kQTile;
+    const int lin = blockIdx.x;
+    const int qt = n_qt - 1 - lin / bhs, hq = lin % Hq, b = (lin / Hq) % B;
     const int G = Hq / Hkv, kvh = hq / G;
     const int q0 = qt * kQTile;
     const float c2 = scale * 1.4426950408889634f;
@@ -329,6 +361,8 @@ dq_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict__
                 mma_16816(dp[2 * np + 1], oa, vbf[2], vbf[3]);
             }
         }
+        // blocks inside the visible region skip the per-element test
+        const bool full = block_visible(vis, q0, kQTile, kb * kKBlk, kKBlk);
         uint32_t sa[2][4];
 #pragma unroll
         for (int n = 0; n < 4; ++n) {
@@ -338,7 +372,7 @@ dq_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict__
                 const int qi = q0 + qrow + gq + ((e >> 1) << 3);
                 const int key = kb * kKBlk + n * 8 + 2 * tq + (e & 1);
                 float dsv = 0.0f;
-                if (vis(qi, key)) {
+                if (full || vis(qi, key)) {
                     const float pr = fast_exp2(s[n][e] * c2 - lrow[e >> 1]);
                     dsv = pr * (dp[n][e] - drow[e >> 1]);
                 }
@@ -391,7 +425,7 @@ static int launch_bwd_d(const void *q, const void *k, const void *v, const void 
     if (int rc = check_cuda(cudaGetLastError(), "rowdot_kernel launch")) return rc;
     Vis vis{Tq, Tkv, causal, causal ? window : 0, sinks};
     constexpr int P = D + 8;
-    const int smem_kv = (2 * kKvTile + 4 * kQBlk) * P * 2;
+    const int smem_kv = (2 * kKvTile + 4 * kQBlk) * P * 2 + 4 * kQBlk * 4;
     const int smem_q = (2 * kQTile + 4 * kKBlk) * P * 2;
     auto kkv = dkdv_kernel<D>;
     auto kq = dq_kernel<D>;
@@ -402,15 +436,17 @@ static int launch_bwd_d(const void *q, const void *k, const void *v, const void 
                                                  smem_q), "cudaFuncSetAttribute(dq)"))
         return rc;
     if (Tkv > 0) {
-        dim3 g1((Tkv + kKvTile - 1) / kKvTile, Hkv, B);
-        kkv<<<g1, kBwThreads, smem_kv, stream>>>(
+        const long long n1 = static_cast<long long>((Tkv + kKvTile - 1) / kKvTile) * Hkv * B;
+        if (n1 > 0x7fffffffLL) return set_error(GQA_ERR_UNSUPPORTED, "backward grid too large");
+        kkv<<<static_cast<unsigned>(n1), kBwThreads, smem_kv, stream>>>(
             static_cast<const bf *>(q), static_cast<const bf *>(k), static_cast<const bf *>(v),
             static_cast<const bf *>(dout), lse, Dsum, static_cast<bf *>(dk), static_cast<bf *>(dv),
             B, Tq, Tkv, Hq, Hkv, vis, scale);
         if (int rc = check_cuda(cudaGetLastError(), "dkdv_kernel launch")) return rc;
     }
-    dim3 g2((Tq + kQTile - 1) / kQTile, Hq, B);
-    kq<<<g2, kBwThreads, smem_q, stream>>>(
+    const long long n2 = static_cast<long long>((Tq + kQTile - 1) / kQTile) * Hq * B;
+    if (n2 > 0x7fffffffLL) return set_error(GQA_ERR_UNSUPPORTED, "backward grid too large");
+    kq<<<static_cast<unsigned>(n2), kBwThreads, smem_q, stream>>>(
         static_cast<const bf *>(q), static_cast<const bf *>(k), static_cast<const bf *>(v),
         static_cast<const bf *>(dout), lse, Dsum, static_cast<bf *>(dq), B, Tq, Tkv, Hq, Hkv, vis,
         scale);
@@ -421,8 +457,6 @@ int launch_bwd(const void *q, const void *k, const void *v, const void *o, const
                const float *lse, void *dq, void *dk, void *dv, int B, int Tq, int Tkv, int Hq,
                int Hkv, int d, int causal, int window, int sinks, float scale, void *workspace,
                cudaStream_t stream) {
-    if (B > 65535 || Hq > 65535)
-        return set_error(GQA_ERR_UNSUPPORTED, "backward: B and Hq must be <= 65535");
     if (d == 128)
         return launch_bwd_d<128>(q, k, v, o, dout, lse, dq, dk, dv, B, Tq, Tkv, Hq, Hkv, causal,
                                  window, sinks, scale, workspace, stream);
