@@ -338,6 +338,13 @@ def run_ours(args, world, rank, local):
     c, dc = PREFILL, DECODE
     stream = torch.cuda.current_stream(dev)
     flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    if args.only == "next":
+        # the rows beyond the hot path alone (profiling runs of their kernels)
+        peaks, peak_kind = load_peaks()
+        nxt = measure_next_rows(dev, stream, flush, peaks, peak_kind, args.next_reps)
+        if rank == 0:
+            print(json.dumps({"next_rows": nxt}), flush=True)
+        return
     if do_pre:
         q_h, k_h, v_h = workloads.prefill_inputs(c["B"], c["T"], c["Hq"], c["Hkv"], c["d"])
         q, k, v = q_h.to(dev), k_h.to(dev), v_h.to(dev)
@@ -506,7 +513,7 @@ def main():
                     help="target seconds of oracle work for the CPU baseline")
     ap.add_argument("--ref-budget", type=float, default=90.0,
                     help="target seconds of oracle work for all steps of --impl reference")
-    ap.add_argument("--only", choices=["prefill", "decode"], default=None,
+    ap.add_argument("--only", choices=["prefill", "decode", "next"], default=None,
                     help="time one kernel family only (profiling runs)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")

@@ -35,10 +35,10 @@ constexpr int kDecThreads = (kDecWarps + 1) * 32;  // + one producer warp
 constexpr int kDecStages = GQA_DEC_STAGES;         // TMA ring depth
 constexpr int kDecChunk = GQA_DEC_CHUNK;           // keys per split (multiple of kDecBK)
 // CTAs per SM the register budget must allow (3 x 66.6 KB of shared memory
-// also fit): more stages in flight per SM
-#ifndef GQA_DEC_MIN_BLOCKS
-#define GQA_DEC_MIN_BLOCKS 3
-#endif
+// also fit): more stages in flight per SM.  Groups of more than 16 heads
+// (MB = 2) hold twice the accumulators and keep the full register budget.
+template <int MB>
+constexpr int dec_min_blocks() { return MB == 1 ? 3 : 1; }
 
 template <int D, int MB = 1>
 struct DecLayout {
@@ -65,7 +65,7 @@ __device__ __forceinline__ uint32_t swz_off(int row, int cg) {
 }
 
 template <int D, int MB>
-__global__ void __launch_bounds__(kDecThreads, GQA_DEC_MIN_BLOCKS)
+__global__ void __launch_bounds__(kDecThreads, dec_min_blocks<MB>())
 decode_split_kernel(const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v,
                     const __nv_bfloat16 *__restrict__ q, const int32_t *__restrict__ seqlens,
