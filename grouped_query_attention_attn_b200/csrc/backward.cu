@@ -1,5 +1,5 @@
 // backward.cu -- gradients of grouped-query attention: dQ, dK, dV (bf16 in and
-// out, fp32 accumulation, warp-level bf16 tensor-core tiles).
+// out, fp32 accumulation).
 //
 // With P = softmax of the masked, scaled scores (recomputed from the forward's
 // log-sum-exp) and D_i = <dO_i, O_i>:
@@ -9,12 +9,13 @@
 // the SUM over the G query heads of its group (K3 notes "GVA", "Backward:
 // view + sum": the backward of a copy is a sum).  Three kernels:
 //   rowdot  D = rowsum(dO * O)                                  (HBM-bound)
-//   dkdv    one CTA per 64 keys of one KV head; loops over every query row
-//           of the G heads of the group, so dK and dV accumulate in
-//           registers with no atomics
-//   dq      one CTA per 64 query rows of one head; loops over the keys
-// Tiles reach shared memory through double-buffered cp.async with padded
-// rows (ldmatrix is then free of bank conflicts).
+//   dkdv    tcgen05: one CTA per 128 keys of one KV head; loops over every
+//           query row of the G heads of the group, so dK and dV accumulate
+//           in tensor memory with no atomics
+//   dq      warp-level mma.sync: one CTA per 64 query rows of one head,
+//           looping over the keys; tiles reach shared memory through
+//           double-buffered cp.async with padded rows (ldmatrix is then free
+//           of bank conflicts)
 #include <cuda_bf16.h>
 #include <climits>
 
@@ -23,9 +24,7 @@
 
 namespace gqa {
 
-constexpr int kBwThreads = 128;   // 4 warps x 16 rows of the MMA M dimension
-constexpr int kKvTile = 64;       // keys per dkdv CTA
-constexpr int kQBlk = 32;         // query rows per dkdv iteration
+constexpr int kBwThreads = 128;   // dq: 4 warps x 16 rows of the MMA M dimension
 constexpr int kQTile = 64;        // query rows per dq CTA
 constexpr int kKBlk = 32;         // keys per dq iteration
 
@@ -33,10 +32,6 @@ __device__ __forceinline__ void cp_async16(uint32_t dst, const void *src, bool v
     // src-size 0 writes zeros (rows past the end of the tensor)
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;"
                  ::"r"(dst), "l"(src), "r"(valid ? 16 : 0) : "memory");
-}
-__device__ __forceinline__ void cp_async4(uint32_t dst, const void *src, bool valid) {
-    asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;"
-                 ::"r"(dst), "l"(src), "r"(valid ? 4 : 0) : "memory");
 }
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 template <int N>
@@ -104,163 +99,335 @@ __device__ __forceinline__ uint32_t tile_addr(uint32_t base, int row, int chunk)
     return base + (row * (D + 8) + chunk * 8) * 2;
 }
 
-// --------------------------------------------------------------- dk dv ---
+// ------------------------------------------------------ dk dv (tcgen05) ---
+// One CTA per 128 keys of one KV head (heaviest causal tiles first).  The K
+// and V tiles stay in shared memory; for every 128-row query block of every
+// query head of the group (an "item"):
+//   tensor pipe   S^T = K Q^T and dP^T = V dO^T into tensor memory (M = 128
+//                 keys, N = 128 queries);
+//   8 warps       P^T = exp2(S^T * scale * log2e - lse_q * log2e) and
+//                 dS^T = P^T (dP^T - D_q), bf16, written back over the first
+//                 columns of each half's S^T / dP^T (two threads per key row,
+//                 one per 64-query half);
+//   tensor pipe   dV += P^T dO and dK += dS^T Q with P^T / dS^T read from
+//                 tensor memory (dV and dK accumulate over all items).
+// Tensor memory (512 columns): S^T | dP^T | dV | dK.  Shared memory: K, V,
+// and a 2-deep ring of (Q, dO, lse, D) per item.
+constexpr int kTcBK = 128;       // keys per CTA
+constexpr int kTcBQ = 128;       // query rows per item
+constexpr int kTcThreads = 384;  // producer, MMA, 2 idle, 8 elementwise warps
+
 template <int D>
-__global__ void __launch_bounds__(kBwThreads)
-dkdv_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict__ k,
-            const __nv_bfloat16 *__restrict__ v, const __nv_bfloat16 *__restrict__ dout,
-            const float *__restrict__ lse, const float *__restrict__ Dsum,
-            __nv_bfloat16 *__restrict__ dk, __nv_bfloat16 *__restrict__ dv, int B, int Tq,
-            int Tkv, int Hq, int Hkv, Vis vis, float scale) {
-    constexpr int P = D + 8;
-    extern __shared__ __align__(16) uint8_t smem[];
-    __nv_bfloat16 *sK = reinterpret_cast<__nv_bfloat16 *>(smem);
-    __nv_bfloat16 *sV = sK + kKvTile * P;
-    __nv_bfloat16 *sQ = sV + kKvTile * P;                // [2][kQBlk][P]
-    __nv_bfloat16 *sO = sQ + 2 * kQBlk * P;              // dO, [2][kQBlk][P]
-    float *sL = reinterpret_cast<float *>(sO + 2 * kQBlk * P);   // lse, [2][kQBlk]
-    float *sD = sL + 2 * kQBlk;                                  // D,   [2][kQBlk]
+struct TcLayout {
+    static constexpr int kPanels = D / 64;
+    static constexpr int kPanel = 128 * 128;               // 128 rows x 64 bf16
+    static constexpr int kTile = kPanels * kPanel;
+    static constexpr int kOffK = 0, kOffV = kTile;
+    static constexpr int kOffQ = 2 * kTile;                // [2] Q tiles
+    static constexpr int kOffO = kOffQ + 2 * kTile;        // [2] dO tiles
+    static constexpr int kOffL = kOffO + 2 * kTile;        // [2][2][128] floats: L, D
+    static constexpr int kBytes = kOffL + 2 * 2 * kTcBQ * 4;
+    static constexpr int kSmemBytes = kBytes + 1024;
+    static constexpr uint32_t kColS = 0, kColP = 128, kColDV = 256, kColDK = 256 + D;
+};
+
+struct TcParams {
+    int B, Tq, Tkv, Hq, Hkv, G;
+    int n_kt;                         // key tiles per (b, kvh)
+    Vis vis;
+    float scale, scale_log2;
+    const float *lse, *Dsum;
+    __nv_bfloat16 *dk, *dv;
+    int *status;
+};
+
+template <int D>
+__global__ void __launch_bounds__(kTcThreads, 1)
+dkdv_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+               const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
+               const TcParams p) {
+    using Lay = TcLayout<D>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    __shared__ uint64_t kv_full, qo_full[2], qo_empty[2], s_full, p_full, acc_done;
+    __shared__ uint32_t tmem_base_sh;
+    __shared__ int abort_flag;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int gq = lane >> 2, tq = lane & 3;
-    // key tiles in decreasing causal work (the first tiles see the most queries)
-    const int bhs = Hkv * B;
-    const int lin = blockIdx.x;
-    const int kb = lin / bhs, kvh = lin % Hkv, b = (lin / Hkv) % B;
-    const int G = Hq / Hkv;
-    const int k0 = kb * kKvTile;
-    const float c2 = scale * 1.4426950408889634f;
 
-    // query rows that can see any key of this tile
-    const int off = Tkv - Tq;
-    int q_lo = 0, q_hi = Tq;
-    if (vis.causal) {
+    const int bhs = p.Hkv * p.B, lin = blockIdx.x;
+    const int kt = lin / bhs, kvh = lin % p.Hkv, b = (lin / p.Hkv) % p.B;
+    const int k0 = kt * kTcBK;
+    // query rows that can see a key of this tile
+    const int off = p.Tkv - p.Tq;
+    int q_lo = 0, q_hi = p.Tq;
+    if (p.vis.causal) {
         q_lo = max(0, k0 - off);
-        if (vis.window > 0 && k0 >= vis.sinks) q_hi = min(Tq, k0 + kKvTile - 1 + vis.window - off);
+        if (p.vis.window > 0 && k0 >= p.vis.sinks)
+            q_hi = min(p.Tq, k0 + kTcBK - 1 + p.vis.window - off);
     }
-    const int qb0 = q_lo / kQBlk;
-    const int n_qb = q_hi > q_lo ? (q_hi + kQBlk - 1) / kQBlk - qb0 : 0;
-    const int n_items = G * n_qb;
+    const int qb0 = q_lo / kTcBQ;
+    const int n_qb = q_hi > q_lo ? (q_hi + kTcBQ - 1) / kTcBQ - qb0 : 0;
+    const int n_items = p.G * n_qb;
 
-    const size_t kstride = static_cast<size_t>(Hkv) * D, qstride = static_cast<size_t>(Hq) * D;
-    const uint32_t aK = smem_u32(sK), aV = smem_u32(sV), aQ = smem_u32(sQ), aO = smem_u32(sO);
-    load_tile<D>(aK, k + (static_cast<size_t>(b) * Tkv * Hkv + kvh) * D, kstride, k0, kKvTile, Tkv);
-    load_tile<D>(aV, v + (static_cast<size_t>(b) * Tkv * Hkv + kvh) * D, kstride, k0, kKvTile, Tkv);
-    const uint32_t aL = smem_u32(sL), aD = smem_u32(sD);
-    auto issue_item = [&](int it) {
-        const int g = it / n_qb, qb = qb0 + it % n_qb, buf = it & 1;
-        const size_t base = (static_cast<size_t>(b) * Tq * Hq + kvh * G + g) * D;
-        load_tile<D>(aQ + buf * kQBlk * P * 2, q + base, qstride, qb * kQBlk, kQBlk, Tq);
-        load_tile<D>(aO + buf * kQBlk * P * 2, dout + base, qstride, qb * kQBlk, kQBlk, Tq);
-        // the block's softmax statistics: lse and D of its kQBlk query rows
-        const int t = threadIdx.x;
-        if (t < 2 * kQBlk) {
-            const int r = t % kQBlk, qi = qb * kQBlk + r;
-            const size_t li = (static_cast<size_t>(b) * Hq + kvh * G + g) * Tq + min(qi, Tq - 1);
-            cp_async4((t < kQBlk ? aL : aD) + (buf * kQBlk + r) * 4,
-                      (t < kQBlk ? lse : Dsum) + li, qi < Tq);
+    if (threadIdx.x == 0) {
+        mbar_init(&kv_full, 1);
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(&qo_full[s], 1);
+            mbar_init(&qo_empty[s], 1);
         }
-    };
-    if (n_items > 0) issue_item(0);
-    cp_async_commit();
+        mbar_init(&s_full, 1);
+        mbar_init(&p_full, 8);
+        mbar_init(&acc_done, 1);
+        abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 0) {
+        tmem_alloc(&tmem_base_sh, 512);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = tmem_base_sh;
+    float *sLD = reinterpret_cast<float *>(smem + Lay::kOffL);   // [stage][L | D][128]
 
-    float dka[D / 8][4], dva[D / 8][4];
-#pragma unroll
-    for (int n = 0; n < D / 8; ++n)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) dka[n][e] = dva[n][e] = 0.0f;
-    const int krow = 16 * warp;                          // this warp's keys in the tile
-
-    for (int it = 0; it < n_items; ++it) {
-        if (it + 1 < n_items) issue_item(it + 1);
-        cp_async_commit();
-        cp_async_wait<1>();
-        __syncthreads();
-        const int qb = qb0 + it % n_qb, buf = it & 1;
-        const uint32_t bQ = aQ + buf * kQBlk * P * 2, bO = aO + buf * kQBlk * P * 2;
-        // S^T (16 keys x 32 queries) and dP^T = V dO^T
-        float st[4][4], dpt[4][4];
-#pragma unroll
-        for (int n = 0; n < 4; ++n)
-#pragma unroll
-            for (int e = 0; e < 4; ++e) st[n][e] = dpt[n][e] = 0.0f;
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-            uint32_t ka[4], va[4];
-            const int ar = krow + (lane & 7) + (((lane >> 3) & 1) << 3), ac = 2 * kk + (lane >> 4);
-            ldsm_x4(ka, tile_addr<D>(aK, ar, ac));
-            ldsm_x4(va, tile_addr<D>(aV, ar, ac));
-#pragma unroll
-            for (int np = 0; np < 2; ++np) {
-                uint32_t qbf[4], obf[4];
-                const int br = np * 16 + (lane & 7) + ((lane >> 4) << 3), bc = 2 * kk + ((lane >> 3) & 1);
-                ldsm_x4(qbf, tile_addr<D>(bQ, br, bc));
-                ldsm_x4(obf, tile_addr<D>(bO, br, bc));
-                mma_16816(st[2 * np], ka, qbf[0], qbf[1]);
-                mma_16816(st[2 * np + 1], ka, qbf[2], qbf[3]);
-                mma_16816(dpt[2 * np], va, obf[0], obf[1]);
-                mma_16816(dpt[2 * np + 1], va, obf[2], obf[3]);
-            }
-        }
-        // P^T and dS^T, packed as A fragments over the 32 queries (2 k-steps).
-        // Blocks inside the visible region skip the per-element test.
-        const bool full = block_visible(vis, qb * kQBlk, kQBlk, k0, kKvTile);
-        const float *bL = sL + buf * kQBlk, *bD = sD + buf * kQBlk;
-        uint32_t pa[2][4], sa[2][4];
-#pragma unroll
-        for (int n = 0; n < 4; ++n) {
-            float pv[4], sv[4];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const int key = k0 + krow + gq + ((e >> 1) << 3);
-                const int ql = n * 8 + 2 * tq + (e & 1);
-                float pr = 0.0f, dsv = 0.0f;
-                if (full || vis(qb * kQBlk + ql, key)) {
-                    pr = fast_exp2(fmaf(st[n][e], c2, -bL[ql] * 1.4426950408889634f));
-                    dsv = pr * (dpt[n][e] - bD[ql]);
+    if (warp == 0) {
+        // ------------------------------------------------ TMA producer ----
+        const bool leader = elect_one();
+        if (n_items > 0) {
+            if (leader) {
+                tma_prefetch_desc(&tm_q);
+                tma_prefetch_desc(&tm_o);
+                mbar_expect_tx(&kv_full, 2 * Lay::kTile);
+                for (int pn = 0; pn < Lay::kPanels; ++pn) {
+                    tma_load_4d(smem + Lay::kOffK + pn * Lay::kPanel, &tm_k, &kv_full, pn * 64,
+                                kvh, k0, b);
+                    tma_load_4d(smem + Lay::kOffV + pn * Lay::kPanel, &tm_v, &kv_full, pn * 64,
+                                kvh, k0, b);
                 }
-                pv[e] = pr;
-                sv[e] = dsv;
             }
-            const int ks = n >> 1, hi = n & 1;
-            pa[ks][2 * hi] = pack_bf16x2(pv[0], pv[1]);
-            pa[ks][2 * hi + 1] = pack_bf16x2(pv[2], pv[3]);
-            sa[ks][2 * hi] = pack_bf16x2(sv[0], sv[1]);
-            sa[ks][2 * hi + 1] = pack_bf16x2(sv[2], sv[3]);
+            __syncwarp();
+            int issued = 0;
+            for (int it = 0; it < n_items; ++it) {
+                const int st = it & 1;
+                const int g = it / n_qb, q0 = (qb0 + it % n_qb) * kTcBQ, hq = kvh * p.G + g;
+                if (!__all_sync(0xffffffffu, mbar_wait(&qo_empty[st], ((it >> 1) & 1) ^ 1,
+                                                       &abort_flag, p.status)))
+                    break;
+                // the item's softmax statistics, lse in log2 units (rows past Tq: 0)
+                const size_t lrow = (static_cast<size_t>(b) * p.Hq + hq) * p.Tq;
+                float *L = sLD + st * 2 * kTcBQ, *Dd = L + kTcBQ;
+#pragma unroll
+                for (int e = 0; e < kTcBQ / 32; ++e) {
+                    const int r = lane + 32 * e, qi = q0 + r;
+                    L[r] = qi < p.Tq ? p.lse[lrow + qi] * 1.4426950408889634f : 0.0f;
+                    Dd[r] = qi < p.Tq ? p.Dsum[lrow + qi] : 0.0f;
+                }
+                __syncwarp();
+                if (leader) {
+                    mbar_expect_tx(&qo_full[st], 2 * Lay::kTile);
+                    for (int pn = 0; pn < Lay::kPanels; ++pn) {
+                        tma_load_4d(smem + Lay::kOffQ + st * Lay::kTile + pn * Lay::kPanel, &tm_q,
+                                    &qo_full[st], pn * 64, hq, q0, b);
+                        tma_load_4d(smem + Lay::kOffO + st * Lay::kTile + pn * Lay::kPanel, &tm_o,
+                                    &qo_full[st], pn * 64, hq, q0, b);
+                    }
+                }
+                __syncwarp();
+                issued = it + 1;
+            }
+            // copies still in flight land before the block exits
+            mbar_wait(&kv_full, 0, &abort_flag, p.status, 1000000ull);
+            for (int it = max(0, issued - 2); it < issued; ++it)
+                mbar_wait(&qo_full[it & 1], (it >> 1) & 1, &abort_flag, p.status, 1000000ull);
         }
-        // dV += P^T dO,  dK += dS^T Q   (B operands: dO / Q rows = queries, trans)
+    } else if (warp == 1 && lane == 0) {
+        // ------------------------------------------------- MMA issuer ----
+        if (n_items > 0) {
+            constexpr uint32_t idesc_s = umma_idesc_bf16(kTcBK, kTcBQ, 0, 0);
+            constexpr uint32_t idesc_o = umma_idesc_bf16(kTcBK, D, 0, 1);
+            const uint32_t base = smem_u32(smem);
+            const uint64_t dK = umma_smem_desc(base + Lay::kOffK, 16, 1024);
+            const uint64_t dV = umma_smem_desc(base + Lay::kOffV, 16, 1024);
+            auto wait = [&](uint64_t *bar, uint32_t parity) {
+                return mbar_wait(bar, parity, &abort_flag, p.status);
+            };
+            bool ok = wait(&kv_full, 0);
+            for (int it = 0; ok && it < n_items; ++it) {
+                const int st = it & 1;
+                if (!(ok = wait(&qo_full[st], (it >> 1) & 1))) break;
+                tc_fence_after();
+                const uint32_t aQ = base + Lay::kOffQ + st * Lay::kTile;
+                const uint32_t aO = base + Lay::kOffO + st * Lay::kTile;
+                // S^T = K Q^T, dP^T = V dO^T: K-major A and B (+32 B per 16 of d)
+                const uint64_t bq = umma_smem_desc(aQ, 16, 1024), bo = umma_smem_desc(aO, 16, 1024);
 #pragma unroll
-        for (int ks = 0; ks < 2; ++ks) {
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint32_t off = ((kk >> 2) * Lay::kPanel + (kk & 3) * 32) >> 4;
+                    umma_ss(tmem + Lay::kColS, dK + off, bq + off, idesc_s, kk > 0);
+                }
 #pragma unroll
-            for (int dp = 0; dp < D / 16; ++dp) {
-                uint32_t ob[4], qbt[4];
-                const int r = ks * 16 + (lane & 7) + (((lane >> 3) & 1) << 3), c = 2 * dp + (lane >> 4);
-                ldsm_x4_trans(ob, tile_addr<D>(bO, r, c));
-                ldsm_x4_trans(qbt, tile_addr<D>(bQ, r, c));
-                mma_16816(dva[2 * dp], pa[ks], ob[0], ob[1]);
-                mma_16816(dva[2 * dp + 1], pa[ks], ob[2], ob[3]);
-                mma_16816(dka[2 * dp], sa[ks], qbt[0], qbt[1]);
-                mma_16816(dka[2 * dp + 1], sa[ks], qbt[2], qbt[3]);
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint32_t off = ((kk >> 2) * Lay::kPanel + (kk & 3) * 32) >> 4;
+                    umma_ss(tmem + Lay::kColP, dV + off, bo + off, idesc_s, kk > 0);
+                }
+                tc_commit(&s_full);
+                if (!(ok = wait(&p_full, it & 1))) break;
+                tc_fence_after();
+                // dV += P^T dO, dK += dS^T Q: A from tensor memory (half h of the
+                // queries at columns 64 h .. 64 h + 31, 8 per 16 queries), B
+                // MN-major (+2048 B per 16 queries)
+                const uint64_t vo = umma_smem_desc(aO, Lay::kPanel, 1024);
+                const uint64_t vq = umma_smem_desc(aQ, Lay::kPanel, 1024);
+#pragma unroll
+                for (int kk = 0; kk < kTcBQ / 16; ++kk) {
+                    const uint32_t ca = (kk >> 2) * 64 + (kk & 3) * 8;
+                    umma_ts(tmem + Lay::kColDV, tmem + Lay::kColS + ca, vo + kk * (2048 >> 4),
+                            idesc_o, (it > 0 || kk > 0) ? 1u : 0u);
+                }
+#pragma unroll
+                for (int kk = 0; kk < kTcBQ / 16; ++kk) {
+                    const uint32_t ca = (kk >> 2) * 64 + (kk & 3) * 8;
+                    umma_ts(tmem + Lay::kColDK, tmem + Lay::kColP + ca, vq + kk * (2048 >> 4),
+                            idesc_o, (it > 0 || kk > 0) ? 1u : 0u);
+                }
+                tc_commit(&qo_empty[st]);
+            }
+            tc_commit(&acc_done);
+            mbar_wait(&acc_done, 0, &abort_flag, p.status, 1000000000ull);
+        }
+    } else if (warp >= 4) {
+        // ---------------------------------------- elementwise + epilogue ----
+        const int h = (warp - 4) >> 2;                  // query half of an item
+        const int g4 = warp & 3;                        // lane group
+        const int r = (g4 << 5) + lane;                 // key row = tensor-memory lane
+        const int key = k0 + r;
+        const uint32_t lane_addr = tmem + ((static_cast<uint32_t>(g4) * 32u) << 16);
+        bool ok = true;
+        for (int it = 0; it < n_items; ++it) {
+            const int st = it & 1, q0 = (qb0 + it % n_qb) * kTcBQ;
+            // qo_full also publishes the item's lse / D the producer stored
+            if (!(ok = __all_sync(0xffffffffu,
+                                  mbar_wait(&qo_full[st], (it >> 1) & 1, &abort_flag, p.status) &&
+                                  mbar_wait(&s_full, it & 1, &abort_flag, p.status))))
+                break;
+            tc_fence_after();
+            const bool full = block_visible(p.vis, q0, kTcBQ, k0, kTcBK);
+            const float *L = sLD + st * 2 * kTcBQ + 64 * h, *Dd = L + kTcBQ;
+#pragma unroll
+            for (int c = 0; c < 2; ++c) {
+                const uint32_t col = 64 * h + 32 * c;
+                uint32_t sv[32], dp[32];
+                tmem_ld32(lane_addr + Lay::kColS + col, sv);
+                tmem_ld32(lane_addr + Lay::kColP + col, dp);
+                tmem_wait_ld();
+                uint32_t pk[16], dk[16];
+#pragma unroll
+                for (int e = 0; e < 32; e += 2) {
+                    float pr[2], ds[2];
+#pragma unroll
+                    for (int t = 0; t < 2; ++t) {
+                        const int ql = 32 * c + e + t;
+                        pr[t] = fast_exp2(fmaf(__uint_as_float(sv[e + t]), p.scale_log2, -L[ql]));
+                        if (!full && !p.vis(q0 + 64 * h + ql, key)) pr[t] = 0.0f;
+                        ds[t] = pr[t] * (__uint_as_float(dp[e + t]) - Dd[ql]);
+                    }
+                    pk[e / 2] = pack_bf16x2(pr[0], pr[1]);
+                    dk[e / 2] = pack_bf16x2(ds[0], ds[1]);
+                }
+                // over columns this thread has already read (its own half)
+                tmem_st16(lane_addr + Lay::kColS + 64 * h + 16 * c, pk);
+                tmem_st16(lane_addr + Lay::kColP + 64 * h + 16 * c, dk);
+            }
+            tmem_wait_st();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&p_full);
+        }
+        // ---- epilogue: dV, dK * scale -> bf16 (half h writes columns h D/2 ..) ----
+        if (ok && n_items > 0)
+            ok = __all_sync(0xffffffffu, mbar_wait(&acc_done, 0, &abort_flag, p.status));
+        tc_fence_after();
+        // the tensor-memory loads are warp-collective: every lane loads, and
+        // only rows of real keys are stored
+        const bool have = ok && n_items > 0;            // warp-uniform
+        const size_t rowoff = ((static_cast<size_t>(b) * p.Tkv + min(key, p.Tkv - 1)) * p.Hkv +
+                               kvh) * D;
+#pragma unroll
+        for (int m = 0; m < 2; ++m) {                   // dV, then dK
+            __nv_bfloat16 *dst = (m ? p.dk : p.dv) + rowoff + (D / 2) * h;
+            const float f = m ? p.scale : 1.0f;
+#pragma unroll
+            for (int c = 0; c < D / 64; ++c) {
+                uint32_t v[32];
+                if (have) {
+                    tmem_ld32(lane_addr + (m ? Lay::kColDK : Lay::kColDV) + (D / 2) * h + 32 * c, v);
+                    tmem_wait_ld();
+                } else {
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) v[e] = 0u;
+                }
+                if (key < p.Tkv) {
+                    uint4 *d4 = reinterpret_cast<uint4 *>(dst + 32 * c);
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const uint32_t *w = &v[8 * e];
+                        d4[e] = make_uint4(
+                            pack_bf16x2(__uint_as_float(w[0]) * f, __uint_as_float(w[1]) * f),
+                            pack_bf16x2(__uint_as_float(w[2]) * f, __uint_as_float(w[3]) * f),
+                            pack_bf16x2(__uint_as_float(w[4]) * f, __uint_as_float(w[5]) * f),
+                            pack_bf16x2(__uint_as_float(w[6]) * f, __uint_as_float(w[7]) * f));
+                    }
+                }
             }
         }
-        __syncthreads();                                 // buffer `buf` is refilled next
     }
-    cp_async_wait<0>();
 
-    // write dK (scaled) and dV for this warp's 16 keys
-#pragma unroll
-    for (int h2 = 0; h2 < 2; ++h2) {
-        const int key = k0 + krow + gq + 8 * h2;
-        if (key >= Tkv) continue;
-        const size_t rowoff = ((static_cast<size_t>(b) * Tkv + key) * Hkv + kvh) * D;
-#pragma unroll
-        for (int n = 0; n < D / 8; ++n) {
-            const int c = n * 8 + 2 * tq;
-            *reinterpret_cast<__nv_bfloat162 *>(dk + rowoff + c) =
-                __floats2bfloat162_rn(dka[n][2 * h2] * scale, dka[n][2 * h2 + 1] * scale);
-            *reinterpret_cast<__nv_bfloat162 *>(dv + rowoff + c) =
-                __floats2bfloat162_rn(dva[n][2 * h2], dva[n][2 * h2 + 1]);
-        }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        __syncwarp();
+        tc_fence_after();
+        tmem_dealloc(tmem, 512);
     }
+}
+
+template <int D>
+static int launch_dkdv_tc(const void *q, const void *k, const void *v, const void *dout,
+                          const float *lse, const float *Dsum, void *dk, void *dv, int B, int Tq,
+                          int Tkv, int Hq, int Hkv, Vis vis, float scale, cudaStream_t stream) {
+    TcParams prm;
+    prm.B = B;
+    prm.Tq = Tq;
+    prm.Tkv = Tkv;
+    prm.Hq = Hq;
+    prm.Hkv = Hkv;
+    prm.G = Hq / Hkv;
+    prm.n_kt = (Tkv + kTcBK - 1) / kTcBK;
+    prm.vis = vis;
+    prm.scale = scale;
+    prm.scale_log2 = scale * 1.4426950408889634f;
+    prm.lse = lse;
+    prm.Dsum = Dsum;
+    prm.dk = static_cast<__nv_bfloat16 *>(dk);
+    prm.dv = static_cast<__nv_bfloat16 *>(dv);
+    prm.status = device_status_ptr();
+    if (!prm.status) return GQA_ERR_CUDA;
+    const long long blocks = static_cast<long long>(prm.n_kt) * Hkv * B;
+    if (blocks > 0x7fffffffLL) return set_error(GQA_ERR_UNSUPPORTED, "backward grid too large");
+    CUtensorMap tq, tk, tv, to;
+    if (int rc = encode_tmap_bf16_4d(&tq, q, D, Hq, Tq, B, 64, 1, kTcBQ, 1, 1)) return rc;
+    if (int rc = encode_tmap_bf16_4d(&to, dout, D, Hq, Tq, B, 64, 1, kTcBQ, 1, 1)) return rc;
+    if (int rc = encode_tmap_bf16_4d(&tk, k, D, Hkv, Tkv, B, 64, 1, kTcBK, 1, 1)) return rc;
+    if (int rc = encode_tmap_bf16_4d(&tv, v, D, Hkv, Tkv, B, 64, 1, kTcBK, 1, 1)) return rc;
+    auto kern = dkdv_tc_kernel<D>;
+    const int smem = TcLayout<D>::kSmemBytes;
+    if (int rc = check_cuda(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                 smem), "cudaFuncSetAttribute(dkdv_tc)"))
+        return rc;
+    kern<<<static_cast<unsigned>(blocks), kTcThreads, smem, stream>>>(tq, tk, tv, to, prm);
+    return check_cuda(cudaGetLastError(), "dkdv_tc_kernel launch");
 }
 
 // ------------------------------------------------------------------ dq ---
@@ -425,24 +592,15 @@ static int launch_bwd_d(const void *q, const void *k, const void *v, const void 
     if (int rc = check_cuda(cudaGetLastError(), "rowdot_kernel launch")) return rc;
     Vis vis{Tq, Tkv, causal, causal ? window : 0, sinks};
     constexpr int P = D + 8;
-    const int smem_kv = (2 * kKvTile + 4 * kQBlk) * P * 2 + 4 * kQBlk * 4;
     const int smem_q = (2 * kQTile + 4 * kKBlk) * P * 2;
-    auto kkv = dkdv_kernel<D>;
     auto kq = dq_kernel<D>;
-    if (int rc = check_cuda(cudaFuncSetAttribute(kkv, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                 smem_kv), "cudaFuncSetAttribute(dkdv)"))
-        return rc;
     if (int rc = check_cuda(cudaFuncSetAttribute(kq, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                                  smem_q), "cudaFuncSetAttribute(dq)"))
         return rc;
     if (Tkv > 0) {
-        const long long n1 = static_cast<long long>((Tkv + kKvTile - 1) / kKvTile) * Hkv * B;
-        if (n1 > 0x7fffffffLL) return set_error(GQA_ERR_UNSUPPORTED, "backward grid too large");
-        kkv<<<static_cast<unsigned>(n1), kBwThreads, smem_kv, stream>>>(
-            static_cast<const bf *>(q), static_cast<const bf *>(k), static_cast<const bf *>(v),
-            static_cast<const bf *>(dout), lse, Dsum, static_cast<bf *>(dk), static_cast<bf *>(dv),
-            B, Tq, Tkv, Hq, Hkv, vis, scale);
-        if (int rc = check_cuda(cudaGetLastError(), "dkdv_kernel launch")) return rc;
+        if (int rc = launch_dkdv_tc<D>(q, k, v, dout, lse, Dsum, dk, dv, B, Tq, Tkv, Hq, Hkv, vis,
+                                       scale, stream))
+            return rc;
     }
     const long long n2 = static_cast<long long>((Tq + kQTile - 1) / kQTile) * Hq * B;
     if (n2 > 0x7fffffffLL) return set_error(GQA_ERR_UNSUPPORTED, "backward grid too large");
