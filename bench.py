@@ -294,7 +294,7 @@ def measure_next_rows(dev, stream, flush, peaks, peak_kind, reps):
                      dtype=torch.uint8, device=dev)
     ms = time_median(lambda: gqa.attn_bwd(q, k, v, o, lse, do, workspace=ws), flush, stream, reps)
     out["backward"] = tensor_row(10 * c["Hq"] * 128 * visible_pairs(c["T"], c["T"]), ms,
-                                 dict(c, kernels="rowdot + dkdv + dq (mma.sync)"))
+                                 dict(c, kernels="rowdot + dkdv (tcgen05) + dq (tcgen05)"))
     # RoPE of q and k of the same workload, in place (read + write)
     ms = time_median(lambda: gqa.rope_qk_(q, k, 0), flush, stream, reps)
     out["rope_qk"] = hbm_row(2 * (q.numel() + k.numel()) * 2, ms, dict(c, theta=10000.0))

@@ -12,10 +12,8 @@
 //   dkdv    tcgen05: one CTA per 128 keys of one KV head; loops over every
 //           query row of the G heads of the group, so dK and dV accumulate
 //           in tensor memory with no atomics
-//   dq      warp-level mma.sync: one CTA per 64 query rows of one head,
-//           looping over the keys; tiles reach shared memory through
-//           double-buffered cp.async with padded rows (ldmatrix is then free
-//           of bank conflicts)
+//   dq      tcgen05: one CTA per 128-row M tile (the group's heads packed by
+//           position, as in the forward), looping over the visible keys
 #include <cuda_bf16.h>
 #include <climits>
 
@@ -23,19 +21,6 @@
 #include "internal.h"
 
 namespace gqa {
-
-constexpr int kBwThreads = 128;   // dq: 4 warps x 16 rows of the MMA M dimension
-constexpr int kQTile = 64;        // query rows per dq CTA
-constexpr int kKBlk = 32;         // keys per dq iteration
-
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void *src, bool valid) {
-    // src-size 0 writes zeros (rows past the end of the tensor)
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;"
-                 ::"r"(dst), "l"(src), "r"(valid ? 16 : 0) : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-template <int N>
-__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 
 // Visibility of key j to the query row at position i (causal bottom-right,
 // optional sliding window with sinks).
@@ -78,25 +63,6 @@ rowdot_kernel(const __nv_bfloat16 *__restrict__ dout, const __nv_bfloat16 *__res
     }
     for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
     if (lane == 0) Dsum[(static_cast<size_t>(b) * H + h) * T + t] = acc;
-}
-
-// Copy `rows` rows of D bf16 (global row stride gstride elements) starting at
-// row r0 into shared memory with row pitch D + 8; rows >= nrows are zeros.
-template <int D>
-__device__ __forceinline__ void load_tile(uint32_t sdst, const __nv_bfloat16 *g, size_t gstride,
-                                          int r0, int rows, int nrows) {
-    constexpr int kChunks = D / 8;
-    for (int idx = threadIdx.x; idx < rows * kChunks; idx += kBwThreads) {
-        const int r = idx / kChunks, c = idx % kChunks;
-        const bool ok = r0 + r < nrows;
-        const __nv_bfloat16 *src = g + static_cast<size_t>(ok ? r0 + r : 0) * gstride + c * 8;
-        cp_async16(sdst + (r * (D + 8) + c * 8) * 2, src, ok);
-    }
-}
-
-template <int D>
-__device__ __forceinline__ uint32_t tile_addr(uint32_t base, int row, int chunk) {
-    return base + (row * (D + 8) + chunk * 8) * 2;
 }
 
 // ------------------------------------------------------ dk dv (tcgen05) ---
@@ -430,149 +396,305 @@ static int launch_dkdv_tc(const void *q, const void *k, const void *v, const voi
     return check_cuda(cudaGetLastError(), "dkdv_tc_kernel launch");
 }
 
-// ------------------------------------------------------------------ dq ---
+// --------------------------------------------------------- dq (tcgen05) ---
+// One CTA per 128-row M tile: the G query heads of one KV group at
+// P = floor(128 / G) positions, as in the forward (one 3-D TMA box; every K / V
+// tile serves the whole group).  For every visible 128-key tile:
+//   tensor pipe   S = Q K^T and dP = dO V^T into tensor memory;
+//   8 warps       dS = P (dP - D_row), P = exp2(S * scale * log2e - lse_row *
+//                 log2e), bf16, over the first columns of each half's S
+//                 (two threads per row, one per 64-key half);
+//   tensor pipe   dQ += dS K with dS read from tensor memory.
+// Tensor memory: S | dP | dQ.  Shared memory: Q, dO, 2-deep K and V rings.
+constexpr int kDqBN = 128;       // keys per tile
+
 template <int D>
-__global__ void __launch_bounds__(kBwThreads)
-dq_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict__ k,
-          const __nv_bfloat16 *__restrict__ v, const __nv_bfloat16 *__restrict__ dout,
-          const float *__restrict__ lse, const float *__restrict__ Dsum,
-          __nv_bfloat16 *__restrict__ dq, int B, int Tq, int Tkv, int Hq, int Hkv, Vis vis,
-          float scale) {
-    constexpr int P = D + 8;
-    extern __shared__ __align__(16) uint8_t smem[];
-    __nv_bfloat16 *sQ = reinterpret_cast<__nv_bfloat16 *>(smem);   // [kQTile][P]
-    __nv_bfloat16 *sO = sQ + kQTile * P;                            // dO
-    __nv_bfloat16 *sK = sO + kQTile * P;                            // [2][kKBlk][P]
-    __nv_bfloat16 *sV = sK + 2 * kKBlk * P;
+struct DqLayout {
+    static constexpr int kPanels = D / 64;
+    static constexpr int kPanel = 128 * 128;               // 128 rows x 64 bf16
+    static constexpr int kTile = kPanels * kPanel;
+    static constexpr int kOffQ = 0, kOffO = kTile;
+    static constexpr int kOffK = 2 * kTile;                // [2]
+    static constexpr int kOffV = kOffK + 2 * kTile;        // [2]
+    static constexpr int kBytes = kOffV + 2 * kTile;
+    static constexpr int kSmemBytes = kBytes + 1024;
+    static constexpr uint32_t kColS = 0, kColP = 128, kColDQ = 256;
+};
+
+struct DqParams {
+    int B, Tq, Tkv, Hq, Hkv, G, P;    // P = positions per M tile
+    int n_mt;                         // M tiles per (b, kvh)
+    Vis vis;
+    float scale, scale_log2;
+    const float *lse, *Dsum;
+    __nv_bfloat16 *dq;
+    int *status;
+};
+
+template <int D>
+__global__ void __launch_bounds__(kTcThreads, 1)
+dq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_o,
+             const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+             const DqParams p) {
+    using Lay = DqLayout<D>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    __shared__ uint64_t qo_full, kv_full[2], kv_empty[2], s_full, p_full, acc_done;
+    __shared__ uint32_t tmem_base_sh;
+    __shared__ int abort_flag;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int gq = lane >> 2, tq = lane & 3;
-    // query tiles in decreasing causal work (the last tiles see the most keys)
-    const int bhs = Hq * B, n_qt = (Tq + kQTile - 1) / kQTile;
-    const int lin = blockIdx.x;
-    const int qt = n_qt - 1 - lin / bhs, hq = lin % Hq, b = (lin / Hq) % B;
-    const int G = Hq / Hkv, kvh = hq / G;
-    const int q0 = qt * kQTile;
-    const float c2 = scale * 1.4426950408889634f;
-    const int off = Tkv - Tq;
 
-    // key blocks: the sink blocks, then the window / causal range
-    const int q_last = min(Tq, q0 + kQTile) - 1;
-    int kend = Tkv;
-    if (vis.causal) kend = min(Tkv, q_last + off + 1);
+    // M tiles in decreasing causal work (the last positions see the most keys)
+    const int bhs = p.Hkv * p.B, lin = blockIdx.x;
+    const int mt = p.n_mt - 1 - lin / bhs, kvh = lin % p.Hkv, b = (lin / p.Hkv) % p.B;
+    const int t0 = mt * p.P;
+    const int last_pos = min(t0 + p.P, p.Tq) - 1;
+    const int off = p.Tkv - p.Tq;
+    int kv_end = p.Tkv;
+    if (p.vis.causal) kv_end = min(p.Tkv, last_pos + off + 1);
     int n_sink = 0, first = 0;
-    if (vis.causal && vis.window > 0 && kend > 0) {
-        n_sink = (min(vis.sinks, kend) + kKBlk - 1) / kKBlk;
-        first = max(n_sink, max(q0 + off - vis.window + 1, 0) / kKBlk);
+    if (p.vis.window > 0 && kv_end > 0) {
+        n_sink = (min(p.vis.sinks, kv_end) + kDqBN - 1) / kDqBN;
+        first = max(n_sink, max(t0 + off - p.vis.window + 1, 0) / kDqBN);
     }
-    const int last = kend > 0 ? (kend + kKBlk - 1) / kKBlk : 0;
-    const int n_kb = n_sink + max(0, last - first);
-    auto block_of = [&](int j) { return j < n_sink ? j : first + (j - n_sink); };
+    const int last = kv_end > 0 ? (kv_end + kDqBN - 1) / kDqBN : 0;
+    const int n_kv = n_sink + max(0, last - first);
+    auto tile_of = [&](int j) { return j < n_sink ? j : first + (j - n_sink); };
 
-    const size_t kstride = static_cast<size_t>(Hkv) * D, qstride = static_cast<size_t>(Hq) * D;
-    const size_t qbase = (static_cast<size_t>(b) * Tq * Hq + hq) * D;
-    const size_t kbase = (static_cast<size_t>(b) * Tkv * Hkv + kvh) * D;
-    const uint32_t aQ = smem_u32(sQ), aO = smem_u32(sO), aK = smem_u32(sK), aV = smem_u32(sV);
-    load_tile<D>(aQ, q + qbase, qstride, q0, kQTile, Tq);
-    load_tile<D>(aO, dout + qbase, qstride, q0, kQTile, Tq);
-    auto issue = [&](int j) {
-        const int buf = j & 1, kb = block_of(j);
-        load_tile<D>(aK + buf * kKBlk * P * 2, k + kbase, kstride, kb * kKBlk, kKBlk, Tkv);
-        load_tile<D>(aV + buf * kKBlk * P * 2, v + kbase, kstride, kb * kKBlk, kKBlk, Tkv);
-    };
-    if (n_kb > 0) issue(0);
-    cp_async_commit();
-
-    const int qrow = 16 * warp;
-    float dqa[D / 8][4];
-#pragma unroll
-    for (int n = 0; n < D / 8; ++n)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) dqa[n][e] = 0.0f;
-    // per-row softmax statistics of this lane's two rows
-    float lrow[2], drow[2];
-#pragma unroll
-    for (int h2 = 0; h2 < 2; ++h2) {
-        const int qi = q0 + qrow + gq + 8 * h2;
-        const size_t li = (static_cast<size_t>(b) * Hq + hq) * Tq + min(qi, Tq - 1);
-        lrow[h2] = lse[li] * 1.4426950408889634f;
-        drow[h2] = Dsum[li];
-    }
-
-    for (int j = 0; j < n_kb; ++j) {
-        if (j + 1 < n_kb) issue(j + 1);
-        cp_async_commit();
-        cp_async_wait<1>();
-        __syncthreads();
-        const int buf = j & 1, kb = block_of(j);
-        const uint32_t bK = aK + buf * kKBlk * P * 2, bV = aV + buf * kKBlk * P * 2;
-        float s[4][4], dp[4][4];
-#pragma unroll
-        for (int n = 0; n < 4; ++n)
-#pragma unroll
-            for (int e = 0; e < 4; ++e) s[n][e] = dp[n][e] = 0.0f;
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-            uint32_t qa[4], oa[4];
-            const int ar = qrow + (lane & 7) + (((lane >> 3) & 1) << 3), ac = 2 * kk + (lane >> 4);
-            ldsm_x4(qa, tile_addr<D>(aQ, ar, ac));
-            ldsm_x4(oa, tile_addr<D>(aO, ar, ac));
-#pragma unroll
-            for (int np = 0; np < 2; ++np) {
-                uint32_t kbf[4], vbf[4];
-                const int br = np * 16 + (lane & 7) + ((lane >> 4) << 3), bc = 2 * kk + ((lane >> 3) & 1);
-                ldsm_x4(kbf, tile_addr<D>(bK, br, bc));
-                ldsm_x4(vbf, tile_addr<D>(bV, br, bc));
-                mma_16816(s[2 * np], qa, kbf[0], kbf[1]);
-                mma_16816(s[2 * np + 1], qa, kbf[2], kbf[3]);
-                mma_16816(dp[2 * np], oa, vbf[0], vbf[1]);
-                mma_16816(dp[2 * np + 1], oa, vbf[2], vbf[3]);
-            }
+    if (threadIdx.x == 0) {
+        mbar_init(&qo_full, 1);
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(&kv_full[s], 1);
+            mbar_init(&kv_empty[s], 1);
         }
-        // blocks inside the visible region skip the per-element test
-        const bool full = block_visible(vis, q0, kQTile, kb * kKBlk, kKBlk);
-        uint32_t sa[2][4];
-#pragma unroll
-        for (int n = 0; n < 4; ++n) {
-            float sv[4];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const int qi = q0 + qrow + gq + ((e >> 1) << 3);
-                const int key = kb * kKBlk + n * 8 + 2 * tq + (e & 1);
-                float dsv = 0.0f;
-                if (full || vis(qi, key)) {
-                    const float pr = fast_exp2(s[n][e] * c2 - lrow[e >> 1]);
-                    dsv = pr * (dp[n][e] - drow[e >> 1]);
+        mbar_init(&s_full, 1);
+        mbar_init(&p_full, 8);
+        mbar_init(&acc_done, 1);
+        abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 0) {
+        tmem_alloc(&tmem_base_sh, 512);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = tmem_base_sh;
+
+    if (warp == 0) {
+        // ------------------------------------------------ TMA producer ----
+        const bool leader = elect_one();
+        if (n_kv > 0) {
+            if (leader) {
+                tma_prefetch_desc(&tm_k);
+                tma_prefetch_desc(&tm_v);
+                const uint32_t box = 64u * p.G * p.P * 2u;
+                mbar_expect_tx(&qo_full, 2 * Lay::kPanels * box);
+                for (int pn = 0; pn < Lay::kPanels; ++pn) {
+                    tma_load_4d(smem + Lay::kOffQ + pn * Lay::kPanel, &tm_q, &qo_full, pn * 64,
+                                kvh * p.G, t0, b);
+                    tma_load_4d(smem + Lay::kOffO + pn * Lay::kPanel, &tm_o, &qo_full, pn * 64,
+                                kvh * p.G, t0, b);
                 }
-                sv[e] = dsv;
             }
-            const int ks = n >> 1, hi = n & 1;
-            sa[ks][2 * hi] = pack_bf16x2(sv[0], sv[1]);
-            sa[ks][2 * hi + 1] = pack_bf16x2(sv[2], sv[3]);
+            __syncwarp();
+            int issued = 0;
+            for (int j = 0; j < n_kv; ++j) {
+                const int st = j & 1;
+                if (!__all_sync(0xffffffffu, mbar_wait(&kv_empty[st], ((j >> 1) & 1) ^ 1,
+                                                       &abort_flag, p.status)))
+                    break;
+                if (leader) {
+                    mbar_expect_tx(&kv_full[st], 2 * Lay::kTile);
+                    const int row = tile_of(j) * kDqBN;
+                    for (int pn = 0; pn < Lay::kPanels; ++pn) {
+                        tma_load_4d(smem + Lay::kOffK + st * Lay::kTile + pn * Lay::kPanel, &tm_k,
+                                    &kv_full[st], pn * 64, kvh, row, b);
+                        tma_load_4d(smem + Lay::kOffV + st * Lay::kTile + pn * Lay::kPanel, &tm_v,
+                                    &kv_full[st], pn * 64, kvh, row, b);
+                    }
+                }
+                __syncwarp();
+                issued = j + 1;
+            }
+            // copies still in flight land before the block exits
+            mbar_wait(&qo_full, 0, &abort_flag, p.status, 1000000ull);
+            for (int j = max(0, issued - 2); j < issued; ++j)
+                mbar_wait(&kv_full[j & 1], (j >> 1) & 1, &abort_flag, p.status, 1000000ull);
         }
-        // dQ += dS K   (B operand: K rows = keys, trans)
+    } else if (warp == 1 && lane == 0) {
+        // ------------------------------------------------- MMA issuer ----
+        if (n_kv > 0) {
+            constexpr uint32_t idesc_s = umma_idesc_bf16(128, kDqBN, 0, 0);
+            constexpr uint32_t idesc_o = umma_idesc_bf16(128, D, 0, 1);
+            const uint32_t base = smem_u32(smem);
+            const uint64_t dQt = umma_smem_desc(base + Lay::kOffQ, 16, 1024);
+            const uint64_t dOt = umma_smem_desc(base + Lay::kOffO, 16, 1024);
+            auto wait = [&](uint64_t *bar, uint32_t parity) {
+                return mbar_wait(bar, parity, &abort_flag, p.status);
+            };
+            bool ok = wait(&qo_full, 0);
+            for (int j = 0; ok && j < n_kv; ++j) {
+                const int st = j & 1;
+                if (!(ok = wait(&kv_full[st], (j >> 1) & 1))) break;
+                tc_fence_after();
+                const uint32_t aK = base + Lay::kOffK + st * Lay::kTile;
+                const uint32_t aV = base + Lay::kOffV + st * Lay::kTile;
+                // S = Q K^T, dP = dO V^T: K-major A and B (+32 B per 16 of d)
+                const uint64_t bk = umma_smem_desc(aK, 16, 1024), bv = umma_smem_desc(aV, 16, 1024);
 #pragma unroll
-        for (int ks = 0; ks < 2; ++ks)
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint32_t o16 = ((kk >> 2) * Lay::kPanel + (kk & 3) * 32) >> 4;
+                    umma_ss(tmem + Lay::kColS, dQt + o16, bk + o16, idesc_s, kk > 0);
+                }
 #pragma unroll
-            for (int dp2 = 0; dp2 < D / 16; ++dp2) {
-                uint32_t kb2[4];
-                const int r = ks * 16 + (lane & 7) + (((lane >> 3) & 1) << 3), c = 2 * dp2 + (lane >> 4);
-                ldsm_x4_trans(kb2, tile_addr<D>(bK, r, c));
-                mma_16816(dqa[2 * dp2], sa[ks], kb2[0], kb2[1]);
-                mma_16816(dqa[2 * dp2 + 1], sa[ks], kb2[2], kb2[3]);
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint32_t o16 = ((kk >> 2) * Lay::kPanel + (kk & 3) * 32) >> 4;
+                    umma_ss(tmem + Lay::kColP, dOt + o16, bv + o16, idesc_s, kk > 0);
+                }
+                tc_commit(&s_full);
+                if (!(ok = wait(&p_full, j & 1))) break;
+                tc_fence_after();
+                // dQ += dS K: dS from tensor memory (key half h at columns
+                // 64 h .. 64 h + 31, 8 per 16 keys), K MN-major (+2048 B per 16 keys)
+                const uint64_t km = umma_smem_desc(aK, Lay::kPanel, 1024);
+#pragma unroll
+                for (int kk = 0; kk < kDqBN / 16; ++kk) {
+                    const uint32_t ca = (kk >> 2) * 64 + (kk & 3) * 8;
+                    umma_ts(tmem + Lay::kColDQ, tmem + Lay::kColS + ca, km + kk * (2048 >> 4),
+                            idesc_o, (j > 0 || kk > 0) ? 1u : 0u);
+                }
+                tc_commit(&kv_empty[st]);
             }
-        __syncthreads();
-    }
-    cp_async_wait<0>();
+            tc_commit(&acc_done);
+            mbar_wait(&acc_done, 0, &abort_flag, p.status, 1000000000ull);
+        }
+    } else if (warp >= 4) {
+        // ---------------------------------------- elementwise + epilogue ----
+        const int h = (warp - 4) >> 2;                  // key half of a tile
+        const int g4 = warp & 3;                        // lane group
+        const int r = (g4 << 5) + lane;                 // row = tensor-memory lane
+        const int pos = t0 + r / p.G, head = kvh * p.G + r % p.G;
+        const bool row_real = (r < p.P * p.G) && (pos < p.Tq);
+        const uint32_t lane_addr = tmem + ((static_cast<uint32_t>(g4) * 32u) << 16);
+        const size_t li = (static_cast<size_t>(b) * p.Hq + head) * p.Tq + (row_real ? pos : 0);
+        const float Lr = row_real ? p.lse[li] * 1.4426950408889634f : 0.0f;
+        const float Dr = row_real ? p.Dsum[li] : 0.0f;
+        bool ok = true;
+        for (int j = 0; j < n_kv; ++j) {
+            if (!(ok = __all_sync(0xffffffffu, mbar_wait(&s_full, j & 1, &abort_flag, p.status))))
+                break;
+            tc_fence_after();
+            const int key0 = tile_of(j) * kDqBN;
+            const bool full = block_visible(p.vis, t0, p.P, key0, kDqBN) &&
+                              __all_sync(0xffffffffu, row_real || r >= p.P * p.G);
 #pragma unroll
-    for (int h2 = 0; h2 < 2; ++h2) {
-        const int qi = q0 + qrow + gq + 8 * h2;
-        if (qi >= Tq) continue;
-        const size_t rowoff = ((static_cast<size_t>(b) * Tq + qi) * Hq + hq) * D;
+            for (int c = 0; c < 2; ++c) {
+                const uint32_t col = 64 * h + 32 * c;
+                uint32_t sv[32], dp[32];
+                tmem_ld32(lane_addr + Lay::kColS + col, sv);
+                tmem_ld32(lane_addr + Lay::kColP + col, dp);
+                tmem_wait_ld();
+                uint32_t pk[16];
 #pragma unroll
-        for (int n = 0; n < D / 8; ++n)
-            *reinterpret_cast<__nv_bfloat162 *>(dq + rowoff + n * 8 + 2 * tq) =
-                __floats2bfloat162_rn(dqa[n][2 * h2] * scale, dqa[n][2 * h2 + 1] * scale);
+                for (int e = 0; e < 32; e += 2) {
+                    float ds[2];
+#pragma unroll
+                    for (int t = 0; t < 2; ++t) {
+                        float pr = fast_exp2(fmaf(__uint_as_float(sv[e + t]), p.scale_log2, -Lr));
+                        const bool vis = row_real && (full || p.vis(pos, key0 + col + e + t));
+                        // rows past the tile's real ones hold stale operands: exact zeros
+                        ds[t] = vis ? pr * (__uint_as_float(dp[e + t]) - Dr) : 0.0f;
+                    }
+                    pk[e / 2] = pack_bf16x2(ds[0], ds[1]);
+                }
+                // over columns this thread has already read (its own half)
+                tmem_st16(lane_addr + Lay::kColS + 64 * h + 16 * c, pk);
+            }
+            tmem_wait_st();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&p_full);
+        }
+        // ---- epilogue: dQ * scale -> bf16 (half h writes columns h D/2 ..) ----
+        if (ok && n_kv > 0)
+            ok = __all_sync(0xffffffffu, mbar_wait(&acc_done, 0, &abort_flag, p.status));
+        tc_fence_after();
+        const bool have = ok && n_kv > 0;               // warp-uniform
+        __nv_bfloat16 *dst = p.dq + ((static_cast<size_t>(b) * p.Tq + (row_real ? pos : 0)) * p.Hq +
+                                     head) * D + (D / 2) * h;
+#pragma unroll
+        for (int c = 0; c < D / 64; ++c) {
+            uint32_t v[32];
+            if (have) {
+                tmem_ld32(lane_addr + Lay::kColDQ + (D / 2) * h + 32 * c, v);
+                tmem_wait_ld();
+            } else {
+#pragma unroll
+                for (int e = 0; e < 32; ++e) v[e] = 0u;
+            }
+            if (row_real) {
+                uint4 *d4 = reinterpret_cast<uint4 *>(dst + 32 * c);
+                const float f = p.scale;
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const uint32_t *w = &v[8 * e];
+                    d4[e] = make_uint4(
+                        pack_bf16x2(__uint_as_float(w[0]) * f, __uint_as_float(w[1]) * f),
+                        pack_bf16x2(__uint_as_float(w[2]) * f, __uint_as_float(w[3]) * f),
+                        pack_bf16x2(__uint_as_float(w[4]) * f, __uint_as_float(w[5]) * f),
+                        pack_bf16x2(__uint_as_float(w[6]) * f, __uint_as_float(w[7]) * f));
+                }
+            }
+        }
     }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        __syncwarp();
+        tc_fence_after();
+        tmem_dealloc(tmem, 512);
+    }
+}
+
+template <int D>
+static int launch_dq_tc(const void *q, const void *k, const void *v, const void *dout,
+                        const float *lse, const float *Dsum, void *dq, int B, int Tq, int Tkv,
+                        int Hq, int Hkv, Vis vis, float scale, cudaStream_t stream) {
+    DqParams prm;
+    prm.B = B;
+    prm.Tq = Tq;
+    prm.Tkv = Tkv;
+    prm.Hq = Hq;
+    prm.Hkv = Hkv;
+    prm.G = Hq / Hkv;
+    prm.P = 128 / prm.G;
+    prm.n_mt = (Tq + prm.P - 1) / prm.P;
+    prm.vis = vis;
+    prm.scale = scale;
+    prm.scale_log2 = scale * 1.4426950408889634f;
+    prm.lse = lse;
+    prm.Dsum = Dsum;
+    prm.dq = static_cast<__nv_bfloat16 *>(dq);
+    prm.status = device_status_ptr();
+    if (!prm.status) return GQA_ERR_CUDA;
+    const long long blocks = static_cast<long long>(prm.n_mt) * Hkv * B;
+    if (blocks > 0x7fffffffLL) return set_error(GQA_ERR_UNSUPPORTED, "backward grid too large");
+    CUtensorMap tq, to, tk, tv;
+    if (int rc = encode_tmap_bf16_4d(&tq, q, D, Hq, Tq, B, 64, prm.G, prm.P, 1, 1)) return rc;
+    if (int rc = encode_tmap_bf16_4d(&to, dout, D, Hq, Tq, B, 64, prm.G, prm.P, 1, 1)) return rc;
+    if (int rc = encode_tmap_bf16_4d(&tk, k, D, Hkv, Tkv, B, 64, 1, kDqBN, 1, 1)) return rc;
+    if (int rc = encode_tmap_bf16_4d(&tv, v, D, Hkv, Tkv, B, 64, 1, kDqBN, 1, 1)) return rc;
+    auto kern = dq_tc_kernel<D>;
+    const int smem = DqLayout<D>::kSmemBytes;
+    if (int rc = check_cuda(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                 smem), "cudaFuncSetAttribute(dq_tc)"))
+        return rc;
+    kern<<<static_cast<unsigned>(blocks), kTcThreads, smem, stream>>>(tq, to, tk, tv, prm);
+    return check_cuda(cudaGetLastError(), "dq_tc_kernel launch");
 }
 
 size_t bwd_workspace_bytes(int B, int Tq, int Hq) {
@@ -591,24 +713,13 @@ static int launch_bwd_d(const void *q, const void *k, const void *v, const void 
         static_cast<const bf *>(dout), static_cast<const bf *>(o), Dsum, B, Tq, Hq, D);
     if (int rc = check_cuda(cudaGetLastError(), "rowdot_kernel launch")) return rc;
     Vis vis{Tq, Tkv, causal, causal ? window : 0, sinks};
-    constexpr int P = D + 8;
-    const int smem_q = (2 * kQTile + 4 * kKBlk) * P * 2;
-    auto kq = dq_kernel<D>;
-    if (int rc = check_cuda(cudaFuncSetAttribute(kq, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                 smem_q), "cudaFuncSetAttribute(dq)"))
+    if (Tkv == 0)   // no key: every query gradient is zero
+        return check_cuda(cudaMemsetAsync(dq, 0, static_cast<size_t>(B) * Tq * Hq * D * 2, stream),
+                          "cudaMemsetAsync(dq)");
+    if (int rc = launch_dkdv_tc<D>(q, k, v, dout, lse, Dsum, dk, dv, B, Tq, Tkv, Hq, Hkv, vis, scale,
+                                   stream))
         return rc;
-    if (Tkv > 0) {
-        if (int rc = launch_dkdv_tc<D>(q, k, v, dout, lse, Dsum, dk, dv, B, Tq, Tkv, Hq, Hkv, vis,
-                                       scale, stream))
-            return rc;
-    }
-    const long long n2 = static_cast<long long>((Tq + kQTile - 1) / kQTile) * Hq * B;
-    if (n2 > 0x7fffffffLL) return set_error(GQA_ERR_UNSUPPORTED, "backward grid too large");
-    kq<<<static_cast<unsigned>(n2), kBwThreads, smem_q, stream>>>(
-        static_cast<const bf *>(q), static_cast<const bf *>(k), static_cast<const bf *>(v),
-        static_cast<const bf *>(dout), lse, Dsum, static_cast<bf *>(dq), B, Tq, Tkv, Hq, Hkv, vis,
-        scale);
-    return check_cuda(cudaGetLastError(), "dq_kernel launch");
+    return launch_dq_tc<D>(q, k, v, dout, lse, Dsum, dq, B, Tq, Tkv, Hq, Hkv, vis, scale, stream);
 }
 
 int launch_bwd(const void *q, const void *k, const void *v, const void *o, const void *dout,

@@ -65,3 +65,14 @@ def test_backward_shared_head_sum(gqa_lib):
     sv = dve.float().view(B, T, Hkv, G, d).sum(3)
     assert float((dk.float() - sk).abs().max()) <= 2e-2 * max(1.0, float(sk.abs().max()))
     assert float((dv.float() - sv).abs().max()) <= 2e-2 * max(1.0, float(sv.abs().max()))
+
+
+def test_backward_without_keys_is_zero(gqa_lib):
+    B, Tq, Hq, Hkv, d = 1, 64, 4, 2, 128
+    q = workloads.randn((B, Tq, Hq, d), 1).cuda()
+    k = torch.empty((B, 0, Hkv, d), dtype=torch.bfloat16, device="cuda")
+    o = torch.zeros_like(q)
+    lse = torch.full((B, Hq, Tq), float("-inf"), device="cuda")
+    dq, dk, dv = gqa.attn_bwd(q, k, k, o, lse, workloads.randn((B, Tq, Hq, d), 2).cuda())
+    torch.cuda.synchronize()
+    assert dq.shape == q.shape and bool((dq == 0).all())
