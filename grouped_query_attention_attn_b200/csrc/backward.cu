@@ -401,11 +401,15 @@ static int launch_dkdv_tc(const void *q, const void *k, const void *v, const voi
 // P = floor(128 / G) positions, as in the forward (one 3-D TMA box; every K / V
 // tile serves the whole group).  For every visible 128-key tile:
 //   tensor pipe   S = Q K^T and dP = dO V^T into tensor memory;
-//   8 warps       dS = P (dP - D_row), P = exp2(S * scale * log2e - lse_row *
-//                 log2e), bf16, over the first columns of each half's S
-//                 (two threads per row, one per 64-key half);
+//   8 warps       load S and dP (two threads per row, one per 64-key half),
+//                 release them, and form dS = P (dP - D_row) with
+//                 P = exp2(S * scale * log2e - lse_row * log2e), bf16, into a
+//                 dS region of tensor memory;
 //   tensor pipe   dQ += dS K with dS read from tensor memory.
-// Tensor memory: S | dP | dQ.  Shared memory: Q, dO, 2-deep K and V rings.
+// Once the warps hold S(j) and dP(j) in registers the next tile's S and dP are
+// computed, overlapping the elementwise work; the warps write dS(j) after
+// dQ(j-1) has read dS(j-1).  Tensor memory: S | dP | dQ | dS.  Shared memory:
+// Q, dO, 2-deep K and V rings.
 constexpr int kDqBN = 128;       // keys per tile
 
 template <int D>
@@ -418,7 +422,8 @@ struct DqLayout {
     static constexpr int kOffV = kOffK + 2 * kTile;        // [2]
     static constexpr int kBytes = kOffV + 2 * kTile;
     static constexpr int kSmemBytes = kBytes + 1024;
-    static constexpr uint32_t kColS = 0, kColP = 128, kColDQ = 256;
+    // S | dP | dQ | dS (bf16, half h of the keys at 384 + 32 h)
+    static constexpr uint32_t kColS = 0, kColP = 128, kColDQ = 256, kColDS = 384;
 };
 
 struct DqParams {
@@ -440,7 +445,8 @@ dq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-    __shared__ uint64_t qo_full, kv_full[2], kv_empty[2], s_full, p_full, acc_done;
+    __shared__ uint64_t qo_full, kv_full[2], kv_empty[2], s_full, s_free, p_full, dq_done,
+        acc_done;
     __shared__ uint32_t tmem_base_sh;
     __shared__ int abort_flag;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -469,7 +475,9 @@ dq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
             mbar_init(&kv_empty[s], 1);
         }
         mbar_init(&s_full, 1);
+        mbar_init(&s_free, 8);
         mbar_init(&p_full, 8);
+        mbar_init(&dq_done, 1);
         mbar_init(&acc_done, 1);
         abort_flag = 0;
         fence_mbar_init();
@@ -535,15 +543,13 @@ dq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
             auto wait = [&](uint64_t *bar, uint32_t parity) {
                 return mbar_wait(bar, parity, &abort_flag, p.status);
             };
-            bool ok = wait(&qo_full, 0);
-            for (int j = 0; ok && j < n_kv; ++j) {
+            // S = Q K_j^T, dP = dO V_j^T: K-major A and B (+32 B per 16 of d)
+            auto issue_s = [&](int j) {
                 const int st = j & 1;
-                if (!(ok = wait(&kv_full[st], (j >> 1) & 1))) break;
+                if (!wait(&kv_full[st], (j >> 1) & 1)) return false;
                 tc_fence_after();
-                const uint32_t aK = base + Lay::kOffK + st * Lay::kTile;
-                const uint32_t aV = base + Lay::kOffV + st * Lay::kTile;
-                // S = Q K^T, dP = dO V^T: K-major A and B (+32 B per 16 of d)
-                const uint64_t bk = umma_smem_desc(aK, 16, 1024), bv = umma_smem_desc(aV, 16, 1024);
+                const uint64_t bk = umma_smem_desc(base + Lay::kOffK + st * Lay::kTile, 16, 1024);
+                const uint64_t bv = umma_smem_desc(base + Lay::kOffV + st * Lay::kTile, 16, 1024);
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
                     const uint32_t o16 = ((kk >> 2) * Lay::kPanel + (kk & 3) * 32) >> 4;
@@ -555,17 +561,25 @@ dq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
                     umma_ss(tmem + Lay::kColP, dOt + o16, bv + o16, idesc_s, kk > 0);
                 }
                 tc_commit(&s_full);
+                return true;
+            };
+            bool ok = wait(&qo_full, 0) && issue_s(0);
+            for (int j = 0; ok && j < n_kv; ++j) {
+                const int st = j & 1;
+                // the warps hold S(j), dP(j) in registers: the next tile's may be written
+                if (!(ok = wait(&s_free, j & 1))) break;
+                if (j + 1 < n_kv && !(ok = issue_s(j + 1))) break;
                 if (!(ok = wait(&p_full, j & 1))) break;
                 tc_fence_after();
-                // dQ += dS K: dS from tensor memory (key half h at columns
-                // 64 h .. 64 h + 31, 8 per 16 keys), K MN-major (+2048 B per 16 keys)
-                const uint64_t km = umma_smem_desc(aK, Lay::kPanel, 1024);
+                // dQ += dS K: dS from tensor memory (key half h at 384 + 32 h,
+                // 8 columns per 16 keys), K MN-major (+2048 B per 16 keys)
+                const uint64_t km =
+                    umma_smem_desc(base + Lay::kOffK + st * Lay::kTile, Lay::kPanel, 1024);
 #pragma unroll
-                for (int kk = 0; kk < kDqBN / 16; ++kk) {
-                    const uint32_t ca = (kk >> 2) * 64 + (kk & 3) * 8;
-                    umma_ts(tmem + Lay::kColDQ, tmem + Lay::kColS + ca, km + kk * (2048 >> 4),
+                for (int kk = 0; kk < kDqBN / 16; ++kk)
+                    umma_ts(tmem + Lay::kColDQ, tmem + Lay::kColDS + kk * 8, km + kk * (2048 >> 4),
                             idesc_o, (j > 0 || kk > 0) ? 1u : 0u);
-                }
+                tc_commit(&dq_done);
                 tc_commit(&kv_empty[st]);
             }
             tc_commit(&acc_done);
@@ -587,32 +601,42 @@ dq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
             if (!(ok = __all_sync(0xffffffffu, mbar_wait(&s_full, j & 1, &abort_flag, p.status))))
                 break;
             tc_fence_after();
-            const int key0 = tile_of(j) * kDqBN;
-            const bool full = block_visible(p.vis, t0, p.P, key0, kDqBN) &&
-                              __all_sync(0xffffffffu, row_real || r >= p.P * p.G);
+            uint32_t sv[2][32], dp[2][32];
 #pragma unroll
             for (int c = 0; c < 2; ++c) {
-                const uint32_t col = 64 * h + 32 * c;
-                uint32_t sv[32], dp[32];
-                tmem_ld32(lane_addr + Lay::kColS + col, sv);
-                tmem_ld32(lane_addr + Lay::kColP + col, dp);
-                tmem_wait_ld();
-                uint32_t pk[16];
+                tmem_ld32(lane_addr + Lay::kColS + 64 * h + 32 * c, sv[c]);
+                tmem_ld32(lane_addr + Lay::kColP + 64 * h + 32 * c, dp[c]);
+            }
+            tmem_wait_ld();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&s_free);        // S and dP may be overwritten
+            const int key0 = tile_of(j) * kDqBN + 64 * h;
+            const bool full = block_visible(p.vis, t0, p.P, tile_of(j) * kDqBN, kDqBN) &&
+                              __all_sync(0xffffffffu, row_real || r >= p.P * p.G);
+            uint32_t pk[2][16];
+#pragma unroll
+            for (int c = 0; c < 2; ++c)
 #pragma unroll
                 for (int e = 0; e < 32; e += 2) {
                     float ds[2];
 #pragma unroll
                     for (int t = 0; t < 2; ++t) {
-                        float pr = fast_exp2(fmaf(__uint_as_float(sv[e + t]), p.scale_log2, -Lr));
-                        const bool vis = row_real && (full || p.vis(pos, key0 + col + e + t));
+                        const float pr =
+                            fast_exp2(fmaf(__uint_as_float(sv[c][e + t]), p.scale_log2, -Lr));
+                        const bool vis = row_real && (full || p.vis(pos, key0 + 32 * c + e + t));
                         // rows past the tile's real ones hold stale operands: exact zeros
-                        ds[t] = vis ? pr * (__uint_as_float(dp[e + t]) - Dr) : 0.0f;
+                        ds[t] = vis ? pr * (__uint_as_float(dp[c][e + t]) - Dr) : 0.0f;
                     }
-                    pk[e / 2] = pack_bf16x2(ds[0], ds[1]);
+                    pk[c][e / 2] = pack_bf16x2(ds[0], ds[1]);
                 }
-                // over columns this thread has already read (its own half)
-                tmem_st16(lane_addr + Lay::kColS + 64 * h + 16 * c, pk);
-            }
+            // dQ(j-1) has read the dS region
+            if (j > 0 && !(ok = __all_sync(0xffffffffu, mbar_wait(&dq_done, (j - 1) & 1,
+                                                                   &abort_flag, p.status))))
+                break;
+            tc_fence_after();
+            tmem_st16(lane_addr + Lay::kColDS + 32 * h, pk[0]);
+            tmem_st16(lane_addr + Lay::kColDS + 32 * h + 16, pk[1]);
             tmem_wait_st();
             tc_fence_before();
             __syncwarp();
