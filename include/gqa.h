@@ -63,6 +63,10 @@ typedef enum {
  *   d in {64, 128} (else UNSUPPORTED); causal 0/1; scale > 0 and finite
  *   (callers normally pass 1/sqrt(d)).  Pointers must be 16-byte aligned
  *   (tensor-memory-access copies need it).
+ * The kernel is persistent: min(#work units, #SMs) CTAs, a unit being two
+ * 128-row tiles of one (batch, KV head).  If the environment variable
+ * GQA_PREFILL_MAX_CTAS holds a positive integer, it caps that grid (read at
+ * every launch; the tests use it to put many units on each CTA).
  */
 int gqa_attn_fwd(const void *q, const void *k, const void *v, void *o,
                  int B, int Tq, int Tkv, int Hq, int Hkv, int d,
