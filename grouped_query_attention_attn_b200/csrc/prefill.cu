@@ -466,8 +466,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                 }
                 tc_fence_after();
                 uint32_t sr[2][32];
-                tmem_ld32(lane_addr + colS, sr[0]);
-                tmem_ld32(lane_addr + colS + 32, sr[1]);
+                tmem_ld64(lane_addr + colS, sr[0], sr[1]);     // one instruction, 64 columns
                 tmem_wait_ld();
                 const int key0 = u.tile(j) * kPfBN + 64 * h;   // key of my first column
                 const bool masked = __any_sync(
