@@ -602,11 +602,8 @@ dq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
                 break;
             tc_fence_after();
             uint32_t sv[2][32], dp[2][32];
-#pragma unroll
-            for (int c = 0; c < 2; ++c) {
-                tmem_ld32(lane_addr + Lay::kColS + 64 * h + 32 * c, sv[c]);
-                tmem_ld32(lane_addr + Lay::kColP + 64 * h + 32 * c, dp[c]);
-            }
+            tmem_ld64(lane_addr + Lay::kColS + 64 * h, sv[0], sv[1]);
+            tmem_ld64(lane_addr + Lay::kColP + 64 * h, dp[0], dp[1]);
             tmem_wait_ld();
             tc_fence_before();
             __syncwarp();
