@@ -71,17 +71,18 @@ rowdot_kernel(const __nv_bfloat16 *__restrict__ dout, const __nv_bfloat16 *__res
 // query head of the group (an "item"):
 //   tensor pipe   S^T = K Q^T and dP^T = V dO^T into tensor memory (M = 128
 //                 keys, N = 128 queries);
-//   8 warps       P^T = exp2(S^T * scale * log2e - lse_q * log2e) and
+//   16 warps      P^T = exp2(S^T * scale * log2e - lse_q * log2e) and
 //                 dS^T = P^T (dP^T - D_q), bf16, written back over the first
-//                 columns of each half's S^T / dP^T (two threads per key row,
-//                 one per 64-query half);
+//                 columns of each quarter's S^T / dP^T (four threads per key
+//                 row, one per 32-query quarter);
 //   tensor pipe   dV += P^T dO and dK += dS^T Q with P^T / dS^T read from
 //                 tensor memory (dV and dK accumulate over all items).
 // Tensor memory (512 columns): S^T | dP^T | dV | dK.  Shared memory: K, V,
 // and a 2-deep ring of (Q, dO, lse, D) per item.
 constexpr int kTcBK = 128;       // keys per CTA
 constexpr int kTcBQ = 128;       // query rows per item
-constexpr int kTcThreads = 384;  // producer, MMA, 2 idle, 8 elementwise warps
+constexpr int kTcThreads = 640;  // producer, MMA, 2 idle, 16 elementwise warps
+constexpr int kTcElemWarps = 16;   // 4 per tensor-memory lane group, 32 columns each
 
 template <int D>
 struct TcLayout {
@@ -143,7 +144,7 @@ dkdv_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             mbar_init(&qo_empty[s], 1);
         }
         mbar_init(&s_full, 1);
-        mbar_init(&p_full, 8);
+        mbar_init(&p_full, kTcElemWarps);
         mbar_init(&acc_done, 1);
         abort_flag = 0;
         fence_mbar_init();
@@ -241,20 +242,20 @@ dkdv_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                 tc_commit(&s_full);
                 if (!(ok = wait(&p_full, it & 1))) break;
                 tc_fence_after();
-                // dV += P^T dO, dK += dS^T Q: A from tensor memory (half h of the
-                // queries at columns 64 h .. 64 h + 31, 8 per 16 queries), B
+                // dV += P^T dO, dK += dS^T Q: A from tensor memory (quarter u of
+                // the queries at columns 32 u .. 32 u + 15, 8 per 16 queries), B
                 // MN-major (+2048 B per 16 queries)
                 const uint64_t vo = umma_smem_desc(aO, Lay::kPanel, 1024);
                 const uint64_t vq = umma_smem_desc(aQ, Lay::kPanel, 1024);
 #pragma unroll
                 for (int kk = 0; kk < kTcBQ / 16; ++kk) {
-                    const uint32_t ca = (kk >> 2) * 64 + (kk & 3) * 8;
+                    const uint32_t ca = (kk >> 1) * 32 + (kk & 1) * 8;
                     umma_ts(tmem + Lay::kColDV, tmem + Lay::kColS + ca, vo + kk * (2048 >> 4),
                             idesc_o, (it > 0 || kk > 0) ? 1u : 0u);
                 }
 #pragma unroll
                 for (int kk = 0; kk < kTcBQ / 16; ++kk) {
-                    const uint32_t ca = (kk >> 2) * 64 + (kk & 3) * 8;
+                    const uint32_t ca = (kk >> 1) * 32 + (kk & 1) * 8;
                     umma_ts(tmem + Lay::kColDK, tmem + Lay::kColP + ca, vq + kk * (2048 >> 4),
                             idesc_o, (it > 0 || kk > 0) ? 1u : 0u);
                 }
@@ -265,7 +266,7 @@ dkdv_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         }
     } else if (warp >= 4) {
         // ---------------------------------------- elementwise + epilogue ----
-        const int h = (warp - 4) >> 2;                  // query half of an item
+        const int u = (warp - 4) >> 2;                  // query quarter of an item
         const int g4 = warp & 3;                        // lane group
         const int r = (g4 << 5) + lane;                 // key row = tensor-memory lane
         const int key = k0 + r;
@@ -279,39 +280,42 @@ dkdv_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                                   mbar_wait(&s_full, it & 1, &abort_flag, p.status))))
                 break;
             tc_fence_after();
+            const uint32_t col = 32 * u;
+            uint32_t sv[32], dp[32];
+            tmem_ld32(lane_addr + Lay::kColS + col, sv);
+            tmem_ld32(lane_addr + Lay::kColP + col, dp);
             const bool full = block_visible(p.vis, q0, kTcBQ, k0, kTcBK);
-            const float *L = sLD + st * 2 * kTcBQ + 64 * h, *Dd = L + kTcBQ;
+            // the quarter's lse / D: the same 32 values for every lane (broadcast)
+            const float4 *L4 = reinterpret_cast<const float4 *>(sLD + st * 2 * kTcBQ + col);
+            const float4 *D4 = reinterpret_cast<const float4 *>(sLD + st * 2 * kTcBQ + kTcBQ + col);
+            tmem_wait_ld();
+            uint32_t pk[16], dk[16];
 #pragma unroll
-            for (int c = 0; c < 2; ++c) {
-                const uint32_t col = 64 * h + 32 * c;
-                uint32_t sv[32], dp[32];
-                tmem_ld32(lane_addr + Lay::kColS + col, sv);
-                tmem_ld32(lane_addr + Lay::kColP + col, dp);
-                tmem_wait_ld();
-                uint32_t pk[16], dk[16];
+            for (int e4 = 0; e4 < 8; ++e4) {
+                const float4 l4 = L4[e4], d4 = D4[e4];
+                const float lv[4] = {l4.x, l4.y, l4.z, l4.w}, dv[4] = {d4.x, d4.y, d4.z, d4.w};
+                float pr[4], ds[4];
 #pragma unroll
-                for (int e = 0; e < 32; e += 2) {
-                    float pr[2], ds[2];
-#pragma unroll
-                    for (int t = 0; t < 2; ++t) {
-                        const int ql = 32 * c + e + t;
-                        pr[t] = fast_exp2(fmaf(__uint_as_float(sv[e + t]), p.scale_log2, -L[ql]));
-                        if (!full && !p.vis(q0 + 64 * h + ql, key)) pr[t] = 0.0f;
-                        ds[t] = pr[t] * (__uint_as_float(dp[e + t]) - Dd[ql]);
-                    }
-                    pk[e / 2] = pack_bf16x2(pr[0], pr[1]);
-                    dk[e / 2] = pack_bf16x2(ds[0], ds[1]);
+                for (int t = 0; t < 4; ++t) {
+                    const int e = 4 * e4 + t;
+                    pr[t] = fast_exp2(fmaf(__uint_as_float(sv[e]), p.scale_log2, -lv[t]));
+                    if (!full && !p.vis(q0 + col + e, key)) pr[t] = 0.0f;
+                    ds[t] = pr[t] * (__uint_as_float(dp[e]) - dv[t]);
                 }
-                // over columns this thread has already read (its own half)
-                tmem_st16(lane_addr + Lay::kColS + 64 * h + 16 * c, pk);
-                tmem_st16(lane_addr + Lay::kColP + 64 * h + 16 * c, dk);
+                pk[2 * e4] = pack_bf16x2(pr[0], pr[1]);
+                pk[2 * e4 + 1] = pack_bf16x2(pr[2], pr[3]);
+                dk[2 * e4] = pack_bf16x2(ds[0], ds[1]);
+                dk[2 * e4 + 1] = pack_bf16x2(ds[2], ds[3]);
             }
+            // over columns this thread has already read (its own quarter)
+            tmem_st16(lane_addr + Lay::kColS + col, pk);
+            tmem_st16(lane_addr + Lay::kColP + col, dk);
             tmem_wait_st();
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&p_full);
         }
-        // ---- epilogue: dV, dK * scale -> bf16 (half h writes columns h D/2 ..) ----
+        // ---- epilogue: dV, dK * scale -> bf16 (quarter u writes columns 32 u ..) ----
         if (ok && n_items > 0)
             ok = __all_sync(0xffffffffu, mbar_wait(&acc_done, 0, &abort_flag, p.status));
         tc_fence_after();
@@ -322,20 +326,19 @@ dkdv_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                                kvh) * D;
 #pragma unroll
         for (int m = 0; m < 2; ++m) {                   // dV, then dK
-            __nv_bfloat16 *dst = (m ? p.dk : p.dv) + rowoff + (D / 2) * h;
+            __nv_bfloat16 *dst = (m ? p.dk : p.dv) + rowoff + 32 * u;
             const float f = m ? p.scale : 1.0f;
-#pragma unroll
-            for (int c = 0; c < D / 64; ++c) {
+            if (32 * u < D) {                           // warp-uniform
                 uint32_t v[32];
                 if (have) {
-                    tmem_ld32(lane_addr + (m ? Lay::kColDK : Lay::kColDV) + (D / 2) * h + 32 * c, v);
+                    tmem_ld32(lane_addr + (m ? Lay::kColDK : Lay::kColDV) + 32 * u, v);
                     tmem_wait_ld();
                 } else {
 #pragma unroll
                     for (int e = 0; e < 32; ++e) v[e] = 0u;
                 }
                 if (key < p.Tkv) {
-                    uint4 *d4 = reinterpret_cast<uint4 *>(dst + 32 * c);
+                    uint4 *d4 = reinterpret_cast<uint4 *>(dst);
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
                         const uint32_t *w = &v[8 * e];
@@ -401,8 +404,8 @@ static int launch_dkdv_tc(const void *q, const void *k, const void *v, const voi
 // P = floor(128 / G) positions, as in the forward (one 3-D TMA box; every K / V
 // tile serves the whole group).  For every visible 128-key tile:
 //   tensor pipe   S = Q K^T and dP = dO V^T into tensor memory;
-//   8 warps       load S and dP (two threads per row, one per 64-key half),
-//                 release them, and form dS = P (dP - D_row) with
+//   16 warps      load S and dP (four threads per row, one per 32-key
+//                 quarter), release them, and form dS = P (dP - D_row) with
 //                 P = exp2(S * scale * log2e - lse_row * log2e), bf16, into a
 //                 dS region of tensor memory;
 //   tensor pipe   dQ += dS K with dS read from tensor memory.
@@ -422,7 +425,7 @@ struct DqLayout {
     static constexpr int kOffV = kOffK + 2 * kTile;        // [2]
     static constexpr int kBytes = kOffV + 2 * kTile;
     static constexpr int kSmemBytes = kBytes + 1024;
-    // S | dP | dQ | dS (bf16, half h of the keys at 384 + 32 h)
+    // S | dP | dQ | dS (bf16, keys 32 u .. 32 u + 31 at 384 + 16 u)
     static constexpr uint32_t kColS = 0, kColP = 128, kColDQ = 256, kColDS = 384;
 };
 
@@ -475,8 +478,8 @@ dq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
             mbar_init(&kv_empty[s], 1);
         }
         mbar_init(&s_full, 1);
-        mbar_init(&s_free, 8);
-        mbar_init(&p_full, 8);
+        mbar_init(&s_free, kTcElemWarps);
+        mbar_init(&p_full, kTcElemWarps);
         mbar_init(&dq_done, 1);
         mbar_init(&acc_done, 1);
         abort_flag = 0;
@@ -571,7 +574,7 @@ dq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
                 if (j + 1 < n_kv && !(ok = issue_s(j + 1))) break;
                 if (!(ok = wait(&p_full, j & 1))) break;
                 tc_fence_after();
-                // dQ += dS K: dS from tensor memory (key half h at 384 + 32 h,
+                // dQ += dS K: dS from tensor memory (keys 32 u .. at 384 + 16 u,
                 // 8 columns per 16 keys), K MN-major (+2048 B per 16 keys)
                 const uint64_t km =
                     umma_smem_desc(base + Lay::kOffK + st * Lay::kTile, Lay::kPanel, 1024);
@@ -587,7 +590,7 @@ dq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
         }
     } else if (warp >= 4) {
         // ---------------------------------------- elementwise + epilogue ----
-        const int h = (warp - 4) >> 2;                  // key half of a tile
+        const int u = (warp - 4) >> 2;                  // key quarter of a tile
         const int g4 = warp & 3;                        // lane group
         const int r = (g4 << 5) + lane;                 // row = tensor-memory lane
         const int pos = t0 + r / p.G, head = kvh * p.G + r % p.G;
@@ -596,68 +599,64 @@ dq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
         const size_t li = (static_cast<size_t>(b) * p.Hq + head) * p.Tq + (row_real ? pos : 0);
         const float Lr = row_real ? p.lse[li] * 1.4426950408889634f : 0.0f;
         const float Dr = row_real ? p.Dsum[li] : 0.0f;
+        const uint32_t col = 32 * u;
         bool ok = true;
         for (int j = 0; j < n_kv; ++j) {
             if (!(ok = __all_sync(0xffffffffu, mbar_wait(&s_full, j & 1, &abort_flag, p.status))))
                 break;
             tc_fence_after();
-            uint32_t sv[2][32], dp[2][32];
-            tmem_ld64(lane_addr + Lay::kColS + 64 * h, sv[0], sv[1]);
-            tmem_ld64(lane_addr + Lay::kColP + 64 * h, dp[0], dp[1]);
+            uint32_t sv[32], dp[32];
+            tmem_ld32(lane_addr + Lay::kColS + col, sv);
+            tmem_ld32(lane_addr + Lay::kColP + col, dp);
             tmem_wait_ld();
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&s_free);        // S and dP may be overwritten
-            const int key0 = tile_of(j) * kDqBN + 64 * h;
+            const int key0 = tile_of(j) * kDqBN + col;
             const bool full = block_visible(p.vis, t0, p.P, tile_of(j) * kDqBN, kDqBN) &&
                               __all_sync(0xffffffffu, row_real || r >= p.P * p.G);
-            uint32_t pk[2][16];
+            uint32_t pk[16];
 #pragma unroll
-            for (int c = 0; c < 2; ++c)
+            for (int e = 0; e < 32; e += 2) {
+                float ds[2];
 #pragma unroll
-                for (int e = 0; e < 32; e += 2) {
-                    float ds[2];
-#pragma unroll
-                    for (int t = 0; t < 2; ++t) {
-                        const float pr =
-                            fast_exp2(fmaf(__uint_as_float(sv[c][e + t]), p.scale_log2, -Lr));
-                        const bool vis = row_real && (full || p.vis(pos, key0 + 32 * c + e + t));
-                        // rows past the tile's real ones hold stale operands: exact zeros
-                        ds[t] = vis ? pr * (__uint_as_float(dp[c][e + t]) - Dr) : 0.0f;
-                    }
-                    pk[c][e / 2] = pack_bf16x2(ds[0], ds[1]);
+                for (int t = 0; t < 2; ++t) {
+                    const float pr = fast_exp2(fmaf(__uint_as_float(sv[e + t]), p.scale_log2, -Lr));
+                    const bool vis = row_real && (full || p.vis(pos, key0 + e + t));
+                    // rows past the tile's real ones hold stale operands: exact zeros
+                    ds[t] = vis ? pr * (__uint_as_float(dp[e + t]) - Dr) : 0.0f;
                 }
+                pk[e / 2] = pack_bf16x2(ds[0], ds[1]);
+            }
             // dQ(j-1) has read the dS region
             if (j > 0 && !(ok = __all_sync(0xffffffffu, mbar_wait(&dq_done, (j - 1) & 1,
                                                                    &abort_flag, p.status))))
                 break;
             tc_fence_after();
-            tmem_st16(lane_addr + Lay::kColDS + 32 * h, pk[0]);
-            tmem_st16(lane_addr + Lay::kColDS + 32 * h + 16, pk[1]);
+            tmem_st16(lane_addr + Lay::kColDS + 16 * u, pk);   // keys 32 u .. 32 u + 31
             tmem_wait_st();
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&p_full);
         }
-        // ---- epilogue: dQ * scale -> bf16 (half h writes columns h D/2 ..) ----
+        // ---- epilogue: dQ * scale -> bf16 (quarter u writes columns 32 u ..) ----
         if (ok && n_kv > 0)
             ok = __all_sync(0xffffffffu, mbar_wait(&acc_done, 0, &abort_flag, p.status));
         tc_fence_after();
         const bool have = ok && n_kv > 0;               // warp-uniform
         __nv_bfloat16 *dst = p.dq + ((static_cast<size_t>(b) * p.Tq + (row_real ? pos : 0)) * p.Hq +
-                                     head) * D + (D / 2) * h;
-#pragma unroll
-        for (int c = 0; c < D / 64; ++c) {
+                                     head) * D + col;
+        if (col < D) {                                  // warp-uniform
             uint32_t v[32];
             if (have) {
-                tmem_ld32(lane_addr + Lay::kColDQ + (D / 2) * h + 32 * c, v);
+                tmem_ld32(lane_addr + Lay::kColDQ + col, v);
                 tmem_wait_ld();
             } else {
 #pragma unroll
                 for (int e = 0; e < 32; ++e) v[e] = 0u;
             }
             if (row_real) {
-                uint4 *d4 = reinterpret_cast<uint4 *>(dst + 32 * c);
+                uint4 *d4 = reinterpret_cast<uint4 *>(dst);
                 const float f = p.scale;
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
