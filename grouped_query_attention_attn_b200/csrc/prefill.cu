@@ -655,6 +655,16 @@ static int launch_prefill_d(const void *q, const void *k, const void *v, void *o
         return rc;
 
     auto kern = prefill_kernel<D>;
+    // the setmaxnreg split adds up only at the launch budget it was sized for:
+    // a build with fewer registers per thread would leave the softmax
+    // warpgroups waiting for registers, so it is refused here
+    cudaFuncAttributes fa;
+    if (int rc = check_cuda(cudaFuncGetAttributes(&fa, kern), "cudaFuncGetAttributes(prefill)"))
+        return rc;
+    if (fa.numRegs != kPfRegsLaunch)
+        return set_error(GQA_ERR_UNSUPPORTED,
+                         "prefill kernel built with %d registers per thread, %d expected",
+                         fa.numRegs, kPfRegsLaunch);
     const int smem = PfLayout<D>::kSmemBytes;
     if (int rc = check_cuda(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                                  smem), "cudaFuncSetAttribute(prefill)"))
