@@ -77,12 +77,19 @@ rowdot_kernel(const __nv_bfloat16 *__restrict__ dout, const __nv_bfloat16 *__res
 //                 row, one per 32-query quarter);
 //   tensor pipe   dV += P^T dO and dK += dS^T Q with P^T / dS^T read from
 //                 tensor memory (dV and dK accumulate over all items).
+// S^T and dP^T are committed separately and P^T and dS^T are published
+// separately, so the tensor pipe computes dV(i) while the warps form dS^T(i)
+// and the next item's dP^T while they form its P^T.
 // Tensor memory (512 columns): S^T | dP^T | dV | dK.  Shared memory: K, V,
 // and a 2-deep ring of (Q, dO, lse, D) per item.
 constexpr int kTcBK = 128;       // keys per CTA
 constexpr int kTcBQ = 128;       // query rows per item
 constexpr int kTcThreads = 640;  // producer, MMA, 2 idle, 16 elementwise warps
 constexpr int kTcElemWarps = 16;   // 4 per tensor-memory lane group, 32 columns each
+#ifndef GQA_BWD_POLY_PER4
+#define GQA_BWD_POLY_PER4 1
+#endif
+constexpr int kTcPolyPer4 = GQA_BWD_POLY_PER4;  // pairs per 4 of P^T on the exp2 polynomial
 
 template <int D>
 struct TcLayout {
@@ -117,7 +124,8 @@ dkdv_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-    __shared__ uint64_t kv_full, qo_full[2], qo_empty[2], s_full, p_full, acc_done;
+    __shared__ uint64_t kv_full, qo_full[2], qo_empty[2], s_full, dp_full, p_full, ds_full,
+        acc_done;
     __shared__ uint32_t tmem_base_sh;
     __shared__ int abort_flag;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -144,7 +152,9 @@ dkdv_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             mbar_init(&qo_empty[s], 1);
         }
         mbar_init(&s_full, 1);
+        mbar_init(&dp_full, 1);
         mbar_init(&p_full, kTcElemWarps);
+        mbar_init(&ds_full, kTcElemWarps);
         mbar_init(&acc_done, 1);
         abort_flag = 0;
         fence_mbar_init();
@@ -220,46 +230,54 @@ dkdv_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             auto wait = [&](uint64_t *bar, uint32_t parity) {
                 return mbar_wait(bar, parity, &abort_flag, p.status);
             };
-            bool ok = wait(&kv_full, 0);
-            for (int it = 0; ok && it < n_items; ++it) {
-                const int st = it & 1;
-                if (!(ok = wait(&qo_full[st], (it >> 1) & 1))) break;
+            // S^T = K Q^T and dP^T = V dO^T of item it: K-major A and B (+32 B
+            // per 16 of d), each with its own commit
+            auto issue_s = [&](int it, uint32_t col, uint64_t a, uint32_t off_b, uint64_t *bar) {
+                const uint64_t bd = umma_smem_desc(base + off_b + (it & 1) * Lay::kTile, 16, 1024);
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint32_t off = ((kk >> 2) * Lay::kPanel + (kk & 3) * 32) >> 4;
+                    umma_ss(tmem + col, a + off, bd + off, idesc_s, kk > 0);
+                }
+                tc_commit(bar);
+            };
+            // dV += P^T dO, dK += dS^T Q: A from tensor memory (quarter u of the
+            // queries at columns 32 u .. 32 u + 15, 8 per 16 queries), B MN-major
+            // (+2048 B per 16 queries)
+            auto issue_acc = [&](int it, uint32_t col_acc, uint32_t col_a, uint32_t off_b) {
+                const uint64_t vb = umma_smem_desc(base + off_b + (it & 1) * Lay::kTile, Lay::kPanel,
+                                                   1024);
+#pragma unroll
+                for (int kk = 0; kk < kTcBQ / 16; ++kk) {
+                    const uint32_t ca = (kk >> 1) * 32 + (kk & 1) * 8;
+                    umma_ts(tmem + col_acc, tmem + col_a + ca, vb + kk * (2048 >> 4), idesc_o,
+                            (it > 0 || kk > 0) ? 1u : 0u);
+                }
+            };
+            // Issue order S(0) dP(0) | dV(0) | dK(0) S(1) dP(1) | dV(1) | ...: dV
+            // runs while the warps form dS^T, the next P^T is formed while dP
+            // runs, and a product always sits between the one that reads a
+            // tensor-memory region and the next one that overwrites it.
+            bool ok = wait(&kv_full, 0) && wait(&qo_full[0], 0);
+            if (ok) {
                 tc_fence_after();
-                const uint32_t aQ = base + Lay::kOffQ + st * Lay::kTile;
-                const uint32_t aO = base + Lay::kOffO + st * Lay::kTile;
-                // S^T = K Q^T, dP^T = V dO^T: K-major A and B (+32 B per 16 of d)
-                const uint64_t bq = umma_smem_desc(aQ, 16, 1024), bo = umma_smem_desc(aO, 16, 1024);
-#pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint32_t off = ((kk >> 2) * Lay::kPanel + (kk & 3) * 32) >> 4;
-                    umma_ss(tmem + Lay::kColS, dK + off, bq + off, idesc_s, kk > 0);
-                }
-#pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint32_t off = ((kk >> 2) * Lay::kPanel + (kk & 3) * 32) >> 4;
-                    umma_ss(tmem + Lay::kColP, dV + off, bo + off, idesc_s, kk > 0);
-                }
-                tc_commit(&s_full);
+                issue_s(0, Lay::kColS, dK, Lay::kOffQ, &s_full);
+                issue_s(0, Lay::kColP, dV, Lay::kOffO, &dp_full);
+            }
+            for (int it = 0; ok && it < n_items; ++it) {
                 if (!(ok = wait(&p_full, it & 1))) break;
                 tc_fence_after();
-                // dV += P^T dO, dK += dS^T Q: A from tensor memory (quarter u of
-                // the queries at columns 32 u .. 32 u + 15, 8 per 16 queries), B
-                // MN-major (+2048 B per 16 queries)
-                const uint64_t vo = umma_smem_desc(aO, Lay::kPanel, 1024);
-                const uint64_t vq = umma_smem_desc(aQ, Lay::kPanel, 1024);
-#pragma unroll
-                for (int kk = 0; kk < kTcBQ / 16; ++kk) {
-                    const uint32_t ca = (kk >> 1) * 32 + (kk & 1) * 8;
-                    umma_ts(tmem + Lay::kColDV, tmem + Lay::kColS + ca, vo + kk * (2048 >> 4),
-                            idesc_o, (it > 0 || kk > 0) ? 1u : 0u);
+                issue_acc(it, Lay::kColDV, Lay::kColS, Lay::kOffO);
+                if (!(ok = wait(&ds_full, it & 1))) break;
+                tc_fence_after();
+                issue_acc(it, Lay::kColDK, Lay::kColP, Lay::kOffQ);
+                tc_commit(&qo_empty[it & 1]);
+                if (it + 1 < n_items) {
+                    if (!(ok = wait(&qo_full[(it + 1) & 1], ((it + 1) >> 1) & 1))) break;
+                    tc_fence_after();
+                    issue_s(it + 1, Lay::kColS, dK, Lay::kOffQ, &s_full);
+                    issue_s(it + 1, Lay::kColP, dV, Lay::kOffO, &dp_full);
                 }
-#pragma unroll
-                for (int kk = 0; kk < kTcBQ / 16; ++kk) {
-                    const uint32_t ca = (kk >> 1) * 32 + (kk & 1) * 8;
-                    umma_ts(tmem + Lay::kColDK, tmem + Lay::kColP + ca, vq + kk * (2048 >> 4),
-                            idesc_o, (it > 0 || kk > 0) ? 1u : 0u);
-                }
-                tc_commit(&qo_empty[st]);
             }
             tc_commit(&acc_done);
             mbar_wait(&acc_done, 0, &abort_flag, p.status, 1000000000ull);
@@ -281,39 +299,64 @@ dkdv_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                 break;
             tc_fence_after();
             const uint32_t col = 32 * u;
-            uint32_t sv[32], dp[32];
+            uint32_t sv[32];
             tmem_ld32(lane_addr + Lay::kColS + col, sv);
-            tmem_ld32(lane_addr + Lay::kColP + col, dp);
             const bool full = block_visible(p.vis, q0, kTcBQ, k0, kTcBK);
             // the quarter's lse / D: the same 32 values for every lane (broadcast)
             const float4 *L4 = reinterpret_cast<const float4 *>(sLD + st * 2 * kTcBQ + col);
             const float4 *D4 = reinterpret_cast<const float4 *>(sLD + st * 2 * kTcBQ + kTcBQ + col);
             tmem_wait_ld();
-            uint32_t pk[16], dk[16];
+            // P^T, over columns this thread has already read (its own quarter)
+            float pr[32];
+            uint32_t pk[16];
+            const float2 cc = make_float2(p.scale_log2, p.scale_log2);
 #pragma unroll
-            for (int e4 = 0; e4 < 8; ++e4) {
-                const float4 l4 = L4[e4], d4 = D4[e4];
-                const float lv[4] = {l4.x, l4.y, l4.z, l4.w}, dv[4] = {d4.x, d4.y, d4.z, d4.w};
-                float pr[4], ds[4];
-#pragma unroll
-                for (int t = 0; t < 4; ++t) {
-                    const int e = 4 * e4 + t;
-                    pr[t] = fast_exp2(fmaf(__uint_as_float(sv[e]), p.scale_log2, -lv[t]));
-                    if (!full && !p.vis(q0 + col + e, key)) pr[t] = 0.0f;
-                    ds[t] = pr[t] * (__uint_as_float(dp[e]) - dv[t]);
+            for (int e2 = 0; e2 < 16; ++e2) {
+                const float2 l2 = reinterpret_cast<const float2 *>(L4)[e2];
+                const float2 x = fma2(make_float2(__uint_as_float(sv[2 * e2]),
+                                                  __uint_as_float(sv[2 * e2 + 1])),
+                                      cc, make_float2(-l2.x, -l2.y));
+                // part of the pairs on the FMA-pipe polynomial, off the MUFU unit
+                const float2 pe = (e2 & 3) < kTcPolyPer4
+                                      ? exp2_poly2(x)
+                                      : make_float2(fast_exp2(x.x), fast_exp2(x.y));
+                pr[2 * e2] = pe.x;
+                pr[2 * e2 + 1] = pe.y;
+                if (!full) {
+                    if (!p.vis(q0 + col + 2 * e2, key)) pr[2 * e2] = 0.0f;
+                    if (!p.vis(q0 + col + 2 * e2 + 1, key)) pr[2 * e2 + 1] = 0.0f;
                 }
-                pk[2 * e4] = pack_bf16x2(pr[0], pr[1]);
-                pk[2 * e4 + 1] = pack_bf16x2(pr[2], pr[3]);
-                dk[2 * e4] = pack_bf16x2(ds[0], ds[1]);
-                dk[2 * e4 + 1] = pack_bf16x2(ds[2], ds[3]);
+                pk[e2] = pack_bf16x2(pr[2 * e2], pr[2 * e2 + 1]);
             }
-            // over columns this thread has already read (its own quarter)
             tmem_st16(lane_addr + Lay::kColS + col, pk);
-            tmem_st16(lane_addr + Lay::kColP + col, dk);
             tmem_wait_st();
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&p_full);
+            // dS^T = P^T (dP^T - D), over the same columns of the dP^T region
+            if (!(ok = __all_sync(0xffffffffu, mbar_wait(&dp_full, it & 1, &abort_flag, p.status))))
+                break;
+            tc_fence_after();
+            uint32_t dp[32];
+            tmem_ld32(lane_addr + Lay::kColP + col, dp);
+            tmem_wait_ld();
+            uint32_t dk[16];
+#pragma unroll
+            for (int e4 = 0; e4 < 8; ++e4) {
+                const float4 d4 = D4[e4];
+                const float dv[4] = {d4.x, d4.y, d4.z, d4.w};
+                float ds[4];
+#pragma unroll
+                for (int t = 0; t < 4; ++t)
+                    ds[t] = pr[4 * e4 + t] * (__uint_as_float(dp[4 * e4 + t]) - dv[t]);
+                dk[2 * e4] = pack_bf16x2(ds[0], ds[1]);
+                dk[2 * e4 + 1] = pack_bf16x2(ds[2], ds[3]);
+            }
+            tmem_st16(lane_addr + Lay::kColP + col, dk);
+            tmem_wait_st();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&ds_full);
         }
         // ---- epilogue: dV, dK * scale -> bf16 (quarter u writes columns 32 u ..) ----
         if (ok && n_items > 0)
@@ -616,15 +659,19 @@ dq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
             const bool full = block_visible(p.vis, t0, p.P, tile_of(j) * kDqBN, kDqBN) &&
                               __all_sync(0xffffffffu, row_real || r >= p.P * p.G);
             uint32_t pk[16];
+            const float2 cc = make_float2(p.scale_log2, p.scale_log2), nl = make_float2(-Lr, -Lr);
 #pragma unroll
             for (int e = 0; e < 32; e += 2) {
-                float ds[2];
+                const float2 x = fma2(make_float2(__uint_as_float(sv[e]), __uint_as_float(sv[e + 1])),
+                                      cc, nl);
+                const float2 pr = make_float2(fast_exp2(x.x), fast_exp2(x.y));
+                float ds[2] = {pr.x * (__uint_as_float(dp[e]) - Dr),
+                               pr.y * (__uint_as_float(dp[e + 1]) - Dr)};
 #pragma unroll
                 for (int t = 0; t < 2; ++t) {
-                    const float pr = fast_exp2(fmaf(__uint_as_float(sv[e + t]), p.scale_log2, -Lr));
                     const bool vis = row_real && (full || p.vis(pos, key0 + e + t));
                     // rows past the tile's real ones hold stale operands: exact zeros
-                    ds[t] = vis ? pr * (__uint_as_float(dp[e + t]) - Dr) : 0.0f;
+                    if (!vis) ds[t] = 0.0f;
                 }
                 pk[e / 2] = pack_bf16x2(ds[0], ds[1]);
             }
