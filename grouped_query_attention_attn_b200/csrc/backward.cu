@@ -86,10 +86,6 @@ constexpr int kTcBK = 128;       // keys per CTA
 constexpr int kTcBQ = 128;       // query rows per item
 constexpr int kTcThreads = 640;  // producer, MMA, 2 idle, 16 elementwise warps
 constexpr int kTcElemWarps = 16;   // 4 per tensor-memory lane group, 32 columns each
-#ifndef GQA_BWD_POLY_PER4
-#define GQA_BWD_POLY_PER4 1
-#endif
-constexpr int kTcPolyPer4 = GQA_BWD_POLY_PER4;  // pairs per 4 of P^T on the exp2 polynomial
 
 template <int D>
 struct TcLayout {
@@ -316,10 +312,7 @@ dkdv_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                 const float2 x = fma2(make_float2(__uint_as_float(sv[2 * e2]),
                                                   __uint_as_float(sv[2 * e2 + 1])),
                                       cc, make_float2(-l2.x, -l2.y));
-                // part of the pairs on the FMA-pipe polynomial, off the MUFU unit
-                const float2 pe = (e2 & 3) < kTcPolyPer4
-                                      ? exp2_poly2(x)
-                                      : make_float2(fast_exp2(x.x), fast_exp2(x.y));
+                const float2 pe = make_float2(fast_exp2(x.x), fast_exp2(x.y));
                 pr[2 * e2] = pe.x;
                 pr[2 * e2 + 1] = pe.y;
                 if (!full) {
