@@ -4,7 +4,8 @@
 // fold: out[b, t, grp, :] = (sum over the contiguous group members, in head
 // order, in fp32) / (H / g), rounded to bf16 -- the position-wise mean over
 // heads[start:start+size] of TT Lab "キー・バリューヘッドだけ減らしてみる",
-// step 2.  HBM-bound: each thread moves 16-byte vectors.
+// step 2.  HBM-bound: each thread moves 16-byte vectors and has all loads of
+// a group in flight before it adds them.
 #include <cuda_bf16.h>
 
 #include "device.cuh"
@@ -12,37 +13,40 @@
 
 namespace gqa {
 
-__global__ void __launch_bounds__(256)
-fold_kv_kernel(const uint4 *__restrict__ in, uint4 *__restrict__ out, size_t n_vec, int H,
-               int g, int d8) {
+constexpr int kFoldBatch = 4;   // group members loaded before any is added
+
+// Index type I: 32-bit when every vector index fits, so the per-vector
+// divisions stay cheap.
+template <typename I>
+__global__ void __launch_bounds__(256, 5)
+fold_kv_kernel(const uint4 *__restrict__ in, uint4 *__restrict__ out, I n_vec, int H, int g,
+               int d8) {
     const int size = H / g;
     const float divisor = static_cast<float>(size);
-    const size_t stride = static_cast<size_t>(gridDim.x) * blockDim.x;
-    for (size_t t = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; t < n_vec;
-         t += stride) {
-        const size_t c8 = t % d8;
-        const size_t grp = (t / d8) % g;
-        const size_t bt = t / (static_cast<size_t>(d8) * g);
-        const uint4 *src = in + (bt * H + grp * size) * d8 + c8;
+    const I stride = static_cast<I>(gridDim.x) * blockDim.x;
+    for (I t = static_cast<I>(blockIdx.x) * blockDim.x + threadIdx.x; t < n_vec; t += stride) {
+        const I c8 = t % d8, rest = t / d8;
+        const I grp = rest % g, bt = rest / g;
+        const uint4 *src = in + (static_cast<size_t>(bt) * H + static_cast<size_t>(grp) * size) *
+                                    d8 + c8;
         float acc[8];
-        {
-            const uint4 x = src[0];
-            const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&x);
+        for (int m0 = 0; m0 < size; m0 += kFoldBatch) {
+            // all loads of the batch in flight, then the adds in head order
+            uint4 x[kFoldBatch];
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const float2 f = __bfloat1622float2(h[e]);
-                acc[2 * e] = f.x;
-                acc[2 * e + 1] = f.y;
-            }
-        }
-        for (int m = 1; m < size; ++m) {
-            const uint4 x = src[static_cast<size_t>(m) * d8];
-            const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&x);
+            for (int j = 0; j < kFoldBatch; ++j)
+                if (m0 + j < size) x[j] = src[static_cast<size_t>(m0 + j) * d8];
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const float2 f = __bfloat1622float2(h[e]);
-                acc[2 * e] = __fadd_rn(acc[2 * e], f.x);
-                acc[2 * e + 1] = __fadd_rn(acc[2 * e + 1], f.y);
+            for (int j = 0; j < kFoldBatch; ++j) {
+                if (m0 + j < size) {
+                    const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&x[j]);
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const float2 f = __bfloat1622float2(h[e]);
+                        acc[2 * e] = m0 + j == 0 ? f.x : __fadd_rn(acc[2 * e], f.x);
+                        acc[2 * e + 1] = m0 + j == 0 ? f.y : __fadd_rn(acc[2 * e + 1], f.y);
+                    }
+                }
             }
         }
         uint4 r;
@@ -61,10 +65,17 @@ int launch_fold_kv(const void *in, void *out, int B, int T, int H, int g, int d,
                    cudaStream_t stream) {
     const int d8 = d / 8;
     const size_t n_vec = static_cast<size_t>(B) * T * g * d8;
-    int blocks = static_cast<int>((n_vec + 255) / 256);
-    if (blocks > 148 * 16) blocks = 148 * 16;
-    fold_kv_kernel<<<blocks, 256, 0, stream>>>(static_cast<const uint4 *>(in),
-                                               static_cast<uint4 *>(out), n_vec, H, g, d8);
+    // one output vector per thread (the loop in the kernel covers larger inputs)
+    size_t blocks = (n_vec + 255) / 256;
+    if (blocks > 0x7fffffffull) blocks = 0x7fffffffull;
+    const uint4 *src = static_cast<const uint4 *>(in);
+    uint4 *dst = static_cast<uint4 *>(out);
+    if (n_vec + static_cast<size_t>(blocks) * 256 <= 0xffffffffull)
+        fold_kv_kernel<uint32_t><<<static_cast<unsigned>(blocks), 256, 0, stream>>>(
+            src, dst, static_cast<uint32_t>(n_vec), H, g, d8);
+    else
+        fold_kv_kernel<size_t><<<static_cast<unsigned>(blocks), 256, 0, stream>>>(src, dst, n_vec,
+                                                                                H, g, d8);
     return check_cuda(cudaGetLastError(), "fold_kv_kernel launch");
 }
 

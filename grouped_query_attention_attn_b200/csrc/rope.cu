@@ -5,13 +5,14 @@
 // and k rotate.  HBM-bound (one read and one write of each element), so the
 // arithmetic is arranged to stay far below the memory time:
 //   * thread (c8, slot) of a block owns 16-byte column c8 (pairs 4 c8 .. 4 c8 + 3)
-//     of one token, computes those four sine / cosine pairs once and applies them
-//     to that column of every head of q and of k: one sincos per head row of
-//     eight pairs, no integer division in the loop;
+//     of up to kRopeBatch head rows of one token (a batch: q's heads, then k's,
+//     in groups of kRopeBatch), computes those four sine / cosine pairs and
+//     applies them to that column of every row of the batch;
 //   * the angle m * theta_i reaches ~10^4 rad at long context, so the number of
 //     turns m * theta_i / (2 pi) is formed and reduced to [-1/2, 1/2] in double,
 //     then sincospif gives the fp32 sine and cosine of 2 pi times that fraction;
-//   * loads are issued in batches of kBatch head rows before any store.
+//   * all loads of a batch are issued before any store, and the batches of a
+//     token are spread over threads so that enough loads are in flight.
 #include <cuda_bf16.h>
 
 #include "device.cuh"
@@ -28,33 +29,34 @@ __device__ __forceinline__ uint32_t rotate_pair(uint32_t w, float cs, float sn) 
     return pack_bf16x2(a.x * cs - a.y * sn, a.x * sn + a.y * cs);
 }
 
-// Rotates column c8 of H head rows starting at row (head-row units of d8 vectors).
-__device__ __forceinline__ void rope_rows(uint4 *__restrict__ row0, int H, int d8,
+// Rotates column c8 of n (<= kRopeBatch) head rows starting at row0 (rows d8
+// vectors apart).
+__device__ __forceinline__ void rope_rows(uint4 *__restrict__ row0, int n, int d8,
                                           const float (&cs)[4], const float (&sn)[4]) {
-    for (int h0 = 0; h0 < H; h0 += kRopeBatch) {
-        uint4 w[kRopeBatch];
+    uint4 w[kRopeBatch];
 #pragma unroll
-        for (int j = 0; j < kRopeBatch; ++j)
-            if (h0 + j < H) w[j] = row0[static_cast<size_t>(h0 + j) * d8];
+    for (int j = 0; j < kRopeBatch; ++j)
+        if (j < n) w[j] = row0[static_cast<size_t>(j) * d8];
 #pragma unroll
-        for (int j = 0; j < kRopeBatch; ++j) {
-            if (h0 + j < H) {
-                w[j].x = rotate_pair(w[j].x, cs[0], sn[0]);
-                w[j].y = rotate_pair(w[j].y, cs[1], sn[1]);
-                w[j].z = rotate_pair(w[j].z, cs[2], sn[2]);
-                w[j].w = rotate_pair(w[j].w, cs[3], sn[3]);
-                row0[static_cast<size_t>(h0 + j) * d8] = w[j];
-            }
+    for (int j = 0; j < kRopeBatch; ++j) {
+        if (j < n) {
+            w[j].x = rotate_pair(w[j].x, cs[0], sn[0]);
+            w[j].y = rotate_pair(w[j].y, cs[1], sn[1]);
+            w[j].z = rotate_pair(w[j].z, cs[2], sn[2]);
+            w[j].w = rotate_pair(w[j].w, cs[3], sn[3]);
+            row0[static_cast<size_t>(j) * d8] = w[j];
         }
     }
 }
 
 // x0 [n_tok, H0, d], x1 [n_tok, H1, d] (x1 may be absent, H1 = 0); token tok =
 // b * T + t sits at position pos0 + t, or at max(seqlens[b] - 1, 0) when seqlens
-// is given (decode queries, T = 1).  blockDim = (d8, slots): one token per slot.
+// is given (decode queries, T = 1).  blockDim = (d8, slots): one batch of
+// kRopeBatch head rows of one token per slot; a token has n_batch =
+// ceil(H0 / kRopeBatch) + ceil(H1 / kRopeBatch) batches.
 __global__ void __launch_bounds__(kRopeThreads)
-rope_kernel(uint4 *__restrict__ x0, int H0, uint4 *__restrict__ x1, int H1, int n_tok, int T,
-            int pos0, const int32_t *__restrict__ seqlens, double log_theta) {
+rope_kernel(uint4 *__restrict__ x0, int H0, uint4 *__restrict__ x1, int H1, long long n_work,
+            int n_batch, int T, int pos0, const int32_t *__restrict__ seqlens, double log_theta) {
     __shared__ double turns[kRopeMaxHalf];         // theta_i / (2 pi)
     const int d8 = blockDim.x, half = 4 * d8;
     const int tid = threadIdx.y * d8 + threadIdx.x;
@@ -62,8 +64,9 @@ rope_kernel(uint4 *__restrict__ x0, int H0, uint4 *__restrict__ x1, int H1, int 
         turns[i] = exp(-static_cast<double>(i) / half * log_theta) *
                    0.15915494309189533576888376337251;
     __syncthreads();
-    const int tok = blockIdx.x * blockDim.y + threadIdx.y;
-    if (tok >= n_tok) return;
+    const long long w = static_cast<long long>(blockIdx.x) * blockDim.y + threadIdx.y;
+    if (w >= n_work) return;
+    const int tok = static_cast<int>(w / n_batch), bi = static_cast<int>(w % n_batch);
     const int c8 = threadIdx.x;
     const int b = tok / T;
     const int m = seqlens ? max(seqlens[b] - 1, 0) : pos0 + (tok - b * T);
@@ -74,19 +77,29 @@ rope_kernel(uint4 *__restrict__ x0, int H0, uint4 *__restrict__ x1, int H1, int 
         const float fr = static_cast<float>(t - rint(t));    // in [-1/2, 1/2]
         sincospif(2.0f * fr, &sn[e], &cs[e]);
     }
-    rope_rows(x0 + static_cast<size_t>(tok) * H0 * d8 + c8, H0, d8, cs, sn);
-    if (x1) rope_rows(x1 + static_cast<size_t>(tok) * H1 * d8 + c8, H1, d8, cs, sn);
+    const int b0 = (H0 + kRopeBatch - 1) / kRopeBatch;
+    if (bi < b0) {
+        const int h = bi * kRopeBatch;
+        rope_rows(x0 + (static_cast<size_t>(tok) * H0 + h) * d8 + c8, min(kRopeBatch, H0 - h), d8,
+                  cs, sn);
+    } else {
+        const int h = (bi - b0) * kRopeBatch;
+        rope_rows(x1 + (static_cast<size_t>(tok) * H1 + h) * d8 + c8, min(kRopeBatch, H1 - h), d8,
+                  cs, sn);
+    }
 }
 
 static int launch_rope(void *x0, int H0, void *x1, int H1, int B, int T, int d, int pos0,
                        const int32_t *seqlens, float theta, cudaStream_t stream) {
     const int d8 = d / 8;
     const int slots = kRopeThreads / d8;
-    const long long n_tok = static_cast<long long>(B) * T;
-    const long long blocks = (n_tok + slots - 1) / slots;
+    const int n_batch = (H0 + kRopeBatch - 1) / kRopeBatch + (H1 + kRopeBatch - 1) / kRopeBatch;
+    const long long n_work = static_cast<long long>(B) * T * n_batch;
+    const long long blocks = (n_work + slots - 1) / slots;
+    if (blocks > 0x7fffffffLL) return set_error(GQA_ERR_UNSUPPORTED, "rope grid too large");
     rope_kernel<<<static_cast<unsigned>(blocks), dim3(d8, slots), 0, stream>>>(
-        static_cast<uint4 *>(x0), H0, static_cast<uint4 *>(x1), H1, static_cast<int>(n_tok), T,
-        pos0, seqlens, log(static_cast<double>(theta)));
+        static_cast<uint4 *>(x0), H0, static_cast<uint4 *>(x1), H1, n_work, n_batch, T, pos0,
+        seqlens, log(static_cast<double>(theta)));
     return check_cuda(cudaGetLastError(), "rope_kernel launch");
 }
 

@@ -32,7 +32,7 @@ def test_rope_matches_oracle(gqa_lib, B, T, H, d, pos0, theta):
 
 
 @pytest.mark.parametrize("B,T,Hq,Hkv,d,pos0", [(2, 77, 8, 2, 128, 0), (1, 300, 32, 8, 128, 9000),
-                                              (3, 5, 3, 1, 24, 11)])
+                                              (3, 5, 3, 1, 24, 11), (1, 9, 20, 4, 64, 3)])
 def test_rope_qk_matches_oracle(gqa_lib, B, T, Hq, Hkv, d, pos0):
     q = workloads.randn((B, T, Hq, d), 40 + T)
     k = workloads.randn((B, T, Hkv, d), 41 + T)
