@@ -87,30 +87,20 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tm_k,
         if (threadIdx.x == 0 && split == 0 && kvh == 0) record_status(status, GQA_ERR_INVALID_ARG);
         L = L < 0 ? 0 : Lmax;
     }
-    const int start = split * chunk;
+    // Sliding window: key j is visible iff j >= lo or j < sinks (and j < L).
+    // The splits cover [lo, L) from lo on, chunk keys each, so none of them
+    // holds only invisible keys; split 0 first takes the sink keys below the
+    // window, [0, s_end), as whole stages.  Without a window lo = s_end = 0.
+    const int lo = window > 0 ? max(0, L - window) : 0;
+    const int s_end = window > 0 ? min(sinks, lo) : 0;
+    const int start = lo + split * chunk;
     if (start >= L) return;                         // whole block: nothing in this split
     const int end = min(start + chunk, L);
-    const int n_stages = (end - start + kDecBK - 1) / kDecBK;
+    const int t_s = split == 0 ? (s_end + kDecBK - 1) / kDecBK : 0;   // sink stages
+    const int n_iter = t_s + (end - start + kDecBK - 1) / kDecBK;
+    const int off_w = start - t_s * kDecBK;         // window stage t starts at key off_w + 64 t
     const int G = Hq / Hkv;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    // Sliding window: key j is visible iff j >= lo or j < sinks (and j < L).
-    const int lo = window > 0 ? L - window : 0;
-    const int n_sinks = window > 0 ? sinks : 0;
-    if (end <= lo && start >= n_sinks) {
-        // no visible key in this split: an empty partial (weight 0 in the merge)
-        const size_t row0 = (static_cast<size_t>(split) * B + b) * Hq + static_cast<size_t>(kvh) * G;
-        for (int idx = threadIdx.x; idx < G * D; idx += blockDim.x) {
-            part_o[row0 * D + idx] = 0.0f;
-            if (idx % D == 0) part_lse[row0 + idx / D] = -INFINITY;
-        }
-        return;
-    }
-    // Stages holding no visible key are not loaded: the sink stages [0, t_s)
-    // and the window stages [t_w, n_stages) of the split, in that order.
-    int t_s = min(n_stages, max(0, (n_sinks - start + kDecBK - 1) / kDecBK));
-    int t_w = min(n_stages, max(0, (lo - start) / kDecBK));
-    if (t_s >= t_w) t_s = t_w = 0;                  // the two runs meet: every stage
-    const int n_iter = t_s + n_stages - t_w;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kDecStages; ++s) {
@@ -133,7 +123,7 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tm_k,
                 uint8_t *kt = smem + st * Lay::kStageBytes;
                 uint8_t *vt = kt + Lay::kTileBytes;
                 mbar_expect_tx(&full_bar[st], Lay::kStageBytes);
-                const int j0 = start + (t < t_s ? t : t_w + t - t_s) * kDecBK;
+                const int j0 = t * kDecBK + (t < t_s ? 0 : off_w);
 #pragma unroll
                 for (int p = 0; p < Lay::kPanels; ++p) {
                     tma_load_4d(kt + p * Lay::kPanelBytes, &tm_k, &full_bar[st], p * 64, kvh, j0, b);
@@ -179,9 +169,11 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tm_k,
         if (!__all_sync(0xffffffffu, mbar_wait(&full_bar[st], ph, &abort_flag, status))) break;
         uint8_t *kt = smem + st * Lay::kStageBytes;
         uint8_t *vt = kt + Lay::kTileBytes;
-        const int stage = t < t_s ? t : t_w + t - t_s;
-        const int key0 = start + stage * kDecBK + warp * 16;  // first key of this warp's slice
-        const int n_valid = end - key0;                   // keys of the slice inside the split
+        // first key of this warp's slice, and how many keys of it are visible:
+        // a sink stage's run ends at s_end, a window stage's at the split end
+        const bool sink = t < t_s;
+        const int key0 = t * kDecBK + (sink ? 0 : off_w) + warp * 16;
+        const int n_valid = (sink ? s_end : end) - key0;
         const bool partial = n_valid > 0 && n_valid < 16;
         if (partial) {
             // Rows past the split end may be another split's keys or the
@@ -223,8 +215,7 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tm_k,
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
                         const int kl = nb * 8 + 2 * tq + (e & 1);
-                        const int key = key0 + kl;
-                        const bool vis = kl < n_valid && (key >= lo || key < n_sinks);
+                        const bool vis = kl < n_valid;
                         s[nb][e] = vis ? sacc[mb][nb][e] * scale_log2 : -INFINITY;
                         mx[e >> 1] = fmaxf(mx[e >> 1], s[nb][e]);
                     }
@@ -332,7 +323,7 @@ template <int D>
 __global__ void __launch_bounds__(128)
 decode_combine_kernel(const float *__restrict__ part_o, const float *__restrict__ part_lse,
                       const int32_t *__restrict__ seqlens, __nv_bfloat16 *__restrict__ o, int B,
-                      int Hq, int Lmax, int chunk) {
+                      int Hq, int Lmax, int chunk, int window) {
     constexpr int kPer = D / 32;
     // launched as a programmatic dependent of the split kernel: wait until all of
     // its memory operations are complete and visible
@@ -342,7 +333,8 @@ decode_combine_kernel(const float *__restrict__ part_o, const float *__restrict_
     const int b = row / Hq;
     int L = seqlens[b];
     L = L < 0 ? 0 : (L > Lmax ? Lmax : L);
-    const int n = (L + chunk - 1) / chunk;
+    const int lo = window > 0 ? max(0, L - window) : 0;   // the splits start at lo
+    const int n = (L - lo + chunk - 1) / chunk;
     const size_t plane = static_cast<size_t>(B) * Hq;
     float acc[kPer];
 #pragma unroll
@@ -389,7 +381,8 @@ static int launch_split(const CUtensorMap &tk, const CUtensorMap &tv, const void
     if (int rc = check_cuda(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                                  smem), "cudaFuncSetAttribute(decode)"))
         return rc;
-    dim3 grid((Lmax + chunk - 1) / chunk, Hkv, B);
+    const int span = window > 0 ? min(Lmax, window) : Lmax;   // keys after the window start
+    dim3 grid((span + chunk - 1) / chunk, Hkv, B);
     kern<<<grid, kDecThreads, smem, stream>>>(tk, tv, static_cast<const __nv_bfloat16 *>(q),
                                               seqlens, part_o, part_lse, B, Hq, Hkv, Lmax, chunk,
                                               window, sinks, scale_log2, status);
@@ -442,9 +435,11 @@ int launch_decode(const void *q, const void *k_cache, const void *v_cache,
     __nv_bfloat16 *ob = static_cast<__nv_bfloat16 *>(o);
     const cudaError_t e =
         d == 128 ? cudaLaunchKernelEx(&cfg, decode_combine_kernel<128>, (const float *)part_o,
-                                      (const float *)part_lse, seqlens, ob, B, Hq, Lmax, chunk)
+                                      (const float *)part_lse, seqlens, ob, B, Hq, Lmax, chunk,
+                                      window)
                  : cudaLaunchKernelEx(&cfg, decode_combine_kernel<64>, (const float *)part_o,
-                                      (const float *)part_lse, seqlens, ob, B, Hq, Lmax, chunk);
+                                      (const float *)part_lse, seqlens, ob, B, Hq, Lmax, chunk,
+                                      window);
     if (int rc = check_cuda(e, "decode_combine_kernel launch")) return rc;
     return check_cuda(cudaGetLastError(), "decode_combine_kernel launch");
 }
