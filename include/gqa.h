@@ -170,7 +170,9 @@ int gqa_decode(const void *q, const void *k_cache, const void *v_cache,
  * (course step 3): the newest token of sequence b sees cache rows
  * j >= seqlens[b] - window and rows j < sinks.  window >= 1, sinks >= 0;
  * everything else (layouts, workspace and its size, errors) as gqa_decode.
- * KV splits that hold no visible row read nothing.
+ * The KV splits start at the window's first row, and split 0 also reads the
+ * sink rows below the window; reads are whole 64-row stages, so apart from
+ * that rounding no invisible row is read.
  */
 int gqa_decode_window(const void *q, const void *k_cache, const void *v_cache,
                       const int32_t *seqlens, void *o,
