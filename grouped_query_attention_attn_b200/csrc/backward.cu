@@ -46,23 +46,52 @@ __device__ __forceinline__ bool block_visible(const Vis &v, int i0, int ni, int 
 }
 
 // ------------------------------------------------------------- rowdot ---
+// D = rowsum(dO o O) per (b, t, h), stored [B, H, T].  A group of D / 8 lanes
+// owns kRowdotRows consecutive rows and reads them as 16-byte vectors (all
+// loads in flight before the products), then reduces each row over the group.
+constexpr int kRowdotRows = 4;
+
+template <int D>
 __global__ void __launch_bounds__(256)
 rowdot_kernel(const __nv_bfloat16 *__restrict__ dout, const __nv_bfloat16 *__restrict__ o,
-              float *__restrict__ Dsum, int B, int T, int H, int d) {
-    const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
+              float *__restrict__ Dsum, int B, int T, int H) {
+    constexpr int kLanes = D / 8;                   // lanes per row: 8 or 16
     const long long rows = static_cast<long long>(B) * T * H;
-    if (warp >= rows) return;
-    const int h = warp % H, t = (warp / H) % T, b = warp / (H * T);
-    const __nv_bfloat16 *a = dout + static_cast<size_t>(warp) * d;
-    const __nv_bfloat16 *c = o + static_cast<size_t>(warp) * d;
-    float acc = 0.0f;
-    for (int e = lane * 2; e < d; e += 64) {
-        const float2 x = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(a + e));
-        const float2 y = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(c + e));
-        acc = fmaf(x.x, y.x, fmaf(x.y, y.y, acc));
+    const long long gt = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+    const int c8 = threadIdx.x % kLanes;
+    const long long row0 = gt / kLanes * kRowdotRows;
+    uint4 x[kRowdotRows], y[kRowdotRows];
+#pragma unroll
+    for (int u = 0; u < kRowdotRows; ++u) {
+        const long long r = row0 + u;
+        if (r < rows) {
+            x[u] = reinterpret_cast<const uint4 *>(dout + r * D)[c8];
+            y[u] = reinterpret_cast<const uint4 *>(o + r * D)[c8];
+        }
     }
-    for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-    if (lane == 0) Dsum[(static_cast<size_t>(b) * H + h) * T + t] = acc;
+#pragma unroll
+    for (int u = 0; u < kRowdotRows; ++u) {
+        const long long r = row0 + u;
+        float acc = 0.0f;
+        if (r < rows) {
+            const uint32_t *xa = reinterpret_cast<const uint32_t *>(&x[u]);
+            const uint32_t *ya = reinterpret_cast<const uint32_t *>(&y[u]);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const float2 xf = bf16x2_to_float2(xa[e]), yf = bf16x2_to_float2(ya[e]);
+                acc = fmaf(xf.x, yf.x, fmaf(xf.y, yf.y, acc));
+            }
+        }
+        // every lane of the warp takes part in the shuffles (rows past the end add 0)
+#pragma unroll
+        for (int off = kLanes / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+        if (c8 == 0 && r < rows) {
+            const long long bt = r / H;
+            const int h = static_cast<int>(r - bt * H);
+            const long long b = bt / T, t = bt - b * T;
+            Dsum[(b * H + h) * T + t] = acc;
+        }
+    }
 }
 
 // ------------------------------------------------------ dk dv (tcgen05) ---
@@ -769,8 +798,12 @@ static int launch_bwd_d(const void *q, const void *k, const void *v, const void 
     using bf = __nv_bfloat16;
     float *Dsum = static_cast<float *>(workspace);
     const long long rows = static_cast<long long>(B) * Tq * Hq;
-    rowdot_kernel<<<static_cast<unsigned>((rows * 32 + 255) / 256), 256, 0, stream>>>(
-        static_cast<const bf *>(dout), static_cast<const bf *>(o), Dsum, B, Tq, Hq, D);
+    const long long threads = (rows + kRowdotRows - 1) / kRowdotRows * (D / 8);
+    if ((threads + 255) / 256 > 0x7fffffffLL)
+        return set_error(GQA_ERR_UNSUPPORTED, "backward: too many rows");
+    if (rows > 0)
+        rowdot_kernel<D><<<static_cast<unsigned>((threads + 255) / 256), 256, 0, stream>>>(
+            static_cast<const bf *>(dout), static_cast<const bf *>(o), Dsum, B, Tq, Hq);
     if (int rc = check_cuda(cudaGetLastError(), "rowdot_kernel launch")) return rc;
     Vis vis{Tq, Tkv, causal, causal ? window : 0, sinks};
     if (Tkv == 0)   // no key: every query gradient is zero
