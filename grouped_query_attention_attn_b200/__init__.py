@@ -1,8 +1,10 @@
 """Grouped-query scaled-dot-product attention for NVIDIA B200 (sm_100a).
 
 The computation lives in the C-ABI library ``libgqa.so`` (declared in
-``include/gqa.h``): a tcgen05/TMEM/TMA prefill kernel, a split-KV decode
-kernel with a log-sum-exp combine, an fp32 path and a head-folding kernel.
+``include/gqa.h``): a tcgen05/TMEM/TMA prefill kernel (causal, full, sliding
+window with sinks, and a host-buffer entry point that pipelines the copies),
+a split-KV decode kernel with a log-sum-exp combine, the tcgen05 backward
+(dQ, dK, dV), in-place RoPE, an fp32 path and a head-folding kernel.
 This package is its Python binding; PyTorch is used for device memory and
 streams only.  The library is loaded on first use and there is no CPU
 fallback: a missing or unloadable library raises.
