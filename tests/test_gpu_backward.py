@@ -76,3 +76,34 @@ def test_backward_without_keys_is_zero(gqa_lib):
     dq, dk, dv = gqa.attn_bwd(q, k, k, o, lse, workloads.randn((B, Tq, Hq, d), 2).cuda())
     torch.cuda.synchronize()
     assert dq.shape == q.shape and bool((dq == 0).all())
+
+
+@pytest.mark.parametrize("g", [0, 7])
+def test_backward_headline_shape(gqa_lib, g):
+    # The causal T=4096, 32 / 8 head workload the bench times, full launch on
+    # the GPU.  KV groups are independent problems, so the oracle takes group g
+    # alone (query heads 4g .. 4g+3, K/V head g).  The output of a query row
+    # depends on that row and K/V only, so the oracle runs over blocks of 512
+    # query rows against keys [0, i1): dq of a block is exact, and dk / dv are
+    # the sums of the blocks' contributions.
+    T, Hq, Hkv, d, G = 4096, 32, 8, 128, 4
+    q, k, v = workloads.prefill_inputs(1, T, Hq, Hkv, d)
+    dout = workloads.randn((1, T, Hq, d), 77)
+    qc, kc, vc = q.cuda(), k.cuda(), v.cuda()
+    o, lse = gqa.attn(qc, kc, vc, causal=True, return_lse=True)
+    dq, dk, dv = gqa.attn_bwd(qc, kc, vc, o, lse, dout.cuda())
+    gqa.device_status()
+    hs = slice(g * G, (g + 1) * G)
+    rq = np.zeros((1, T, G, d))
+    rk = np.zeros((1, T, 1, d))
+    rv = np.zeros((1, T, 1, d))
+    for i0 in range(0, T, 512):
+        i1 = i0 + 512
+        a, b, c = ref.attn_bwd(q[:, i0:i1, hs], k[:, :i1, g:g + 1], v[:, :i1, g:g + 1],
+                               dout[:, i0:i1, hs], True)
+        rq[:, i0:i1] = a
+        rk[:, :i1] += b
+        rv[:, :i1] += c
+    assert rel_err(dq[:, :, hs], rq) <= 2e-2
+    assert rel_err(dk[:, :, g:g + 1], rk) <= 2e-2
+    assert rel_err(dv[:, :, g:g + 1], rv) <= 2e-2

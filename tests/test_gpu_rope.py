@@ -69,3 +69,13 @@ def test_attention_with_rope(gqa_lib):
     qg, kg = gqa.rope_(q.cuda(), 0), gqa.rope_(k.cuda(), 0)
     o = gqa.attn(qg, kg, v.cuda(), causal=True)
     assert max_abs(o, o_ref) <= BF16_TOL
+
+
+def test_rope_qk_headline_shape(gqa_lib):
+    # q and k of the B=1, T=4096, 32 / 8 head workload, one launch, positions 0..4095
+    q, k, _ = workloads.prefill_inputs(1, 4096, 32, 8, 128)
+    gq, gk = gqa.rope_qk_(q.cuda(), k.cuda(), 0)
+    for got, x in ((gq, q), (gk, k)):
+        want = ref.rope_tensor(x, 0)
+        rel = np.abs(got.float().cpu().numpy() - want) / np.maximum(np.abs(want), 1e-30)
+        assert np.max(np.where(np.abs(want) > 1e-3, rel, 0.0)) <= 2.0 ** -8

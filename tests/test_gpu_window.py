@@ -59,3 +59,32 @@ def test_decode_window(gqa_lib, Hq, Hkv, window, sinks):
     o = gqa.decode(q.cuda(), kc.cuda(), vc.cuda(), sl.cuda(), window=window, sinks=sinks)
     gqa.device_status()
     assert max_abs(o, o_ref) <= BF16_TOL
+
+
+# ----------------------------------------------------- bench workload sizes --
+
+def test_prefill_window_bench_workload(gqa_lib):
+    # B=1, Hq=32, Hkv=8, T=16384, W=4096, 4 sinks, the inputs the bench times.
+    # The oracle computes blocks of query rows [i0, i1) against keys [0, i1):
+    # with bottom-right alignment those rows see exactly what they see in the
+    # full problem (the start, the first rows past the window, the middle, the end).
+    T, W, S = 16384, 4096, 4
+    q, k, v = workloads.prefill_inputs(1, T, 32, 8, 128, seeds=(11, 12, 13))
+    o, lse = gqa.attn(q.cuda(), k.cuda(), v.cuda(), causal=True, return_lse=True, window=W,
+                      sinks=S)
+    gqa.device_status()
+    assert bool(torch.isfinite(o).all())
+    for i0, i1 in ((0, 128), (W - 64, W + 128), (8128, 8256), (T - 128, T)):
+        o_ref, lse_ref = ref.attn_fwd_window(q[:, i0:i1], k[:, :i1], v[:, :i1], W, S)
+        assert max_abs(o[:, i0:i1], o_ref) <= BF16_TOL
+        assert max_abs(lse[:, :, i0:i1], lse_ref) <= BF16_TOL
+
+
+def test_decode_window_bench_workload(gqa_lib):
+    # the batched-decode workload (B=64, Hq=32, Hkv=8, L ~ U{1024..8192}, NaN
+    # padding) with W=2048 and 4 sinks: every output row
+    q, kc, vc, sl = workloads.decode_inputs(64, 32, 8, 128, 1024, 8192)
+    o_ref, _ = ref.decode_window(q, kc, vc, sl, 2048, 4)
+    o = gqa.decode(q.cuda(), kc.cuda(), vc.cuda(), sl.cuda(), window=2048, sinks=4)
+    gqa.device_status()
+    assert max_abs(o, o_ref) <= BF16_TOL

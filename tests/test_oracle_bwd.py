@@ -70,3 +70,27 @@ def test_dv_closed_form():
     P = np.array(lab.attention_probs(q[0, :, 0].double().tolist(), k[0, :, 0].double().tolist(),
                                      causal=True))
     assert np.allclose(dv[0, :, 0], P.T @ do[0, :, 0].double().numpy(), rtol=0, atol=1e-12)
+
+
+def test_backward_over_query_blocks_and_groups_sums_to_the_whole():
+    # The full-size GPU test takes one KV group and blocks of query rows
+    # against keys [0, i1): groups are independent problems and each query
+    # row's output depends on that row and K/V only, so dq of a block is exact
+    # and dk / dv are the sums of the blocks' contributions.
+    B, T, Hq, Hkv, d, G, blk = 1, 96, 8, 2, 16, 4, 32
+    q, k, v = rand((B, T, Hq, d), 11), rand((B, T, Hkv, d), 12), rand((B, T, Hkv, d), 13)
+    do = rand((B, T, Hq, d), 14)
+    fq, fk, fv = ref.attn_bwd(q, k, v, do, True)
+    for g in range(Hkv):
+        hs = slice(g * G, (g + 1) * G)
+        rq, rk, rv = np.zeros((B, T, G, d)), np.zeros((B, T, 1, d)), np.zeros((B, T, 1, d))
+        for i0 in range(0, T, blk):
+            i1 = i0 + blk
+            a, b, c = ref.attn_bwd(q[:, i0:i1, hs], k[:, :i1, g:g + 1], v[:, :i1, g:g + 1],
+                                   do[:, i0:i1, hs], True)
+            rq[:, i0:i1] = a
+            rk[:, :i1] += b
+            rv[:, :i1] += c
+        assert np.allclose(rq, fq[:, :, hs], atol=1e-12)
+        assert np.allclose(rk, fk[:, :, g:g + 1], atol=1e-12)
+        assert np.allclose(rv, fv[:, :, g:g + 1], atol=1e-12)

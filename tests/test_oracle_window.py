@@ -108,3 +108,16 @@ def test_window_rejects_bad_arguments():
         ref.attn_fwd_window(q, k, v, window=0)
     with pytest.raises(ValueError):
         ref.attn_fwd_window(q, k, v, window=4, sinks=-1)
+
+
+def test_query_block_against_keys_up_to_its_end_equals_the_full_rows():
+    # The full-size GPU window test checks blocks of query rows [i0, i1) against
+    # the oracle run on keys [0, i1) only: with bottom-right alignment those rows
+    # keep their positions, so window and sinks select the same keys.
+    T, W, S = 300, 70, 3
+    q, k, v = rand((1, T, 4, 8), 21), rand((1, T, 2, 8), 22), rand((1, T, 2, 8), 23)
+    o, lse = ref.attn_fwd_window(q, k, v, W, S)
+    for i0, i1 in ((0, 40), (60, 130), (250, 300)):
+        ob, lb = ref.attn_fwd_window(q[:, i0:i1], k[:, :i1], v[:, :i1], W, S)
+        assert np.array_equal(ob, o[:, i0:i1])
+        assert np.array_equal(lb, lse[:, :, i0:i1])
