@@ -8,7 +8,7 @@ import torch
 import grouped_query_attention_attn_b200 as gqa
 from grouped_query_attention_attn_b200 import workloads
 from oracle import ref
-from parity import BF16_TOL, max_abs
+from parity import BF16_TOL, gather_rows, max_abs, sample_rows
 
 pytestmark = pytest.mark.gpu
 
@@ -67,3 +67,16 @@ def test_host_forward_with_completion_event(gqa_lib):
         ev.synchronize()
         o_ref, _ = ref.attn_fwd(q, k, v, True)
         assert max_abs(o, o_ref) <= BF16_TOL
+
+
+def test_host_forward_headline_shape(gqa_lib):
+    # the end-to-end path the bench times: causal B=1, T=4096, 32 / 8 heads from
+    # pinned host tensors (16 chunks of 256 rows), sampled rows against the oracle
+    q, k, v = workloads.prefill_inputs(1, 4096, 32, 8, 128)
+    qp, kp, vp = q.pin_memory(), k.pin_memory(), v.pin_memory()
+    o = gqa.attn_host(qp, kp, vp, causal=True)
+    torch.cuda.synchronize()
+    gqa.device_status()
+    rows = sample_rows(1, 4096, 32, 512, 3)
+    o_ref, _ = ref.attn_fwd_rows(q, k, v, rows, True)
+    assert max_abs(gather_rows(o, rows, 4096, 32), o_ref) <= BF16_TOL
