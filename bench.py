@@ -7,7 +7,8 @@ One step = one pass of the whole hot path over one batch of synthetic input:
   1. causal prefill, B=1, Hq=32, Hkv=8, T=4096, d=128 (Llama-3-8B head
      shapes), bf16 in/out, fp32 accumulation -- the headline workload;
   2. batched decode, B=64 sequences, Hq=32, Hkv=8, d=128, cache lengths
-     uniform on [1024, 8192], split-KV kernel + log-sum-exp combine.
+     uniform on [1024, 8192], split-KV kernel whose last split per group
+     merges the splits (log-sum-exp).
 Inputs are seeded synthetic tensors already resident in HBM.  L2 (126 MB) is
 flushed by writing a 256 MB buffer before every timed launch; each launch is
 timed with CUDA events on the stream it runs on.
@@ -91,22 +92,68 @@ def recorded_traffic(kernel, src_hash):
 
 
 class ClockSampler:
-    """nvidia-smi clock / throttle sampling while the timed region runs."""
+    """SM clock and throttle reasons sampled while a timed region runs.
 
-    FIELDS = ("clocks.sm,clocks.max.sm,clocks_event_reasons.hw_slowdown,"
-              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
-              "clocks_event_reasons.sw_power_cap")
+    A background thread polls NVML (read-only queries) every ``period_s``, so
+    even a region of a few milliseconds gets samples; without NVML it falls back
+    to ``nvidia-smi -lms``.  ``stop()`` returns the median SM clock under load,
+    the maximum SM clock, the sample count and every throttle reason seen."""
 
-    def __init__(self, device):
+    REASONS = (("hw_slowdown", "nvmlClocksEventReasonHwSlowdown"),
+               ("hw_thermal_slowdown", "nvmlClocksEventReasonHwThermalSlowdown"),
+               ("sw_thermal_slowdown", "nvmlClocksEventReasonSwThermalSlowdown"),
+               ("sw_power_cap", "nvmlClocksEventReasonSwPowerCap"))
+
+    def __init__(self, device, period_s=0.001):
+        import threading
+        self.period_s = period_s
+        self.samples, self.reasons, self.smax = [], set(), None
+        self.stop_evt = threading.Event()
+        self.thread = None
+        self.handle = None
         self.proc = None
         try:
             self.uuid = "GPU-" + str(torch.cuda.get_device_properties(device).uuid)
         except Exception:
             self.uuid = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nvml = pynvml
+            self.handle = pynvml.nvmlDeviceGetHandleByUUID(self.uuid.encode()) if self.uuid \
+                else pynvml.nvmlDeviceGetHandleByIndex(torch.cuda.current_device())
+            self.smax = float(pynvml.nvmlDeviceGetMaxClockInfo(self.handle, pynvml.NVML_CLOCK_SM))
+        except Exception:
+            self.handle = None
+
+    def _poll(self):
+        nv, h = self.nvml, self.handle
+        masks = [(name, getattr(nv, attr, 0)) for name, attr in self.REASONS]
+        while not self.stop_evt.is_set():
+            try:
+                self.samples.append(float(nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)))
+                bits = nv.nvmlDeviceGetCurrentClocksEventReasons(h)
+                for name, m in masks:
+                    if m and bits & m:
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            self.stop_evt.wait(self.period_s)
 
     def start(self):
-        cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-               "-lms", "50"]
+        if self.handle is not None:
+            import threading
+            # the launch loop holds the GIL between launches: switch threads
+            # every 0.1 ms so the poller runs during a short timed region
+            self.old_switch = sys.getswitchinterval()
+            sys.setswitchinterval(1e-4)
+            self.thread = threading.Thread(target=self._poll, daemon=True)
+            self.thread.start()
+            return
+        fields = ("clocks.sm,clocks.max.sm,clocks_event_reasons.hw_slowdown,"
+                  "clocks_event_reasons.hw_thermal_slowdown,"
+                  "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+        cmd = ["nvidia-smi", f"--query-gpu={fields}", "--format=csv,noheader,nounits", "-lms", "10"]
         if self.uuid:
             cmd += ["-i", self.uuid]
         try:
@@ -116,26 +163,35 @@ class ClockSampler:
             self.proc = None
 
     def stop(self):
-        if self.proc is None:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
-        self.proc.terminate()
-        out, _ = self.proc.communicate(timeout=10)
-        sm, smax, reasons = [], None, set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for line in out.strip().splitlines():
-            parts = [x.strip() for x in line.split(",")]
-            if len(parts) < 6:
-                continue
-            try:
-                sm.append(float(parts[0]))
-                smax = float(parts[1])
-            except ValueError:
-                continue
-            for n, v in zip(names, parts[2:6]):
-                if v.lower().startswith("active"):
-                    reasons.add(n)
-        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax,
-                "samples": len(sm), "reasons": sorted(reasons)}
+        if self.thread is not None:
+            self.stop_evt.set()
+            self.thread.join(timeout=5)
+            sys.setswitchinterval(self.old_switch)
+            src = "nvml"
+        elif self.proc is not None:
+            self.proc.terminate()
+            out, _ = self.proc.communicate(timeout=10)
+            names = [n for n, _ in self.REASONS]
+            for line in out.strip().splitlines():
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) < 6:
+                    continue
+                try:
+                    self.samples.append(float(parts[0]))
+                    self.smax = float(parts[1])
+                except ValueError:
+                    continue
+                for n, v in zip(names, parts[2:6]):
+                    if v.lower().startswith("active"):
+                        self.reasons.add(n)
+            src = "nvidia-smi"
+        else:
+            return {"sm_mhz": None, "sm_max_mhz": None, "samples": 0,
+                    "reasons": ["no clock source"]}
+        sm = self.samples
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": self.smax,
+                "sm_min_mhz": min(sm) if sm else None, "samples": len(sm),
+                "reasons": sorted(self.reasons), "source": src}
 
 
 def dist_init(n_gpus):
@@ -255,16 +311,26 @@ def time_median(fn, flush, stream, reps):
     return statistics.median(ts)
 
 
-def measure_next_rows(dev, stream, flush, peaks, peak_kind, reps):
-    """Throughput of the rows built after the hot path (each on its own workload)."""
+SWEEP = dict(B=4, Hq=32, T=2048, d=128, causal=True)          # Hkv in {32, 8, 1}
+LONG = dict(B=1, Hq=64, Hkv=8, T=32768, d=128, causal=True, qk_std=8.0)
+NEXT_ROWS = ("prefill_sweep_hkv32", "prefill_sweep_hkv8", "prefill_sweep_hkv1",
+             "prefill_long_t32768", "prefill_window", "backward", "rope_qk", "prefill_rope_fused",
+             "fold_kv", "decode_window", "decode_rope_fused")
+
+
+def measure_next_rows(dev, stream, flush, peaks, peak_kind, reps, which=None):
+    """Throughput of the other prefill workloads and of the rows built after the
+    hot path, each on its own workload; ``which`` selects rows by name."""
     import grouped_query_attention_attn_b200 as gqa
     from grouped_query_attention_attn_b200 import workloads
+    want = set(NEXT_ROWS if not which else which)
 
     def tensor_row(flops, ms, cfg):
         a = flops / (ms / 1e3) / 1e12
         return {"value": a, "unit": "TFLOP/s", "ms": ms, "config": cfg,
                 "roofline": {"bound": "tensor", "achieved": a, "peak": peaks["bf16_tflops"],
                              "unit": "TFLOP/s", "frac": a / peaks["bf16_tflops"],
+                             "frac_of_nominal_2250": a / 2250.0,
                              "peak_kind": f"{peak_kind} bf16 burst", "flops_per_launch": flops}}
 
     def hbm_row(nbytes, ms, cfg):
@@ -275,49 +341,123 @@ def measure_next_rows(dev, stream, flush, peaks, peak_kind, reps):
                              "peak_kind": f"{peak_kind} copy", "bytes_per_launch": nbytes}}
 
     out = {}
+    sampler = ClockSampler(dev)
+    sampler.start()
+    # the same-weights head-sharing sweep: one q, the Hkv=32 K/V and its GPU
+    # folds to 8 and 1 heads; the FLOPs do not depend on Hkv
+    if want & {"prefill_sweep_hkv32", "prefill_sweep_hkv8", "prefill_sweep_hkv1"}:
+        c = SWEEP
+        q, k32, v32 = (t.to(dev) for t in workloads.prefill_inputs(c["B"], c["T"], c["Hq"],
+                                                                   32, c["d"]))
+        o = torch.empty_like(q)
+        flops = 4 * c["B"] * c["Hq"] * c["d"] * visible_pairs(c["T"], c["T"])
+        for hkv in (32, 8, 1):
+            name = f"prefill_sweep_hkv{hkv}"
+            if name not in want:
+                continue
+            k, v = (k32, v32) if hkv == 32 else (gqa.fold_kv(k32, hkv), gqa.fold_kv(v32, hkv))
+            ms = time_median(lambda: gqa.attn(q, k, v, causal=True, out=o), flush, stream, reps)
+            out[name] = tensor_row(flops, ms, dict(c, Hkv=hkv, G=c["Hq"] // hkv,
+                                                   kv="fold_kv of the Hkv=32 K/V"))
+        del q, k32, v32, o
+    # long-context causal prefill with q, k x 8 (logits of sigma ~ 64)
+    if "prefill_long_t32768" in want:
+        c = LONG
+        q, k, v = (t.to(dev) for t in workloads.prefill_inputs(c["B"], c["T"], c["Hq"], c["Hkv"],
+                                                              c["d"], qk_std=c["qk_std"]))
+        o = torch.empty_like(q)
+        ms = time_median(lambda: gqa.attn(q, k, v, causal=True, out=o), flush, stream,
+                         max(3, reps // 4))
+        out["prefill_long_t32768"] = tensor_row(
+            4 * c["Hq"] * c["d"] * visible_pairs(c["T"], c["T"]), ms, c)
+        del q, k, v, o
     # sliding window + sinks prefill (Mistral-like window over a long prompt)
-    cw = dict(B=1, Hq=32, Hkv=8, T=16384, d=128, window=4096, sinks=4)
-    q, k, v = (t.to(dev) for t in workloads.prefill_inputs(1, cw["T"], cw["Hq"], cw["Hkv"], 128,
-                                                          seeds=(11, 12, 13)))
-    o = torch.empty_like(q)
-    ms = time_median(lambda: gqa.attn(q, k, v, causal=True, out=o, window=cw["window"],
-                                      sinks=cw["sinks"]), flush, stream, reps)
-    flops = 4 * cw["Hq"] * 128 * visible_pairs(cw["T"], cw["T"], True, cw["window"], cw["sinks"])
-    out["prefill_window"] = tensor_row(flops, ms, cw)
-    del q, k, v, o
-    # backward on the headline prefill workload (5 algorithmic matmuls)
-    c = PREFILL
-    q, k, v = (t.to(dev) for t in workloads.prefill_inputs(1, c["T"], c["Hq"], c["Hkv"], 128))
-    do = workloads.randn((1, c["T"], c["Hq"], 128), 77).to(dev)
-    o, lse = gqa.attn(q, k, v, causal=True, return_lse=True)
-    ws = torch.empty(int(gqa._binding.gqa_attn_bwd_workspace_size(1, c["T"], c["Hq"])),
-                     dtype=torch.uint8, device=dev)
-    ms = time_median(lambda: gqa.attn_bwd(q, k, v, o, lse, do, workspace=ws), flush, stream, reps)
-    out["backward"] = tensor_row(10 * c["Hq"] * 128 * visible_pairs(c["T"], c["T"]), ms,
-                                 dict(c, kernels="rowdot + dkdv (tcgen05) + dq (tcgen05)"))
-    # RoPE of q and k of the same workload, in place (read + write)
-    ms = time_median(lambda: gqa.rope_qk_(q, k, 0), flush, stream, reps)
-    out["rope_qk"] = hbm_row(2 * (q.numel() + k.numel()) * 2, ms, dict(c, theta=10000.0))
-    del q, k, v, o, lse, do, ws
+    if "prefill_window" in want:
+        cw = dict(B=1, Hq=32, Hkv=8, T=16384, d=128, window=4096, sinks=4)
+        q, k, v = (t.to(dev) for t in workloads.prefill_inputs(1, cw["T"], cw["Hq"], cw["Hkv"],
+                                                              128, seeds=(11, 12, 13)))
+        o = torch.empty_like(q)
+        ms = time_median(lambda: gqa.attn(q, k, v, causal=True, out=o, window=cw["window"],
+                                          sinks=cw["sinks"]), flush, stream, reps)
+        flops = 4 * cw["Hq"] * 128 * visible_pairs(cw["T"], cw["T"], True, cw["window"],
+                                                   cw["sinks"])
+        out["prefill_window"] = tensor_row(flops, ms, cw)
+        del q, k, v, o
+    # backward and RoPE on the headline prefill workload
+    if want & {"backward", "rope_qk", "prefill_rope_fused"}:
+        c = PREFILL
+        q, k, v = (t.to(dev) for t in workloads.prefill_inputs(1, c["T"], c["Hq"], c["Hkv"], 128))
+        if "backward" in want:
+            do = workloads.randn((1, c["T"], c["Hq"], 128), 77).to(dev)
+            o, lse = gqa.attn(q, k, v, causal=True, return_lse=True)
+            ws = torch.empty(int(gqa._binding.gqa_attn_bwd_workspace_size(1, c["T"], c["Hq"])),
+                             dtype=torch.uint8, device=dev)
+            ms = time_median(lambda: gqa.attn_bwd(q, k, v, o, lse, do, workspace=ws), flush,
+                             stream, reps)
+            out["backward"] = tensor_row(10 * c["Hq"] * 128 * visible_pairs(c["T"], c["T"]), ms,
+                                         dict(c, kernels="rowdot + dkdv (tcgen05) + dq (tcgen05)"))
+            del o, lse, do, ws
+        if "rope_qk" in want:
+            # q and k rotated in place (read + write)
+            ms = time_median(lambda: gqa.rope_qk_(q, k, 0), flush, stream, reps)
+            out["rope_qk"] = hbm_row(2 * (q.numel() + k.numel()) * 2, ms, dict(c, theta=10000.0))
+        if "prefill_rope_fused" in want:
+            # rotary embedding + attention: k rotated once (as when it enters the
+            # cache) and q rotated inside the prefill as its tiles are loaded,
+            # against rotating q and k in one launch and then the plain prefill
+            o = torch.empty_like(q)
+            ms_f = time_median(lambda: (gqa.rope_(k, 0),
+                                        gqa.attn(q, k, v, causal=True, out=o, rope_theta=10000.0)),
+                               flush, stream, reps)
+            ms_u = time_median(lambda: (gqa.rope_qk_(q, k, 0), gqa.attn(q, k, v, causal=True, out=o)),
+                               flush, stream, reps)
+            row = tensor_row(prefill_flops(c), ms_f, dict(c, theta=10000.0,
+                                                          launches="rope(k) + prefill(rope q)"))
+            row["unfused_ms"] = ms_u
+            row["unfused"] = "rope_qk(q, k) + prefill"
+            out["prefill_rope_fused"] = row
+            del o
+        del q, k, v
     # MHA -> GQA fold of the head-sharing sweep's K (32 -> 8 heads)
-    kv = workloads.randn((4, 2048, 32, 128), 2).to(dev)
-    ms = time_median(lambda: gqa.fold_kv(kv, 8), flush, stream, reps)
-    out["fold_kv"] = hbm_row(kv.numel() * 2 + kv.numel() // 4 * 2, ms,
-                             dict(B=4, T=2048, H=32, g=8, d=128))
-    del kv
+    if "fold_kv" in want:
+        kv = workloads.randn((4, 2048, 32, 128), 2).to(dev)
+        ms = time_median(lambda: gqa.fold_kv(kv, 8), flush, stream, reps)
+        out["fold_kv"] = hbm_row(kv.numel() * 2 + kv.numel() // 4 * 2, ms,
+                                 dict(B=4, T=2048, H=32, g=8, d=128))
+        del kv
     # sliding-window decode on the batched-decode workload
-    dc = DECODE
-    dq_, kc, vc, sl = workloads.decode_inputs(dc["B"], dc["Hq"], dc["Hkv"], dc["d"], dc["Lmin"],
-                                              dc["Lmax"])
-    W, S = 2048, 4
-    rows = sum(min(int(L), W) + min(S, max(0, int(L) - W)) for L in sl)
-    nbytes = rows * dc["Hkv"] * dc["d"] * 4 + 2 * dc["B"] * dc["Hq"] * dc["d"] * 2
-    dq_, kc, vc, sl = dq_.to(dev), kc.to(dev), vc.to(dev), sl.to(dev)
-    ws = torch.empty(gqa.decode_workspace_size(dc["B"], dc["Hq"], dc["Hkv"], dc["d"], dc["Lmax"]),
-                     dtype=torch.uint8, device=dev)
-    ms = time_median(lambda: gqa.decode(dq_, kc, vc, sl, workspace=ws, window=W, sinks=S), flush,
-                     stream, reps)
-    out["decode_window"] = hbm_row(nbytes, ms, dict(dc, window=W, sinks=S))
+    if "decode_window" in want:
+        dc = DECODE
+        dq_, kc, vc, sl = workloads.decode_inputs(dc["B"], dc["Hq"], dc["Hkv"], dc["d"],
+                                                  dc["Lmin"], dc["Lmax"])
+        W, S = 2048, 4
+        rows = sum(min(int(L), W) + min(S, max(0, int(L) - W)) for L in sl)
+        nbytes = rows * dc["Hkv"] * dc["d"] * 4 + 2 * dc["B"] * dc["Hq"] * dc["d"] * 2
+        dq_, kc, vc, sl = dq_.to(dev), kc.to(dev), vc.to(dev), sl.to(dev)
+        ws = torch.empty(gqa.decode_workspace_size(dc["B"], dc["Hq"], dc["Hkv"], dc["d"],
+                                                   dc["Lmax"]), dtype=torch.uint8, device=dev)
+        ms = time_median(lambda: gqa.decode(dq_, kc, vc, sl, workspace=ws, window=W, sinks=S),
+                         flush, stream, reps)
+        out["decode_window"] = hbm_row(nbytes, ms, dict(dc, window=W, sinks=S))
+    if "decode_rope_fused" in want:
+        dc = DECODE
+        dq_, kc, vc, sl = workloads.decode_inputs(dc["B"], dc["Hq"], dc["Hkv"], dc["d"],
+                                                  dc["Lmin"], dc["Lmax"])
+        nbytes = decode_bytes(sl, dc)
+        dq_, kc, vc, sl = dq_.to(dev), kc.to(dev), vc.to(dev), sl.to(dev)
+        ws = torch.empty(gqa.decode_workspace_size(dc["B"], dc["Hq"], dc["Hkv"], dc["d"],
+                                                   dc["Lmax"]), dtype=torch.uint8, device=dev)
+        o = torch.empty_like(dq_)
+        ms_f = time_median(lambda: gqa.decode(dq_, kc, vc, sl, workspace=ws, out=o,
+                                              rope_theta=10000.0), flush, stream, reps)
+        ms_u = time_median(lambda: (gqa.rope_decode_q_(dq_, sl),
+                                    gqa.decode(dq_, kc, vc, sl, workspace=ws, out=o)),
+                           flush, stream, reps)
+        row = hbm_row(nbytes, ms_f, dict(dc, theta=10000.0, launches="decode(rope q)"))
+        row["unfused_ms"] = ms_u
+        row["unfused"] = "rope_decode_q + decode"
+        out["decode_rope_fused"] = row
+    out["clocks"] = sampler.stop()
     return out
 
 
@@ -341,7 +481,8 @@ def run_ours(args, world, rank, local):
     if args.only == "next":
         # the rows beyond the hot path alone (profiling runs of their kernels)
         peaks, peak_kind = load_peaks()
-        nxt = measure_next_rows(dev, stream, flush, peaks, peak_kind, args.next_reps)
+        nxt = measure_next_rows(dev, stream, flush, peaks, peak_kind, args.next_reps,
+                                args.rows.split(",") if args.rows else None)
         if rank == 0:
             print(json.dumps({"next_rows": nxt}), flush=True)
         return
@@ -467,7 +608,7 @@ def run_ours(args, world, rank, local):
                     "traffic": recorded_traffic("decode_split_kernel",
                                                 kernel_source_hash(["decode.cu", "device.cuh"])),
                     "bytes_per_step": d_bytes, "launch_ms": launch_ms,
-                    "kernels": "decode_split_kernel<128,1> + decode_combine_kernel<128>"}
+                    "kernels": "decode_split_kernel<128,1> (split merge fused)"}
         dec_roof["frac"] = dec_roof["achieved"] / dec_roof["peak"]
         dec_roof["frac_of_nominal_8000"] = dec_roof["achieved"] / 8000.0
         dec = {"value": world * d_bytes * K / (dec_ms / 1e3) / 1e9, "unit": "GB/s",
@@ -492,7 +633,7 @@ def run_ours(args, world, rank, local):
             "roofline": roofline if do_pre else (dec or {}).get("roofline"),
             "clocks": clocks,
             "e2e": e2e,
-            "gpu_launches": K * ((1 if do_pre else 0) + (2 if do_dec else 0)),
+            "gpu_launches": K * ((1 if do_pre else 0) + (1 if do_dec else 0)),
             "wall_s_timed_region": wall,
             "cpu_baseline": cpu,
             "next_rows": nxt,
@@ -520,6 +661,9 @@ def main():
     ap.add_argument("--no-next", action="store_true",
                     help="skip the measurements of the rows beyond the hot path")
     ap.add_argument("--next-reps", type=int, default=20)
+    ap.add_argument("--rows", default=None,
+                    help="with --only next: comma-separated row names (default: all of "
+                         + ", ".join(NEXT_ROWS) + ")")
     args = ap.parse_args()
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")

@@ -3,7 +3,7 @@
 The computation lives in the C-ABI library ``libgqa.so`` (declared in
 ``include/gqa.h``): a tcgen05/TMEM/TMA prefill kernel (causal, full, sliding
 window with sinks, and a host-buffer entry point that pipelines the copies),
-a split-KV decode kernel with a log-sum-exp combine, the tcgen05 backward
+a split-KV decode kernel whose last split per group merges the splits (log-sum-exp), the tcgen05 backward
 (dQ, dK, dV), in-place RoPE, an fp32 path and a head-folding kernel.
 This package is its Python binding; PyTorch is used for device memory and
 streams only.  The library is loaded on first use and there is no CPU

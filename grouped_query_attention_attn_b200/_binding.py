@@ -47,6 +47,11 @@ _SIGNATURES = {
     "gqa_last_error": (ctypes.c_char_p, []),
     "gqa_device_status": (_I, [_I]),
     "gqa_selftest_wait_timeout": (_I, [_I]),
+    "gqa_set_prefill_grid_cap": (None, [_I]),
+    "gqa_selftest_exp2_poly": (_I, [_P, _P, _I, _P]),
+    "gqa_attn_fwd_rope": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _I, _F, _P]),
+    "gqa_decode_rope": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _F, _P, ctypes.c_size_t,
+                             _P]),
 }
 
 
@@ -79,6 +84,12 @@ def gqa_attn_fwd_window(q, k, v, o, lse, B, Tq, Tkv, Hq, Hkv, d, window, sinks, 
                                      scale, stream)
 
 
+def gqa_attn_fwd_rope(q, k, v, o, lse, B, Tq, Tkv, Hq, Hkv, d, causal, scale, q_pos0, theta,
+                      stream):
+    return lib().gqa_attn_fwd_rope(q, k, v, o, lse, B, Tq, Tkv, Hq, Hkv, d, causal, scale, q_pos0,
+                                   theta, stream)
+
+
 def gqa_attn_fwd_f32(q, k, v, o, lse, B, Tq, Tkv, Hq, Hkv, d, causal, scale, stream):
     return lib().gqa_attn_fwd_f32(q, k, v, o, lse, B, Tq, Tkv, Hq, Hkv, d, causal, scale, stream)
 
@@ -91,6 +102,12 @@ def gqa_decode(q, k_cache, v_cache, seqlens, o, B, Hq, Hkv, d, Lmax, scale, work
                workspace_bytes, stream):
     return lib().gqa_decode(q, k_cache, v_cache, seqlens, o, B, Hq, Hkv, d, Lmax, scale,
                             workspace, workspace_bytes, stream)
+
+
+def gqa_decode_rope(q, k_cache, v_cache, seqlens, o, B, Hq, Hkv, d, Lmax, scale, theta, workspace,
+                    workspace_bytes, stream):
+    return lib().gqa_decode_rope(q, k_cache, v_cache, seqlens, o, B, Hq, Hkv, d, Lmax, scale,
+                                 theta, workspace, workspace_bytes, stream)
 
 
 def gqa_decode_window(q, k_cache, v_cache, seqlens, o, B, Hq, Hkv, d, Lmax, window, sinks, scale,
@@ -148,3 +165,12 @@ def gqa_device_status(reset):
 
 def gqa_selftest_wait_timeout(timeout_us):
     return lib().gqa_selftest_wait_timeout(timeout_us)
+
+
+def gqa_set_prefill_grid_cap(max_ctas):
+    """Cap the persistent prefill grid (testing aid; 0 removes the cap)."""
+    lib().gqa_set_prefill_grid_cap(max_ctas)
+
+
+def gqa_selftest_exp2_poly(x, y, n, stream):
+    return lib().gqa_selftest_exp2_poly(x, y, n, stream)

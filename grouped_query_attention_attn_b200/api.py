@@ -49,14 +49,16 @@ def _shapes(q, k, v):
     return B, Tq, Tkv, Hq, Hkv, d
 
 
-def attn(q, k, v, causal=True, scale=None, out=None, return_lse=False, window=None, sinks=0):
+def attn(q, k, v, causal=True, scale=None, out=None, return_lse=False, window=None, sinks=0,
+         rope_theta=None, q_pos0=None):
     """Grouped-query attention forward, bf16.
 
     q [B, Tq, Hq, d], k/v [B, Tkv, Hkv, d] (bf16, contiguous, on one GPU);
     query head h reads K/V head h // (Hq // Hkv).  Returns o [B, Tq, Hq, d]
     (and lse [B, Hq, Tq] fp32 when ``return_lse``).  ``window`` (an int >= 1)
     selects causal sliding-window attention with ``sinks`` always-visible
-    leading keys.
+    leading keys.  ``rope_theta`` rotates q as it is loaded (query row t at
+    position ``q_pos0`` + t, default Tkv - Tq); k must already be rotated.
     """
     for t, n in ((q, "q"), (k, "k"), (v, "v")):
         _need(t, n, torch.bfloat16, 4)
@@ -66,7 +68,14 @@ def attn(q, k, v, causal=True, scale=None, out=None, return_lse=False, window=No
     _need(o, "out", torch.bfloat16, 4)
     lse = torch.empty((B, Hq, Tq), dtype=torch.float32, device=q.device) if return_lse else None
     lp = lse.data_ptr() if lse is not None else None
-    if window is None:
+    if rope_theta is not None:
+        if window is not None:
+            raise NotImplementedError("rope_theta with a sliding window")
+        pos0 = Tkv - Tq if q_pos0 is None else int(q_pos0)
+        rc = _b.gqa_attn_fwd_rope(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lp,
+                                  B, Tq, Tkv, Hq, Hkv, d, int(bool(causal)), scale, pos0,
+                                  float(rope_theta), _stream(q))
+    elif window is None:
         rc = _b.gqa_attn_fwd_lse(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lp,
                                  B, Tq, Tkv, Hq, Hkv, d, int(bool(causal)), scale, _stream(q))
     else:
@@ -152,12 +161,13 @@ def decode_workspace_size(B, Hq, Hkv, d, Lmax):
 
 
 def decode(q, k_cache, v_cache, seqlens, scale=None, workspace=None, out=None, window=None,
-           sinks=0):
+           sinks=0, rope_theta=None):
     """One query token per sequence against a bf16 KV cache.
 
     q [B, Hq, d], caches [B, Lmax, Hkv, d], seqlens int32 [B] on the device.
     ``workspace``: a uint8 CUDA tensor of at least decode_workspace_size(...)
-    bytes (allocated here when None).
+    bytes (allocated here when None).  ``rope_theta`` rotates q as it is loaded
+    (position max(seqlens[b] - 1, 0)); the cached keys must already be rotated.
     """
     _need(q, "q", torch.bfloat16, 3)
     _need(k_cache, "k_cache", torch.bfloat16, 4)
@@ -172,7 +182,14 @@ def decode(q, k_cache, v_cache, seqlens, scale=None, workspace=None, out=None, w
     if workspace is None:
         workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
     o = torch.empty_like(q) if out is None else out
-    if window is None:
+    if rope_theta is not None:
+        if window is not None:
+            raise NotImplementedError("rope_theta with a sliding window")
+        rc = _b.gqa_decode_rope(q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(),
+                                seqlens.data_ptr(), o.data_ptr(), B, Hq, Hkv, d, Lmax, scale,
+                                float(rope_theta), workspace.data_ptr(), workspace.numel(),
+                                _stream(q))
+    elif window is None:
         rc = _b.gqa_decode(q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(),
                            seqlens.data_ptr(), o.data_ptr(), B, Hq, Hkv, d, Lmax, scale,
                            workspace.data_ptr(), workspace.numel(), _stream(q))

@@ -457,8 +457,11 @@ static int launch_dkdv_tc(const void *q, const void *k, const void *v, const voi
     if (int rc = encode_tmap_bf16_4d(&tv, v, D, Hkv, Tkv, B, 64, 1, kTcBK, 1, 1)) return rc;
     auto kern = dkdv_tc_kernel<D>;
     const int smem = TcLayout<D>::kSmemBytes;
-    if (int rc = check_cuda(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                 smem), "cudaFuncSetAttribute(dkdv_tc)"))
+    static CtxSlot setup;   // the shared-memory opt-in, once per context
+    if (int rc = once_per_context(setup, [&](int) {
+            return check_cuda(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                   smem), "cudaFuncSetAttribute(dkdv_tc)");
+        }))
         return rc;
     kern<<<static_cast<unsigned>(blocks), kTcThreads, smem, stream>>>(tq, tk, tv, to, prm);
     return check_cuda(cudaGetLastError(), "dkdv_tc_kernel launch");
@@ -779,8 +782,11 @@ static int launch_dq_tc(const void *q, const void *k, const void *v, const void 
     if (int rc = encode_tmap_bf16_4d(&tv, v, D, Hkv, Tkv, B, 64, 1, kDqBN, 1, 1)) return rc;
     auto kern = dq_tc_kernel<D>;
     const int smem = DqLayout<D>::kSmemBytes;
-    if (int rc = check_cuda(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                 smem), "cudaFuncSetAttribute(dq_tc)"))
+    static CtxSlot setup;   // the shared-memory opt-in, once per context
+    if (int rc = once_per_context(setup, [&](int) {
+            return check_cuda(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                   smem), "cudaFuncSetAttribute(dq_tc)");
+        }))
         return rc;
     kern<<<static_cast<unsigned>(blocks), kTcThreads, smem, stream>>>(tq, to, tk, tv, prm);
     return check_cuda(cudaGetLastError(), "dq_tc_kernel launch");

@@ -1,5 +1,5 @@
 // decode.cu -- split-KV grouped-query decode (one query token per sequence)
-// and the log-sum-exp combine of the splits.
+// with the log-sum-exp merge of the splits in the same kernel.
 //
 // Work unit: one CTA per (split, KV head, sequence).  A split is `chunk`
 // consecutive cache rows; the CTA streams its K and V rows from HBM exactly
@@ -9,14 +9,20 @@
 //   - warp 4 (one thread) issues the TMA copies: per stage 64 keys of K and V
 //     (four 64-column panels with 128-byte swizzle for d = 128);
 //   - warps 0-3 each take 16 keys of every stage: S = Q K^T, the running-max
-//     softmax of the course's step 1 (mask of keys past the sequence end,
-//     max subtracted, exp2 with scale * log2 e folded in), then O += P V;
-//     row max / sum reductions are warp shuffles inside each quad of lanes;
+//     softmax of course "Неделя 7. Внимание", step 1 (mask of keys past the
+//     sequence end, max subtracted, exp2 with scale * log2 e folded in), then
+//     O += P V; row max / sum reductions are warp shuffles inside each quad;
 //   - at the end the four warps' (m, l, O) are merged through shared memory
 //     and the split's normalised O and natural-log lse go to the workspace.
-// The combine kernel then merges the splits of each (sequence, query head):
-//   O = sum_s e^(lse_s - M) O_s / sum_s e^(lse_s - M),  M = max_s lse_s.
+// The last split of a (sequence, KV head) to finish -- found with an arrival
+// counter in the workspace -- then merges the splits of the group's G heads:
+//   O = sum_s e^(lse_s - M) O_s / sum_s e^(lse_s - M),  M = max_s lse_s,
+// so the merge of one group overlaps the other groups' streaming and no
+// second kernel waits for the whole grid.
 #include <cuda_bf16.h>
+#include <atomic>
+#include <chrono>
+#include <cmath>
 
 #include "device.cuh"
 #include "internal.h"
@@ -64,23 +70,24 @@ __device__ __forceinline__ uint32_t swz_off(int row, int cg) {
     return (cg >> 3) * DecLayout<D>::kPanelBytes + row * 128 + (((cg & 7) ^ (row & 7)) << 4);
 }
 
-template <int D, int MB>
+// kRope: the query is rotated (rotary position embedding) in registers as it
+// is loaded, at position max(seqlens[b] - 1, 0); the cached keys are rotated.
+template <int D, int MB, bool kRope>
 __global__ void __launch_bounds__(kDecThreads, dec_min_blocks<MB>())
 decode_split_kernel(const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v,
                     const __nv_bfloat16 *__restrict__ q, const int32_t *__restrict__ seqlens,
-                    float *__restrict__ part_o, float *__restrict__ part_lse, int B, int Hq,
-                    int Hkv, int Lmax, int chunk, int window, int sinks, float scale_log2,
-                    int *status) {
+                    float *__restrict__ part_o, float *__restrict__ part_lse,
+                    unsigned long long *__restrict__ arrivals, unsigned long long call_id,
+                    __nv_bfloat16 *__restrict__ o, int B, int Hq, int Hkv, int Lmax, int chunk,
+                    int window, int sinks, float scale_log2, double log_theta, int *status) {
     using Lay = DecLayout<D, MB>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
     __shared__ uint64_t full_bar[kDecStages], empty_bar[kDecStages];
-    __shared__ int abort_flag;
+    __shared__ int abort_flag, merger;
 
-    // the combine grid may be scheduled now; it waits for this grid's results
-    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     const int split = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z;
     int L = seqlens[b];
     if (L > Lmax || L < 0) {
@@ -93,13 +100,23 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tm_k,
     // window, [0, s_end), as whole stages.  Without a window lo = s_end = 0.
     const int lo = window > 0 ? max(0, L - window) : 0;
     const int s_end = window > 0 ? min(sinks, lo) : 0;
+    const int n_splits = (L - lo + chunk - 1) / chunk;   // splits that hold visible keys
+    const int G = Hq / Hkv;
+    if (split >= n_splits) {
+        // nothing in this split; with no visible key at all (an empty
+        // sequence) split 0 writes the group's output rows as zeros
+        if (split == 0 && threadIdx.x < kDecWarps * 32) {
+            __nv_bfloat16 *og = o + (static_cast<size_t>(b) * Hq + static_cast<size_t>(kvh) * G) * D;
+            for (int idx = threadIdx.x; idx < G * D / 8; idx += kDecWarps * 32)
+                reinterpret_cast<uint4 *>(og)[idx] = make_uint4(0u, 0u, 0u, 0u);
+        }
+        return;
+    }
     const int start = lo + split * chunk;
-    if (start >= L) return;                         // whole block: nothing in this split
     const int end = min(start + chunk, L);
     const int t_s = split == 0 ? (s_end + kDecBK - 1) / kDecBK : 0;   // sink stages
     const int n_iter = t_s + (end - start + kDecBK - 1) / kDecBK;
     const int off_w = start - t_s * kDecBK;         // window stage t starts at key off_w + 64 t
-    const int G = Hq / Hkv;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
     if (threadIdx.x == 0) {
@@ -149,6 +166,28 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tm_k,
             qa[mb][kk][2] = r0 < G ? ld_b32(qg + r0 * D + c1) : 0u;
             qa[mb][kk][3] = r1 < G ? ld_b32(qg + r1 * D + c1) : 0u;
         }
+    }
+    if constexpr (kRope) {
+        // one cosine / sine per coordinate pair, shared by the G heads
+        __shared__ float2 rope_cs[D / 2];
+        const int m = max(seqlens[b] - 1, 0);
+        for (int i = threadIdx.x; i < D / 2; i += kDecWarps * 32) {
+            float cs, sn;
+            rope_cos_sin(m, rope_turns(i, D / 2, log_theta), cs, sn);
+            rope_cs[i] = make_float2(cs, sn);
+        }
+        named_barrier_sync(1, kDecWarps * 32);
+#pragma unroll
+        for (int mb = 0; mb < MB; ++mb)
+#pragma unroll
+            for (int kk = 0; kk < D / 16; ++kk) {
+                // words 0 / 1 hold pair kk * 8 + tq of rows r0 / r1, words 2 / 3 pair + 4
+                const float2 c0 = rope_cs[kk * 8 + tq], c1 = rope_cs[kk * 8 + tq + 4];
+                qa[mb][kk][0] = rope_rotate_pair(qa[mb][kk][0], c0.x, c0.y);
+                qa[mb][kk][1] = rope_rotate_pair(qa[mb][kk][1], c0.x, c0.y);
+                qa[mb][kk][2] = rope_rotate_pair(qa[mb][kk][2], c1.x, c1.y);
+                qa[mb][kk][3] = rope_rotate_pair(qa[mb][kk][3], c1.x, c1.y);
+            }
     }
     float oacc[MB][D / 8][4];
     float m_run[MB][2], l_run[MB][2];
@@ -317,131 +356,157 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tm_k,
         part_o[(row0 + r) * D + c] = acc / wsum;
         if (c == 0) part_lse[row0 + r] = (M + __log2f(wsum)) * 0.69314718055994531f;
     }
-}
 
-template <int D>
-__global__ void __launch_bounds__(128)
-decode_combine_kernel(const float *__restrict__ part_o, const float *__restrict__ part_lse,
-                      const int32_t *__restrict__ seqlens, __nv_bfloat16 *__restrict__ o, int B,
-                      int Hq, int Lmax, int chunk, int window) {
-    constexpr int kPer = D / 32;
-    // launched as a programmatic dependent of the split kernel: wait until all of
-    // its memory operations are complete and visible
-    asm volatile("griddepcontrol.wait;" ::: "memory");
-    const int row = blockIdx.x * 4 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
-    if (row >= B * Hq) return;
-    const int b = row / Hq;
-    int L = seqlens[b];
-    L = L < 0 ? 0 : (L > Lmax ? Lmax : L);
-    const int lo = window > 0 ? max(0, L - window) : 0;   // the splits start at lo
-    const int n = (L - lo + chunk - 1) / chunk;
+    // ---- the last split of this (sequence, KV head) merges all of them ----
+    // Arrival word: call id in the high 48 bits, arrivals of that call in the
+    // low 16.  A word left by another call (or uninitialised memory) restarts
+    // the count at this call; the merging CTA leaves (call id, 0), so a replay
+    // of the same launch (a CUDA graph) counts from zero again.  The CAS loop
+    // ends: every failed attempt means another split's attempt succeeded.
+    __threadfence();                                 // my partial rows, device-wide
+    named_barrier_sync(1, kDecWarps * 32);
+    if (threadIdx.x == 0) {
+        unsigned long long *word = arrivals + static_cast<size_t>(b) * Hkv + kvh;
+        unsigned long long cur = *reinterpret_cast<volatile unsigned long long *>(word), seen;
+        unsigned long long next;
+        do {
+            seen = cur;
+            next = (seen >> 16) == call_id ? seen + 1 : ((call_id << 16) | 1ull);
+            cur = atomicCAS(word, seen, next);
+        } while (cur != seen);
+        const bool last = static_cast<int>(next & 0xFFFFu) == n_splits;
+        if (last) *reinterpret_cast<volatile unsigned long long *>(word) = call_id << 16;
+        merger = last;
+    }
+    named_barrier_sync(1, kDecWarps * 32);
+    if (!merger) return;
+    __threadfence();                                 // every split's partial rows are visible
     const size_t plane = static_cast<size_t>(B) * Hq;
-    float acc[kPer];
-#pragma unroll
-    for (int e = 0; e < kPer; ++e) acc[e] = 0.0f;
-    if (n > 0) {
+    const size_t grow0 = static_cast<size_t>(b) * Hq + static_cast<size_t>(kvh) * G;
+    for (int idx = threadIdx.x; idx < G * D / 2; idx += kDecWarps * 32) {
+        const int r = idx / (D / 2), c = (idx % (D / 2)) * 2;
         float M = -INFINITY;
-        for (int s = 0; s < n; ++s) M = fmaxf(M, part_lse[s * plane + row]);
-        float wsum = 0.0f;
-        for (int s = 0; s < n; ++s) {
-            const float w = __expf(part_lse[s * plane + row] - M);
+        for (int sp = 0; sp < n_splits; ++sp) M = fmaxf(M, __ldcg(part_lse + sp * plane + grow0 + r));
+        float wsum = 0.0f, a0 = 0.0f, a1 = 0.0f;
+        for (int sp = 0; sp < n_splits; ++sp) {
+            const float w = __expf(__ldcg(part_lse + sp * plane + grow0 + r) - M);
+            const float2 v = __ldcg(reinterpret_cast<const float2 *>(
+                part_o + (sp * plane + grow0 + r) * D + c));
             wsum += w;
-            const float *src = part_o + (s * plane + row) * D + lane * kPer;
-#pragma unroll
-            for (int e = 0; e < kPer; ++e) acc[e] += w * src[e];
+            a0 += w * v.x;
+            a1 += w * v.y;
         }
         const float inv = 1.0f / wsum;
-#pragma unroll
-        for (int e = 0; e < kPer; ++e) acc[e] *= inv;
+        *reinterpret_cast<__nv_bfloat162 *>(o + (grow0 + r) * D + c) =
+            __floats2bfloat162_rn(a0 * inv, a1 * inv);
     }
-    __nv_bfloat16 *dst = o + static_cast<size_t>(row) * D + lane * kPer;
-#pragma unroll
-    for (int e = 0; e < kPer; e += 2)
-        *reinterpret_cast<__nv_bfloat162 *>(dst + e) = __floats2bfloat162_rn(acc[e], acc[e + 1]);
 }
 
-int decode_chunk(int /*B*/, int /*Hkv*/, int /*Lmax*/) { return kDecChunk; }
+// Keys per split: kDecChunk; a windowed call (at most `window` keys after the
+// window start) takes half-size splits when the workspace, sized for the
+// plain chunk over Lmax, has room for them -- more, shorter CTAs fill the
+// last wave of a short grid better.
+static int decode_chunk(int Lmax, int window) {
+    const long long plain_splits = (static_cast<long long>(Lmax) + kDecChunk - 1) / kDecChunk;
+    if (window > 0) {
+        const int half = kDecChunk / 2;
+        const long long span = window < Lmax ? window : Lmax;
+        if ((span + half - 1) / half <= plain_splits) return half;
+    }
+    return kDecChunk;
+}
 
 static size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
+// Workspace: partial O [splits, B, Hq, d] fp32 | partial lse [splits, B, Hq]
+// fp32 | arrival words [B, Hkv] u64, splits = ceil(Lmax / kDecChunk).
+struct DecWorkspace {
+    size_t splits, rows, off_lse, off_arrivals, bytes;
+    DecWorkspace(int B, int Hq, int Hkv, int d, int Lmax) {
+        splits = (static_cast<size_t>(Lmax) + kDecChunk - 1) / kDecChunk;
+        rows = splits * B * Hq;
+        off_lse = align256(rows * d * sizeof(float));
+        off_arrivals = off_lse + align256(rows * sizeof(float));
+        bytes = splits ? off_arrivals + align256(static_cast<size_t>(B) * Hkv * 8) : 0;
+    }
+};
+
 size_t decode_workspace_bytes(int B, int Hq, int Hkv, int d, int Lmax) {
-    const int chunk = decode_chunk(B, Hkv, Lmax);
-    const size_t splits = (static_cast<size_t>(Lmax) + chunk - 1) / chunk;
-    const size_t rows = splits * B * Hq;
-    return align256(rows * d * sizeof(float)) + align256(rows * sizeof(float));
+    return DecWorkspace(B, Hq, Hkv, d, Lmax).bytes;
 }
 
-template <int D, int MB>
+// Per-call ids for the arrival words: 48 bits, never 0, different for every
+// launch of the process (the start is drawn from the clock, so a workspace
+// reused by another process is unlikely to hold a matching word either).
+static unsigned long long next_call_id() {
+    static std::atomic<unsigned long long> counter{
+        static_cast<unsigned long long>(
+            std::chrono::steady_clock::now().time_since_epoch().count()) * 0x9E3779B97F4A7C15ull};
+    for (;;) {
+        const unsigned long long id = counter.fetch_add(1) & 0xFFFFFFFFFFFFull;
+        if (id != 0) return id;
+    }
+}
+
+template <int D, int MB, bool kRope>
 static int launch_split(const CUtensorMap &tk, const CUtensorMap &tv, const void *q,
-                        const int32_t *seqlens, float *part_o, float *part_lse, int B, int Hq,
-                        int Hkv, int Lmax, int chunk, int window, int sinks, float scale_log2,
+                        const int32_t *seqlens, float *part_o, float *part_lse,
+                        unsigned long long *arrivals, void *o, int B, int Hq, int Hkv, int Lmax,
+                        int chunk, int window, int sinks, float scale_log2, double log_theta,
                         int *status, cudaStream_t stream) {
-    auto kern = decode_split_kernel<D, MB>;
+    auto kern = decode_split_kernel<D, MB, kRope>;
     const int smem = DecLayout<D, MB>::kSmemBytes;
-    if (int rc = check_cuda(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                 smem), "cudaFuncSetAttribute(decode)"))
+    static CtxSlot setup;   // one per instantiation: the opt-in is set once per context
+    if (int rc = once_per_context(setup, [&](int) {
+            return check_cuda(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                   smem), "cudaFuncSetAttribute(decode)");
+        }))
         return rc;
     const int span = window > 0 ? min(Lmax, window) : Lmax;   // keys after the window start
     dim3 grid((span + chunk - 1) / chunk, Hkv, B);
     kern<<<grid, kDecThreads, smem, stream>>>(tk, tv, static_cast<const __nv_bfloat16 *>(q),
-                                              seqlens, part_o, part_lse, B, Hq, Hkv, Lmax, chunk,
-                                              window, sinks, scale_log2, status);
+                                              seqlens, part_o, part_lse, arrivals, next_call_id(),
+                                              static_cast<__nv_bfloat16 *>(o), B, Hq, Hkv, Lmax,
+                                              chunk, window, sinks, scale_log2, log_theta,
+                                              status);
     return check_cuda(cudaGetLastError(), "decode_split_kernel launch");
 }
 
 int launch_decode(const void *q, const void *k_cache, const void *v_cache,
                   const int32_t *seqlens, void *o, int B, int Hq, int Hkv, int d, int Lmax,
-                  int window, int sinks, float scale, void *workspace, cudaStream_t stream) {
+                  int window, int sinks, float scale, void *workspace, cudaStream_t stream,
+                  float rope_theta) {
     if (B > 65535 || Hkv > 65535)
         return set_error(GQA_ERR_UNSUPPORTED, "decode: B and Hkv must be <= 65535");
+    const DecWorkspace ws(B, Hq, Hkv, d, Lmax);
+    if (ws.splits > 0xFFFF)
+        return set_error(GQA_ERR_UNSUPPORTED, "decode: Lmax=%d gives more than 65535 splits", Lmax);
+    // an empty cache: every output row is zero
+    if (ws.splits == 0) return launch_empty_rows(o, nullptr, 2, B, 1, Hq, d, stream);
     int *status = device_status_ptr();
     if (!status) return GQA_ERR_CUDA;
-    const int chunk = decode_chunk(B, Hkv, Lmax);
-    const size_t splits = (static_cast<size_t>(Lmax) + chunk - 1) / chunk;
-    const size_t rows = splits * B * Hq;
-    float *part_o = static_cast<float *>(workspace);
-    float *part_lse = reinterpret_cast<float *>(static_cast<uint8_t *>(workspace) +
-                                                align256(rows * d * sizeof(float)));
+    const int chunk = decode_chunk(Lmax, window);
+    uint8_t *base = static_cast<uint8_t *>(workspace);
+    float *part_o = reinterpret_cast<float *>(base);
+    float *part_lse = reinterpret_cast<float *>(base + ws.off_lse);
+    auto *arrivals = reinterpret_cast<unsigned long long *>(base + ws.off_arrivals);
     const int G = Hq / Hkv;
     const float scale_log2 = scale * 1.4426950408889634f;
-    if (splits > 0) {
-        CUtensorMap tk, tv;
-        if (int rc = encode_tmap_bf16_4d(&tk, k_cache, d, Hkv, Lmax, B, 64, 1, kDecBK, 1, 1)) return rc;
-        if (int rc = encode_tmap_bf16_4d(&tv, v_cache, d, Hkv, Lmax, B, 64, 1, kDecBK, 1, 1)) return rc;
-        int rc;
-        if (d == 128)
-            rc = G <= 16 ? launch_split<128, 1>(tk, tv, q, seqlens, part_o, part_lse, B, Hq, Hkv,
-                                                Lmax, chunk, window, sinks, scale_log2, status, stream)
-                         : launch_split<128, 2>(tk, tv, q, seqlens, part_o, part_lse, B, Hq, Hkv,
-                                                Lmax, chunk, window, sinks, scale_log2, status, stream);
-        else
-            rc = G <= 16 ? launch_split<64, 1>(tk, tv, q, seqlens, part_o, part_lse, B, Hq, Hkv,
-                                               Lmax, chunk, window, sinks, scale_log2, status, stream)
-                         : launch_split<64, 2>(tk, tv, q, seqlens, part_o, part_lse, B, Hq, Hkv,
-                                               Lmax, chunk, window, sinks, scale_log2, status, stream);
-        if (rc) return rc;
+    CUtensorMap tk, tv;
+    if (int rc = encode_tmap_bf16_4d(&tk, k_cache, d, Hkv, Lmax, B, 64, 1, kDecBK, 1, 1)) return rc;
+    if (int rc = encode_tmap_bf16_4d(&tv, v_cache, d, Hkv, Lmax, B, 64, 1, kDecBK, 1, 1)) return rc;
+    const bool rope = rope_theta > 0.0f;
+    const double log_theta = rope ? log(static_cast<double>(rope_theta)) : 0.0;
+#define GQA_DEC_LAUNCH(DD, MBB, RR)                                                             \
+    launch_split<DD, MBB, RR>(tk, tv, q, seqlens, part_o, part_lse, arrivals, o, B, Hq, Hkv, Lmax, \
+                              chunk, window, sinks, scale_log2, log_theta, status, stream)
+    if (d == 128) {
+        if (G <= 16) return rope ? GQA_DEC_LAUNCH(128, 1, true) : GQA_DEC_LAUNCH(128, 1, false);
+        return rope ? GQA_DEC_LAUNCH(128, 2, true) : GQA_DEC_LAUNCH(128, 2, false);
     }
-    // The combine kernel is a programmatic dependent launch: it is scheduled
-    // while the split kernel drains and waits (griddepcontrol.wait) for its results.
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((B * Hq + 3) / 4);
-    cfg.blockDim = dim3(128);
-    cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    __nv_bfloat16 *ob = static_cast<__nv_bfloat16 *>(o);
-    const cudaError_t e =
-        d == 128 ? cudaLaunchKernelEx(&cfg, decode_combine_kernel<128>, (const float *)part_o,
-                                      (const float *)part_lse, seqlens, ob, B, Hq, Lmax, chunk,
-                                      window)
-                 : cudaLaunchKernelEx(&cfg, decode_combine_kernel<64>, (const float *)part_o,
-                                      (const float *)part_lse, seqlens, ob, B, Hq, Lmax, chunk,
-                                      window);
-    if (int rc = check_cuda(e, "decode_combine_kernel launch")) return rc;
-    return check_cuda(cudaGetLastError(), "decode_combine_kernel launch");
+    if (G <= 16) return rope ? GQA_DEC_LAUNCH(64, 1, true) : GQA_DEC_LAUNCH(64, 1, false);
+    return rope ? GQA_DEC_LAUNCH(64, 2, true) : GQA_DEC_LAUNCH(64, 2, false);
+#undef GQA_DEC_LAUNCH
 }
 
 }  // namespace gqa

@@ -11,10 +11,10 @@
 // The scratch is a file-scope __device__ array of kStaticScratchBytes.  Every
 // GPU that loads this code holds it until the process exits.  In host code the
 // array's name is only a host-side stand-in, so its device address is looked
-// up with cudaGetSymbolAddress once per device (on the first call made with
-// that device current) and that address is what the kernels receive.
-#include <mutex>
-
+// up with cudaGetSymbolAddress and that address is what the kernels receive.
+// The lookup runs on the first call made in a CUDA context (the first call on
+// each device, and again after a cudaDeviceReset, which loads the module anew)
+// and is cached for that context.
 #include "internal.h"
 
 namespace gqa {
@@ -24,29 +24,12 @@ constexpr size_t kStaticScratchBytes = 32u << 20;
 
 static __device__ __align__(256) unsigned char g_decode_scratch[kStaticScratchBytes];
 
-// Device address of g_decode_scratch on the current device, looked up once per
-// device; nullptr (message set) on failure.
+// Device address of g_decode_scratch in the current context; nullptr (message
+// set) on failure.
 static void *static_scratch_ptr() {
-    static void *cache[64] = {};
-    static std::mutex mu;
-    int dev = 0;
-    if (int rc = check_cuda(cudaGetDevice(&dev), "cudaGetDevice")) {
-        (void)rc;
-        return nullptr;
-    }
-    if (dev < 0 || dev >= 64) {
-        set_error(GQA_ERR_UNSUPPORTED, "gqa_decode_static: device ordinal %d >= 64", dev);
-        return nullptr;
-    }
-    std::lock_guard<std::mutex> lock(mu);
-    if (!cache[dev]) {
-        void *ptr = nullptr;
-        if (check_cuda(cudaGetSymbolAddress(&ptr, g_decode_scratch),
-                       "gqa_decode_static: cudaGetSymbolAddress"))
-            return nullptr;
-        cache[dev] = ptr;
-    }
-    return cache[dev];
+    static SymbolSlot slot;
+    return symbol_address(reinterpret_cast<const void *>(&g_decode_scratch), slot,
+                          "gqa_decode_static: cudaGetSymbolAddress");
 }
 
 }  // namespace gqa
@@ -55,23 +38,28 @@ extern "C" int gqa_decode_static(const void *q, const void *k_cache, const void 
                                  const int32_t *seqlens, void *o, int B, int Hq, int Hkv, int d,
                                  int Lmax, float scale, gqa_stream_t stream) {
     using namespace gqa;
-    // Sizes are checked before the scratch is touched, so an oversize request
-    // fails cleanly (and nothing is launched).
-    const size_t need = gqa_decode_workspace_size(B, Hq, Hkv, d, Lmax);
+    clear_error();
+    // The same argument checks and errors as gqa_decode, before anything else.
+    if (int rc = validate_decode(q, k_cache, v_cache, seqlens, o, B, Hq, Hkv, d, Lmax, scale))
+        return rc;
+    // Then the size check, before the scratch is touched: an oversize request
+    // fails cleanly and nothing is launched.
+    const size_t need = decode_workspace_bytes(B, Hq, Hkv, d, Lmax);
     if (need > kStaticScratchBytes)
         return set_error(GQA_ERR_WORKSPACE,
                          "gqa_decode_static: B=%d, Hq=%d, d=%d, Lmax=%d need %zu bytes of "
                          "scratch; the built-in scratch holds %zu (use gqa_decode with a "
                          "caller workspace)",
                          B, Hq, d, Lmax, need, kStaticScratchBytes);
-    // No scratch needed (empty batch, empty cache) or invalid sizes: gqa_decode
-    // validates and answers without touching any scratch.
-    if (need == 0) return gqa_decode(q, k_cache, v_cache, seqlens, o, B, Hq, Hkv, d, Lmax, scale,
-                                     nullptr, 0, stream);
-    void *scratch = static_scratch_ptr();
-    if (!scratch) return GQA_ERR_CUDA;
+    if (B == 0) return GQA_OK;
+    if (int rc = require_sm100()) return rc;
+    void *scratch = nullptr;
+    if (need > 0) {
+        scratch = static_scratch_ptr();
+        if (!scratch) return GQA_ERR_CUDA;
+    }
     // Nothing in the scratch has to start at zero: every partial result the
-    // combine kernel reads is written earlier in the same call.
-    return gqa_decode(q, k_cache, v_cache, seqlens, o, B, Hq, Hkv, d, Lmax, scale, scratch,
-                      kStaticScratchBytes, stream);
+    // merge reads is written earlier in the same call.
+    return launch_decode(q, k_cache, v_cache, seqlens, o, B, Hq, Hkv, d, Lmax, 0, 0, scale,
+                         scratch, reinterpret_cast<cudaStream_t>(stream));
 }

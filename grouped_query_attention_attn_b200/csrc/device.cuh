@@ -188,6 +188,17 @@ __device__ __forceinline__ void tmem_ld64(uint32_t taddr, uint32_t (&a)[32], uin
         : "r"(taddr));
 }
 
+// 32 lanes x 16 consecutive 32-bit columns (thread t: lane 32 * (warp % 4) + t).
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]),
+          "=r"(r[6]), "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]),
+          "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr));
+}
+
 __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
     asm volatile(
         "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
@@ -337,15 +348,17 @@ __device__ __forceinline__ uint32_t pack_hi16(float lo, float hi) {
 // fitted by csrc/fit_exp2_poly.py (max relative error 7.5e-5); 2^n applied by
 // adding n to the exponent field with an integer multiply-add
 // (bits(t) * 2^23 == n << 23 mod 2^32 because the constant's low 9 bits are
-// zero).  x is clamped to >= -126 so the result stays a normal float
-// (2^-126 stands in for anything smaller).  Not for x = -inf: masked scores
+// zero).  x is clamped to >= -125 so the result stays a normal float: 2^f can
+// fall just below 1 (exponent field 126), and with n = -126 the add would
+// leave an exponent field of 0, a denormal that reads as 2 * 2^f - 1 times
+// 2^-126.  Anything below -125 gives 2^-125.  Not for x = -inf: masked scores
 // use the MUFU path.
 __device__ __forceinline__ float2 exp2_poly2(float2 x) {
     constexpr float kC0 = 9.999280572e-01f, kC1 = 6.932609677e-01f;
     constexpr float kC2 = 2.426111251e-01f, kC3 = 5.517166853e-02f;
     constexpr float kRound = 12582912.0f;                    // 1.5 * 2^23
-    x.x = fmaxf(x.x, -126.0f);
-    x.y = fmaxf(x.y, -126.0f);
+    x.x = fmaxf(x.x, -125.0f);
+    x.y = fmaxf(x.y, -125.0f);
     const float2 t = add2(x, make_float2(kRound, kRound));  // round(x) in the low bits
     const float2 n = add2(t, make_float2(-kRound, -kRound));
     const float2 f = add2(x, make_float2(-n.x, -n.y));
@@ -369,6 +382,33 @@ __device__ __forceinline__ float add_bf16x2(float acc, uint32_t w) {
 // The two bf16 halves of a packed word, widened to fp32 (exact).
 __device__ __forceinline__ float2 bf16x2_to_float2(uint32_t w) {
     return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u));
+}
+
+// ------------------------------------------------------------------ RoPE --
+// Course "Неделя 7. Внимание", step 3: coordinate pair (2i, 2i+1) of a row at
+// position m turns by m * theta_i, theta_i = theta^(-2i/d).  The angle reaches
+// ~10^4 rad at long context, so it is carried as a number of turns
+// m * theta_i / (2 pi), reduced to [-1/2, 1/2] in double, and sincospif gives
+// the fp32 sine and cosine.  Every kernel that rotates uses these three
+// functions, so a fused rotation gives the same bits as the standalone one.
+
+// theta_i / (2 pi) for pair i of `half` = d / 2 pairs (log_theta = ln theta).
+__device__ __forceinline__ double rope_turns(int i, int half, double log_theta) {
+    return exp(-static_cast<double>(i) / half * log_theta) * 0.15915494309189533576888376337251;
+}
+
+__device__ __forceinline__ void rope_cos_sin(int m, double turns, float &cs, float &sn) {
+    const double t = static_cast<double>(m) * turns;
+    const float fr = static_cast<float>(t - rint(t));      // in [-1/2, 1/2]
+    sincospif(2.0f * fr, &sn, &cs);
+}
+
+// One bf16 pair (x, y) -> (x cs - y sn, x sn + y cs), rounded to bf16; the
+// operation order is fixed so that every caller rounds alike.
+__device__ __forceinline__ uint32_t rope_rotate_pair(uint32_t w, float cs, float sn) {
+    const float2 a = bf16x2_to_float2(w);
+    return pack_bf16x2(__fmaf_rn(a.x, cs, -__fmul_rn(a.y, sn)),
+                       __fmaf_rn(a.x, sn, __fmul_rn(a.y, cs)));
 }
 
 __device__ __forceinline__ void named_barrier_sync(int id, int nthreads) {

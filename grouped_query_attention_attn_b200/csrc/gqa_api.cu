@@ -14,22 +14,65 @@ namespace gqa {
 // First error any kernel of the library recorded on this device (GQA_OK when none).
 __device__ int g_device_status = 0;
 
-int *device_status_ptr() {
-    static int *cache[64] = {};
-    static std::mutex mu;
+using CtxGetCurrentFn = CUresult (*)(CUcontext *);
+using CtxGetIdFn = CUresult (*)(CUcontext, unsigned long long *);
+
+template <class Fn>
+static Fn driver_fn(const char *name) {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint(name, &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+        return reinterpret_cast<Fn>(p);
+    return nullptr;
+}
+
+int current_ctx_key(int *dev, unsigned long long *ctx_id) {
+    static CtxGetCurrentFn get_current = nullptr;
+    static CtxGetIdFn get_id = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        get_current = driver_fn<CtxGetCurrentFn>("cuCtxGetCurrent");
+        get_id = driver_fn<CtxGetIdFn>("cuCtxGetId");
+    });
+    if (int rc = check_cuda(cudaGetDevice(dev), "cudaGetDevice")) return rc;
+    if (*dev < 0 || *dev >= kMaxDevices)
+        return set_error(GQA_ERR_UNSUPPORTED, "device ordinal %d >= %d", *dev, kMaxDevices);
+    *ctx_id = 0;
+    if (!get_current || !get_id) return GQA_OK;
+    CUcontext ctx = nullptr;
+    if (get_current(&ctx) == CUDA_SUCCESS && !ctx) {
+        // no context yet (first call, or after cudaDeviceReset): cudaSetDevice
+        // makes the device's primary context current
+        if (int rc = check_cuda(cudaSetDevice(*dev), "cudaSetDevice")) return rc;
+        get_current(&ctx);
+    }
+    unsigned long long id = 0;
+    if (ctx && get_id(ctx, &id) == CUDA_SUCCESS) *ctx_id = id;
+    return GQA_OK;
+}
+
+void *symbol_address(const void *symbol, SymbolSlot &slot, const char *what) {
     int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
-        set_error(GQA_ERR_CUDA, "cudaGetDevice failed");
-        return nullptr;
-    }
-    std::lock_guard<std::mutex> lock(mu);
-    if (!cache[dev]) {
-        void *p = nullptr;
-        if (check_cuda(cudaGetSymbolAddress(&p, g_device_status), "cudaGetSymbolAddress"))
-            return nullptr;
-        cache[dev] = static_cast<int *>(p);
-    }
-    return cache[dev];
+    unsigned long long id = 0;
+    if (current_ctx_key(&dev, &id)) return nullptr;
+    std::lock_guard<std::mutex> lock(slot.ctx.mu);
+    if (id != 0 && slot.ctx.ctx_id[dev] == id && slot.addr[dev]) return slot.addr[dev];
+    void *p = nullptr;
+    if (check_cuda(cudaGetSymbolAddress(&p, symbol), what)) return nullptr;
+    // the lookup may have made the primary context current: key on it
+    int dev2 = 0;
+    unsigned long long id2 = 0;
+    const bool keyed = current_ctx_key(&dev2, &id2) == GQA_OK && dev2 == dev;
+    slot.ctx.ctx_id[dev] = keyed ? id2 : 0;
+    slot.addr[dev] = p;
+    return p;
+}
+
+int *device_status_ptr() {
+    static SymbolSlot slot;
+    return static_cast<int *>(symbol_address(reinterpret_cast<const void *>(&g_device_status),
+                                             slot, "cudaGetSymbolAddress(status)"));
 }
 
 static thread_local char t_last_error[512] = "";
@@ -174,7 +217,8 @@ const char *gqa_last_error(void) { return t_last_error; }
 // Shared by the plain and the sliding-window forward (window = 0: none).
 static int attn_fwd_bf16(const void *q, const void *k, const void *v, void *o, float *lse,
                          int B, int Tq, int Tkv, int Hq, int Hkv, int d, int causal, int window,
-                         int sinks, float scale, gqa_stream_t stream) {
+                         int sinks, float scale, gqa_stream_t stream, float rope_theta = 0.0f,
+                         int q_pos0 = 0) {
     if (int rc = check_fwd_common(B, Tq, Tkv, Hq, Hkv, d, causal, scale)) return rc;
     if (d != 64 && d != 128)
         return set_error(GQA_ERR_UNSUPPORTED, "head dim d=%d: the bf16 path supports 64 and 128", d);
@@ -190,7 +234,13 @@ static int attn_fwd_bf16(const void *q, const void *k, const void *v, void *o, f
     if (int rc = check_ptr(k, 16, "k")) return rc;
     if (int rc = check_ptr(v, 16, "v")) return rc;
     return launch_prefill(q, k, v, o, lse, B, Tq, Tkv, Hq, Hkv, d, causal, window, sinks, scale,
-                          s);
+                          s, 0, 0, rope_theta, q_pos0);
+}
+
+static int check_theta(float theta) {
+    if (!(theta > 0.0f) || !std::isfinite(theta))
+        return set_error(GQA_ERR_INVALID_ARG, "theta=%g must be finite and > 0", (double)theta);
+    return GQA_OK;
 }
 
 int gqa_attn_fwd_host(const void *q_host, const void *k_host, const void *v_host, void *o_host,
@@ -238,6 +288,18 @@ int gqa_attn_fwd_window(const void *q, const void *k, const void *v, void *o, fl
     return attn_fwd_bf16(q, k, v, o, lse, B, Tq, Tkv, Hq, Hkv, d, 1, window, sinks, scale, stream);
 }
 
+int gqa_attn_fwd_rope(const void *q, const void *k, const void *v, void *o, float *lse, int B,
+                      int Tq, int Tkv, int Hq, int Hkv, int d, int causal, float scale, int q_pos0,
+                      float theta, gqa_stream_t stream) {
+    t_last_error[0] = 0;
+    if (int rc = check_theta(theta)) return rc;
+    if (q_pos0 < 0 || static_cast<long long>(q_pos0) + Tq > 0x7fffffffLL)
+        return set_error(GQA_ERR_INVALID_ARG, "q_pos0=%d must be >= 0 and q_pos0 + Tq fit an int",
+                         q_pos0);
+    return attn_fwd_bf16(q, k, v, o, lse, B, Tq, Tkv, Hq, Hkv, d, causal, 0, 0, scale, stream, theta,
+                         q_pos0);
+}
+
 int gqa_attn_fwd(const void *q, const void *k, const void *v, void *o, int B, int Tq, int Tkv,
                  int Hq, int Hkv, int d, int causal, float scale, gqa_stream_t stream) {
     return gqa_attn_fwd_lse(q, k, v, o, nullptr, B, Tq, Tkv, Hq, Hkv, d, causal, scale, stream);
@@ -266,10 +328,13 @@ size_t gqa_decode_workspace_size(int B, int Hq, int Hkv, int d, int Lmax) {
     return decode_workspace_bytes(B, Hq, Hkv, d, Lmax);
 }
 
-static int decode_bf16(const void *q, const void *k_cache, const void *v_cache,
-                       const int32_t *seqlens, void *o, int B, int Hq, int Hkv, int d, int Lmax,
-                       int window, int sinks, float scale, void *workspace,
-                       size_t workspace_bytes, gqa_stream_t stream) {
+} // extern "C"
+
+namespace gqa {
+
+int validate_decode(const void *q, const void *k_cache, const void *v_cache,
+                    const int32_t *seqlens, const void *o, int B, int Hq, int Hkv, int d,
+                    int Lmax, float scale) {
     if (B < 0 || Lmax < 0) return set_error(GQA_ERR_INVALID_ARG, "B=%d, Lmax=%d must be >= 0", B, Lmax);
     if (int rc = check_heads(Hq, Hkv, d)) return rc;
     if (int rc = check_scale(scale)) return rc;
@@ -286,6 +351,20 @@ static int decode_bf16(const void *q, const void *k_cache, const void *v_cache,
         if (int rc = check_ptr(k_cache, 16, "k_cache")) return rc;
         if (int rc = check_ptr(v_cache, 16, "v_cache")) return rc;
     }
+    return GQA_OK;
+}
+
+}  // namespace gqa
+
+extern "C" {
+
+static int decode_bf16(const void *q, const void *k_cache, const void *v_cache,
+                       const int32_t *seqlens, void *o, int B, int Hq, int Hkv, int d, int Lmax,
+                       int window, int sinks, float scale, void *workspace,
+                       size_t workspace_bytes, gqa_stream_t stream, float rope_theta = 0.0f) {
+    if (int rc = validate_decode(q, k_cache, v_cache, seqlens, o, B, Hq, Hkv, d, Lmax, scale))
+        return rc;
+    if (B == 0) return GQA_OK;
     const size_t need = decode_workspace_bytes(B, Hq, Hkv, d, Lmax);
     if (need > 0) {
         if (!workspace) return set_error(GQA_ERR_WORKSPACE, "workspace is NULL (%zu bytes needed)", need);
@@ -297,7 +376,7 @@ static int decode_bf16(const void *q, const void *k_cache, const void *v_cache,
     }
     if (int rc = require_sm100()) return rc;
     return launch_decode(q, k_cache, v_cache, seqlens, o, B, Hq, Hkv, d, Lmax, window, sinks,
-                         scale, workspace, reinterpret_cast<cudaStream_t>(stream));
+                         scale, workspace, reinterpret_cast<cudaStream_t>(stream), rope_theta);
 }
 
 int gqa_decode(const void *q, const void *k_cache, const void *v_cache, const int32_t *seqlens,
@@ -306,6 +385,16 @@ int gqa_decode(const void *q, const void *k_cache, const void *v_cache, const in
     t_last_error[0] = 0;
     return decode_bf16(q, k_cache, v_cache, seqlens, o, B, Hq, Hkv, d, Lmax, 0, 0, scale,
                        workspace, workspace_bytes, stream);
+}
+
+int gqa_decode_rope(const void *q, const void *k_cache, const void *v_cache,
+                    const int32_t *seqlens, void *o, int B, int Hq, int Hkv, int d, int Lmax,
+                    float scale, float theta, void *workspace, size_t workspace_bytes,
+                    gqa_stream_t stream) {
+    t_last_error[0] = 0;
+    if (int rc = check_theta(theta)) return rc;
+    return decode_bf16(q, k_cache, v_cache, seqlens, o, B, Hq, Hkv, d, Lmax, 0, 0, scale,
+                       workspace, workspace_bytes, stream, theta);
 }
 
 int gqa_decode_window(const void *q, const void *k_cache, const void *v_cache,
@@ -400,6 +489,8 @@ int gqa_device_status(int reset) {
     if (status != 0) return set_error(status, "a kernel recorded status %d", status);
     return GQA_OK;
 }
+
+void gqa_set_prefill_grid_cap(int max_ctas) { set_prefill_grid_cap(max_ctas); }
 
 int gqa_selftest_wait_timeout(int timeout_us) {
     t_last_error[0] = 0;

@@ -21,23 +21,25 @@ namespace gqa {
 namespace {
 
 constexpr int kMaxChunks = 16;
-constexpr int kMaxDevices = 64;
 
-// Copy streams and events, created once per device and reused by every call
-// (the enqueue sequence below runs under a lock, so calls from several host
-// threads cannot interleave their event records).
+// Copy streams and events, created once per CUDA context and reused by every
+// call (the enqueue sequence below runs under a lock, so calls from several
+// host threads cannot interleave their event records).  They are created again
+// when another context is current, e.g. after a cudaDeviceReset destroyed them.
 struct PipeRes {
     cudaStream_t up = nullptr, down = nullptr;
     cudaEvent_t ev[2 * kMaxChunks + 2] = {};
+    unsigned long long ctx_id = 0;
     bool ready = false;
 };
 
 std::mutex g_pipe_mu;
 PipeRes g_pipe[kMaxDevices];
 
-int pipe_res(int dev, PipeRes **out) {
+int pipe_res(int dev, unsigned long long ctx_id, PipeRes **out) {
     PipeRes &r = g_pipe[dev];
-    if (!r.ready) {
+    if (!r.ready || (ctx_id != 0 && r.ctx_id != ctx_id)) {
+        r.ready = false;
         if (int rc = check_cuda(cudaStreamCreateWithFlags(&r.up, cudaStreamNonBlocking),
                                 "cudaStreamCreateWithFlags"))
             return rc;
@@ -48,6 +50,10 @@ int pipe_res(int dev, PipeRes **out) {
             if (int rc = check_cuda(cudaEventCreateWithFlags(&e, cudaEventDisableTiming),
                                     "cudaEventCreateWithFlags"))
                 return rc;
+        // key on the context now current (creating a stream may have made it so)
+        int dev2 = 0;
+        unsigned long long id2 = 0;
+        r.ctx_id = (current_ctx_key(&dev2, &id2) == GQA_OK && dev2 == dev) ? id2 : 0;
         r.ready = true;
     }
     *out = &r;
@@ -73,11 +79,11 @@ int launch_fwd_host_pipeline(const void *q_host, const void *k_host, const void 
                              int B, int Tq, int Tkv, int Hq, int Hkv, int d, int causal,
                              float scale, cudaStream_t stream, cudaEvent_t done) {
     int dev = 0;
-    if (int rc = check_cuda(cudaGetDevice(&dev), "cudaGetDevice")) return rc;
-    if (dev < 0 || dev >= kMaxDevices) return set_error(GQA_ERR_UNSUPPORTED, "device %d", dev);
+    unsigned long long ctx_id = 0;
+    if (int rc = current_ctx_key(&dev, &ctx_id)) return rc;
     std::lock_guard<std::mutex> lock(g_pipe_mu);
     PipeRes *r = nullptr;
-    if (int rc = pipe_res(dev, &r)) return rc;
+    if (int rc = pipe_res(dev, ctx_id, &r)) return rc;
 
     // chunks of at least 256 rows, at most kMaxChunks of them
     int rows = (Tq + 7) / 8;

@@ -25,26 +25,31 @@
 // Softmax warps rescale O_k by exp2(m_old - m_new) before the next PV, which
 // is safe because the commit that signals S_k(j) also covers PV_k(j-1).
 #include <cuda_bf16.h>
+#include <atomic>
 #include <climits>
-#include <cstdlib>
+#include <cmath>
 
 #include "device.cuh"
 #include "internal.h"
 
 namespace gqa {
 
+// Upper bound on the persistent grid set by gqa_set_prefill_grid_cap (0: none).
+static std::atomic<int> g_prefill_grid_cap{0};
+
 constexpr int kPfBM = 128;      // rows per M tile
 constexpr int kPfBN = 128;      // keys per K/V tile
-constexpr int kPfThreads = 640;   // 4 warps producer / MMA + 2 x 8 softmax warps
+constexpr int kPfThreads = 384;   // 4 warps producer / MMA + 2 x 4 softmax warps
 constexpr int kPfStages = 2;
-// Register budget per warpgroup (setmaxnreg): 640 threads launch with 96
-// registers each; warpgroup 0 (producer, MMA, two idle warps) drops to 72 and
-// the softmax warpgroups keep 96 (measured: 979 against 947 TFLOP/s at the
-// Llama-3-8B shape; raising the softmax warps to 104 gave 955).
-constexpr int kPfRegsLaunch = 96;
-constexpr int kPfRegsIo = 72;
-constexpr int kPfRegsSoftmax = 96;
-static_assert(4 * 32 * kPfRegsIo + 16 * 32 * kPfRegsSoftmax <= kPfThreads * kPfRegsLaunch,
+// Register budget per warpgroup (setmaxnreg): 384 threads launch with 168
+// registers each; warpgroup 0 (producer, MMA, two idle warps) drops to 104 and
+// each softmax thread, which holds a whole 128-score row, gets 200 (the
+// smallest producer budget that compiles without spills; the sum is the
+// launch budget exactly).
+constexpr int kPfRegsLaunch = 168;
+constexpr int kPfRegsIo = 104;
+constexpr int kPfRegsSoftmax = 200;
+static_assert(4 * 32 * kPfRegsIo + 8 * 32 * kPfRegsSoftmax <= kPfThreads * kPfRegsLaunch,
               "register split");
 constexpr float kRescaleLog2 = 8.0f;  // lazy rescale threshold (log2 units)
 #ifndef GQA_POLY_PER4
@@ -76,6 +81,8 @@ struct PfParams {
     int causal;
     int window, sinks;                // sliding window (0 = none) and sink keys
     float scale_log2;                 // scale * log2(e)
+    int q_pos0;                       // RoPE: query row t sits at position q_pos0 + t
+    double log_theta;                 // RoPE: ln(theta)
     __nv_bfloat16 *o;
     float *lse;
     int *status;
@@ -149,7 +156,9 @@ __device__ __forceinline__ bool pf_unit(const PfParams &p, int i, PfUnit &u) {
 // the current unit's epilogue.  Iteration counters run over all units of the
 // CTA (ring stages and barrier phases), unit counters over units with at
 // least one KV tile.
-template <int D>
+// kRope: warps 2 and 3 rotate each Q tile in shared memory (rotary position
+// embedding) after its TMA copy lands and before the first S product reads it.
+template <int D, bool kRope>
 __global__ void __launch_bounds__(kPfThreads, 1)
 prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                const __grid_constant__ CUtensorMap tm_v, const PfParams p) {
@@ -158,12 +167,9 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     uint8_t *smem = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
     __shared__ uint64_t q_full[2], q_empty[2], k_full[kPfStages], k_empty[kPfStages],
-        v_full[kPfStages], v_empty[kPfStages], s_full[2], p_full[2], o_done[2], o_free[2],
-        mma_drain;
+        v_full[kPfStages], v_empty[kPfStages], s_full[2], p_full[2][2], o_done[2], o_free[2],
+        q_ready[2], mma_drain;
     __shared__ uint32_t tmem_base_sh;
-    // row-max / l exchange between the two warps that share rows:
-    // [exchange parity][tile][half][row]
-    __shared__ float xchg[2][2][2][kPfBM];
     __shared__ int abort_flag;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -179,9 +185,11 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             mbar_init(&q_full[k], 1);
             mbar_init(&q_empty[k], 1);
             mbar_init(&s_full[k], 1);
-            mbar_init(&p_full[k], 8);   // every softmax warp of the tile
+            mbar_init(&p_full[k][0], 4);   // every softmax warp of the tile, per key half
+            mbar_init(&p_full[k][1], 4);
             mbar_init(&o_done[k], 1);
-            mbar_init(&o_free[k], 8);
+            mbar_init(&o_free[k], 4);
+            mbar_init(&q_ready[k], 2);     // the two rotating warps (kRope only)
         }
         mbar_init(&mma_drain, 1);
         abort_flag = 0;
@@ -306,14 +314,15 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             }
             __syncwarp();
         };
-        // O_k (+)= P_k V_st : P from tensor memory, V MN-major (d contiguous)
-        auto issue_pv = [&](int k, int st, bool acc) {
+        // O_k (+)= P_k V_st over the keys of half `hf` (64 keys): P from tensor
+        // memory, V MN-major (d contiguous)
+        auto issue_pv = [&](int k, int st, int hf, bool acc) {
             const uint32_t ts = tmem + (k ? Lay::kColS1 : Lay::kColS0);
             const uint32_t to = tmem + (k ? Lay::kColO1 : Lay::kColO0);
             const uint64_t bv = st ? dv1 : dv0;
             if (leader) {
 #pragma unroll
-                for (int kk = 0; kk < kPfBN / 16; ++kk)
+                for (int kk = hf * (kPfBN / 32); kk < (hf + 1) * (kPfBN / 32); ++kk)
                     umma_ts(to, ts + kk * 8, bv + kk * (2048 >> 4), idesc_o,
                             (acc || kk > 0) ? 1u : 0u);
             }
@@ -330,11 +339,16 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         // overwrites O_k) the previous unit's epilogue read of O_k.
         int pv_st = 0, pv_j = 0, pv_n = 0, pv_ui = 0, pv_gi = 0;
         bool pv_pending = false;
+        // The softmax releases P_k in two key halves, so the first half's PV
+        // runs while the second half's exponentials are computed.
         auto pv_step = [&](int k) {
-            if (!wait_all(&p_full[k], pv_gi & 1)) return false;
+            if (!wait_all(&p_full[k][0], pv_gi & 1)) return false;
             if (pv_j == 0 && pv_ui > 0 && !wait_all(&o_free[k], (pv_ui - 1) & 1)) return false;
             tc_fence_after();
-            issue_pv(k, pv_st, pv_j > 0);
+            issue_pv(k, pv_st, 0, pv_j > 0);
+            if (!wait_all(&p_full[k][1], pv_gi & 1)) return false;
+            tc_fence_after();
+            issue_pv(k, pv_st, 1, true);
             if (pv_j == pv_n - 1) commit(&o_done[k]);
             return true;
         };
@@ -356,7 +370,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                     commit(&v_empty[pv_st]);
                     pv_pending = false;
                 }
-                if (j == 0 && !(ok = wait_all(&q_full[0], ui & 1))) break;
+                if (j == 0 && !(ok = wait_all(kRope ? &q_ready[0] : &q_full[0], ui & 1))) break;
                 tc_fence_after();
                 issue_s(0, st);
                 commit(&s_full[0]);
@@ -365,7 +379,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                     if (!(ok = pv_step(1))) break;
                     commit(&v_empty[pv_st]);
                 }
-                if (j == 0 && !(ok = wait_all(&q_full[1], ui & 1))) break;
+                if (j == 0 && !(ok = wait_all(kRope ? &q_ready[1] : &q_full[1], ui & 1))) break;
                 tc_fence_after();
                 issue_s(1, st);
                 commit(&s_full[1]);
@@ -388,37 +402,61 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         // every MMA this warp issued has finished before tensor memory is freed
         commit(&mma_drain);
         mbar_wait(&mma_drain, 0, &abort_flag, p.status, 1000000000ull);
+    } else if (kRope) {
+        // -------------------------------------------- Q rotation (RoPE) ----
+        // Thread i of warps 2-3 owns coordinate pair i (columns 2i, 2i+1) of
+        // every row of the tile: one cosine / sine per position, applied to the
+        // G rows (heads) of that position.  Pairs never straddle a 16-byte
+        // chunk, so the 128-byte swizzle only moves whole pairs; a warp touches
+        // one 128-byte row of one panel at a time (no bank conflicts).
+        const int i = (warp - 2) * 32 + lane;
+        const bool active = i < D / 2;
+        const double turns = active ? rope_turns(i, D / 2, p.log_theta) : 0.0;
+        const int panel = (2 * i) / 64, chunk = ((2 * i) % 64) / 8, word = ((2 * i) % 8) / 2;
+        int ui = 0;
+        bool ok = true;
+        PfUnit u;
+        for (int it = 0; ok && pf_unit(p, it, u); ++it) {
+            if (u.n_kv == 0) continue;
+            for (int k = 0; k < 2; ++k) {
+                ok = __all_sync(0xffffffffu, mbar_wait(&q_full[k], ui & 1, &abort_flag, p.status));
+                if (!ok) break;
+                if (active) {
+                    uint8_t *tile = sQ + k * Lay::kQTile + panel * Lay::kQPanel;
+                    const int first = u.t0 + k * p.P;            // position of the tile's row 0
+                    const int n_pos = min(p.P, p.Tq - first);    // rows past Tq are zero fill
+                    for (int pl = 0; pl < n_pos; ++pl) {
+                        float cs, sn;
+                        rope_cos_sin(p.q_pos0 + first + pl, turns, cs, sn);
+                        for (int g = 0; g < p.G; ++g) {
+                            const int r = pl * p.G + g;
+                            uint32_t *w = reinterpret_cast<uint32_t *>(
+                                tile + r * 128 + ((chunk ^ (r & 7)) << 4) + word * 4);
+                            *w = rope_rotate_pair(*w, cs, sn);
+                        }
+                    }
+                }
+                // the tensor core reads the tile through the async proxy
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&q_ready[k]);
+            }
+            ++ui;
+        }
     }
     } else {
         regs_inc<kPfRegsSoftmax>();      // marks the softmax code's budget for the compiler
         // -------------------------------------------- softmax + epilogue ----
-        // Two threads per row: warps 4-11 serve M tile 0, warps 12-19 M tile 1;
-        // within a tile, half h = 0 owns S/O columns 0-63 and h = 1 columns
-        // 64-127 of the 32 rows of tensor-memory lane group (warp % 4).
-        const int k = (warp - 4) >> 3;                  // M tile
-        const int h = ((warp - 4) >> 2) & 1;            // column half
+        // One thread per row: warps 4-7 serve M tile 0, warps 8-11 M tile 1;
+        // warp w reads tensor-memory lanes 32 (w % 4) .. 32 (w % 4) + 31, and
+        // each thread holds all 128 scores of its row, so the row max needs no
+        // exchange between threads.
+        const int k = (warp - 4) >> 2;                  // M tile
         const int g4 = warp & 3;                        // lane group = SM sub-partition
         const int r = (g4 << 5) + lane;                 // row = tensor-memory lane
         const uint32_t lane_addr = tmem + ((static_cast<uint32_t>(g4) * 32u) << 16);
-        const uint32_t colS = (k ? Lay::kColS1 : Lay::kColS0) + 64u * h;
-        const uint32_t colP = (k ? Lay::kColS1 : Lay::kColS0) + 32u * h;
-        const uint32_t colO = (k ? Lay::kColO1 : Lay::kColO0) + (D / 2) * h;
-        const int bar_id = 1 + k * 4 + g4;              // the two warps sharing these rows
-        // Publish a value for my row and take the other half's.  Both warps of
-        // the pair make the same sequence of exchanges (every continue / abort
-        // decision is taken jointly from exchanged values), so the hardware
-        // barrier always completes.  Slots alternate by exchange so a fast
-        // warp cannot overwrite a value its partner has not read yet.
-        int xc = 0;
-        auto exchange = [&](float mine, float &other) {
-            const int slot = xc & 1;
-            ++xc;
-            xchg[slot][k][h][r] = mine;
-            named_barrier_sync(bar_id, 64);
-            other = xchg[slot][k][h ^ 1][r];
-        };
-        const float kAbortMark = __int_as_float(0x7fc00001);   // a NaN no max can produce
-        auto is_abort = [](float x) { return __float_as_int(x) == 0x7fc00001; };
+        const uint32_t colS = k ? Lay::kColS1 : Lay::kColS0;
+        const uint32_t colO = k ? Lay::kColO1 : Lay::kColO0;
         const float c2 = p.scale_log2;
         const int n_sinks = p.window > 0 ? p.sinks : 0;
         int gi = 0, ui = 0;
@@ -429,16 +467,16 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             const int head = u.kvh * p.G + r % p.G;
             const bool row_real = (r < p.P * p.G) && (pos < p.Tq);
             __nv_bfloat16 *dst =
-                p.o + ((static_cast<size_t>(u.b) * p.tq_pitch + pos) * p.Hq + head) * D + (D / 2) * h;
+                p.o + ((static_cast<size_t>(u.b) * p.tq_pitch + pos) * p.Hq + head) * D;
             float *lse_dst = p.lse ? p.lse + (static_cast<size_t>(u.b) * p.Hq + head) * p.Tq + pos
                                    : nullptr;
             if (u.n_kv == 0) {
                 // no visible key for any row of the unit: o = 0, lse = -inf
                 if (row_real) {
 #pragma unroll
-                    for (int e = 0; e < D / 16; ++e)
+                    for (int e = 0; e < D / 8; ++e)
                         reinterpret_cast<uint4 *>(dst)[e] = make_uint4(0u, 0u, 0u, 0u);
-                    if (lse_dst && h == 0) *lse_dst = -INFINITY;
+                    if (lse_dst) *lse_dst = -INFINITY;
                 }
                 continue;
             }
@@ -449,31 +487,26 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             const int lo =
                 (p.window > 0 && row_real) ? pos + (p.Tkv - p.Tq) - p.window + 1 : INT_MIN;
             // Online softmax with a lazily moved reference max: O and l stay
-            // scaled by exp2(-m_ref) and m_ref only moves when a row's max
+            // scaled by exp2(-m_ref) and m_ref only moves when the row's max
             // exceeds it by more than kRescaleLog2 (P then stays <=
             // 2^kRescaleLog2).  Exact in real arithmetic: the epilogue divides
-            // by l taken at the same m_ref.  Both halves of a row see the same
-            // row max, so they take identical m_ref / alpha decisions; each
-            // keeps the partial l of its columns.
+            // by l taken at the same m_ref.
             float m_ref = -INFINITY, l_run = 0.0f;
             for (int j = 0; j < u.n_kv; ++j, ++gi) {
                 // warp-uniform outcome: the tensor-memory accesses below are .sync.aligned
                 ok = __all_sync(0xffffffffu, mbar_wait(&s_full[k], gi & 1, &abort_flag, p.status));
-                if (!ok) {
-                    float dummy;
-                    exchange(kAbortMark, dummy);    // tell the partner
-                    break;
-                }
+                if (!ok) break;
                 tc_fence_after();
-                uint32_t sr[2][32];
-                tmem_ld64(lane_addr + colS, sr[0], sr[1]);     // one instruction, 64 columns
+                uint32_t sr[4][32];
+                tmem_ld64(lane_addr + colS, sr[0], sr[1]);
+                tmem_ld64(lane_addr + colS + 64, sr[2], sr[3]);
                 tmem_wait_ld();
-                const int key0 = u.tile(j) * kPfBN + 64 * h;   // key of my first column
+                const int key0 = u.tile(j) * kPfBN;             // key of column 0
                 const bool masked = __any_sync(
-                    0xffffffffu, key0 + 63 > lim || (key0 < lo && key0 + 63 >= n_sinks));
+                    0xffffffffu, key0 + kPfBN - 1 > lim || (key0 < lo && key0 + kPfBN - 1 >= n_sinks));
                 if (masked) {
 #pragma unroll
-                    for (int c = 0; c < 2; ++c)
+                    for (int c = 0; c < 4; ++c)
 #pragma unroll
                         for (int e = 0; e < 32; ++e) {
                             const int key = key0 + 32 * c + e;
@@ -481,108 +514,93 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                                 sr[c][e] = __float_as_uint(-INFINITY);
                         }
                 }
-                // row max of the raw scores (scale > 0 keeps the order), then
-                // the other half's max through shared memory
-                float mx4[4];
+                // row max of the raw scores (scale > 0 keeps the order):
+                // 8 independent chains of 16 scores
+                float mx8[8];
 #pragma unroll
-                for (int c = 0; c < 4; ++c) {            // 4 independent chains of 16 scores
+                for (int c = 0; c < 8; ++c) {
                     const uint32_t *v = &sr[c >> 1][(c & 1) * 16];
                     float m = __uint_as_float(v[0]);
 #pragma unroll
                     for (int e = 1; e < 15; e += 2)
                         m = max3f(m, __uint_as_float(v[e]), __uint_as_float(v[e + 1]));
-                    mx4[c] = fmaxf(m, __uint_as_float(v[15]));
+                    mx8[c] = fmaxf(m, __uint_as_float(v[15]));
                 }
-                const float mx_mine = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
-                float mx_other;
-                tc_fence_before();                      // my S loads precede the other half's P stores
-                exchange(mx_mine, mx_other);
-                tc_fence_after();
-                if (__any_sync(0xffffffffu, is_abort(mx_other))) {
-                    ok = false;
-                    break;
-                }
-                const float mxs = fmaxf(mx_mine, mx_other) * c2;
+                const float mxs = max3f(max3f(mx8[0], mx8[1], mx8[2]), max3f(mx8[3], mx8[4], mx8[5]),
+                                        fmaxf(mx8[6], mx8[7])) * c2;
                 const bool move = mxs > m_ref + kRescaleLog2;  // always true on the first key seen
                 float alpha = 1.0f;
                 if (move) {
                     alpha = fast_exp2(m_ref - mxs);     // 0 when nothing was seen before
                     m_ref = mxs;
                 }
-                const float m_use = (m_ref == -INFINITY) ? 0.0f : m_ref;
-                const float2 cc = make_float2(c2, c2), nm = make_float2(-m_use, -m_use);
-                float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-                // P = exp2(s * scale * log2e - m_ref), truncated to bf16; P
-                // overwrites the first 64 columns of S (this half: packed
-                // columns 32h..32h+31).  l sums exactly the bf16 weights the PV
-                // product uses, so O / l is a convex combination of V rows.
-                // Tiles with masked (-inf) scores use the MUFU exp only; full
-                // tiles send part of the pairs to the FMA-pipe polynomial.
-                if (masked) {
-#pragma unroll
-                    for (int c = 0; c < 2; ++c) {
-                        uint32_t pk[16];
-                        softmax_chunk<false>(sr[c], cc, nm, pk, acc);
-                        tmem_st16(lane_addr + colP + 16 * c, pk);
-                    }
-                } else {
-#pragma unroll
-                    for (int c = 0; c < 2; ++c) {
-                        uint32_t pk[16];
-                        softmax_chunk<true>(sr[c], cc, nm, pk, acc);
-                        tmem_st16(lane_addr + colP + 16 * c, pk);
-                    }
-                }
-                l_run = l_run * alpha + ((acc[0] + acc[1]) + (acc[2] + acc[3]));
-                // O holds tiles < j at the old reference: rescale rows whose reference moved
+                // O holds tiles < j at the old reference: rescale rows whose
+                // reference moved, before this tile's first PV half is released
                 if (j > 0 && __any_sync(0xffffffffu, move)) {
                     const float2 a2 = make_float2(alpha, alpha);
-#pragma unroll
-                    for (int c = 0; c < D / 64; ++c) {
-                        uint32_t orr[32];
-                        tmem_ld32(lane_addr + colO + 32 * c, orr);
+                    // 16 columns at a time: the row's 128 scores stay live meanwhile
+#pragma unroll 1
+                    for (int c = 0; c < D / 16; ++c) {
+                        uint32_t orr[16];
+                        tmem_ld16(lane_addr + colO + 16 * c, orr);
                         tmem_wait_ld();
 #pragma unroll
-                        for (int e = 0; e < 32; e += 2) {
+                        for (int e = 0; e < 16; e += 2) {
                             const float2 v2 = mul2(make_float2(__uint_as_float(orr[e]),
                                                                __uint_as_float(orr[e + 1])), a2);
                             orr[e] = __float_as_uint(v2.x);
                             orr[e + 1] = __float_as_uint(v2.y);
                         }
-                        tmem_st32(lane_addr + colO + 32 * c, orr);
+                        tmem_st16(lane_addr + colO + 16 * c, orr);
                     }
                 }
-                tmem_wait_st();
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&p_full[k]);
+                const float m_use = (m_ref == -INFINITY) ? 0.0f : m_ref;
+                const float2 cc = make_float2(c2, c2), nm = make_float2(-m_use, -m_use);
+                float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+                // P = exp2(s * scale * log2e - m_ref), truncated to bf16; P
+                // overwrites the first 64 columns of S (keys 2c, 2c + 1 in packed
+                // column c).  l sums exactly the bf16 weights the PV product
+                // uses, so O / l is a convex combination of V rows.  Tiles with
+                // masked (-inf) scores use the MUFU exp only; full tiles send part
+                // of the pairs to the FMA-pipe polynomial.  Each half of the keys
+                // is released to the PV product as soon as it is stored.
+#pragma unroll
+                for (int hf = 0; hf < 2; ++hf) {
+#pragma unroll
+                    for (int c = 2 * hf; c < 2 * hf + 2; ++c) {
+                        uint32_t pk[16];
+                        if (masked)
+                            softmax_chunk<false>(sr[c], cc, nm, pk, acc);
+                        else
+                            softmax_chunk<true>(sr[c], cc, nm, pk, acc);
+                        tmem_st16(lane_addr + colS + 16 * c, pk);
+                    }
+                    tmem_wait_st();
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&p_full[k][hf]);
+                }
+                l_run = l_run * alpha + ((acc[0] + acc[1]) + (acc[2] + acc[3]));
             }
             if (!ok) break;
-            // ---- epilogue: O / l -> bf16, lse (each half writes its d/2 columns) ----
+            // ---- epilogue: O / l -> bf16, lse ----
             // O_k is read out of tensor memory, then released to the next
             // unit's first PV before the conversion and the global stores.
-            const bool done = __all_sync(0xffffffffu,
-                                         mbar_wait(&o_done[k], ui & 1, &abort_flag, p.status));
-            float l_other;
-            exchange(done ? l_run : kAbortMark, l_other);
-            if (!done || __any_sync(0xffffffffu, is_abort(l_other))) {
-                ok = false;
-                break;
-            }
+            ok = __all_sync(0xffffffffu, mbar_wait(&o_done[k], ui & 1, &abort_flag, p.status));
+            if (!ok) break;
             tc_fence_after();
-            uint32_t orr[D / 64][32];
+            uint32_t orr[D / 32][32];
 #pragma unroll
-            for (int c = 0; c < D / 64; ++c) tmem_ld32(lane_addr + colO + 32 * c, orr[c]);
+            for (int c = 0; c < D / 32; ++c) tmem_ld32(lane_addr + colO + 32 * c, orr[c]);
             tmem_wait_ld();
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&o_free[k]);
             ++ui;
-            const float l_row = l_run + l_other;
-            const float inv_l = (l_row > 0.0f) ? 1.0f / l_row : 0.0f;
+            const float inv_l = (l_run > 0.0f) ? 1.0f / l_run : 0.0f;
             if (row_real) {
 #pragma unroll
-                for (int c = 0; c < D / 64; ++c) {
+                for (int c = 0; c < D / 32; ++c) {
                     uint4 *d4 = reinterpret_cast<uint4 *>(dst + 32 * c);
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
@@ -594,8 +612,8 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                             pack_bf16x2(__uint_as_float(v[6]) * inv_l, __uint_as_float(v[7]) * inv_l));
                     }
                 }
-                if (lse_dst && h == 0)
-                    *lse_dst = (l_row > 0.0f) ? (m_ref + __log2f(l_row)) * 0.69314718055994531f
+                if (lse_dst)
+                    *lse_dst = (l_run > 0.0f) ? (m_ref + __log2f(l_run)) * 0.69314718055994531f
                                               : -INFINITY;
             }
         }
@@ -610,12 +628,14 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     }
 }
 
-template <int D>
+template <int D, bool kRope>
 static int launch_prefill_d(const void *q, const void *k, const void *v, void *o, float *lse,
                             int B, int Tq, int Tkv, int Hq, int Hkv, int causal, int window,
                             int sinks, float scale, cudaStream_t stream, int tq_pitch,
-                            int tkv_pitch) {
+                            int tkv_pitch, int q_pos0, float theta) {
     PfParams prm;
+    prm.q_pos0 = q_pos0;
+    prm.log_theta = kRope ? log(static_cast<double>(theta)) : 0.0;
     prm.tq_pitch = tq_pitch > 0 ? tq_pitch : Tq;
     prm.window = window;
     prm.sinks = sinks;
@@ -639,11 +659,8 @@ static int launch_prefill_d(const void *q, const void *k, const void *v, void *o
     int n_sm = 0;
     if (int rc = sm_count(&n_sm)) return rc;
     long long blocks = units < n_sm ? units : n_sm;   // persistent: one CTA per SM
-    // GQA_PREFILL_MAX_CTAS caps the grid (tests use it to put many units on each CTA)
-    if (const char *cap = getenv("GQA_PREFILL_MAX_CTAS")) {
-        const long long m = atoll(cap);
-        if (m > 0 && m < blocks) blocks = m;
-    }
+    const int cap = g_prefill_grid_cap.load(std::memory_order_relaxed);
+    if (cap > 0 && cap < blocks) blocks = cap;
 
     CUtensorMap tq, tk, tv;
     const uint64_t kv_pitch = tkv_pitch > 0 ? tkv_pitch : Tkv;
@@ -654,33 +671,50 @@ static int launch_prefill_d(const void *q, const void *k, const void *v, void *o
     if (int rc = encode_tmap_bf16_4d(&tv, v, D, Hkv, Tkv, B, 64, 1, kPfBN, 1, 1, kv_pitch))
         return rc;
 
-    auto kern = prefill_kernel<D>;
-    // the setmaxnreg split adds up only at the launch budget it was sized for:
-    // a build with fewer registers per thread would leave the softmax
-    // warpgroups waiting for registers, so it is refused here
-    cudaFuncAttributes fa;
-    if (int rc = check_cuda(cudaFuncGetAttributes(&fa, kern), "cudaFuncGetAttributes(prefill)"))
-        return rc;
-    if (fa.numRegs != kPfRegsLaunch)
-        return set_error(GQA_ERR_UNSUPPORTED,
-                         "prefill kernel built with %d registers per thread, %d expected",
-                         fa.numRegs, kPfRegsLaunch);
+    auto kern = prefill_kernel<D, kRope>;
     const int smem = PfLayout<D>::kSmemBytes;
-    if (int rc = check_cuda(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                 smem), "cudaFuncSetAttribute(prefill)"))
+    // once per context: the register check and the shared-memory opt-in
+    static CtxSlot setup;
+    if (int rc = once_per_context(setup, [&](int) {
+            // the setmaxnreg split adds up only at the launch budget it was sized
+            // for: a build with fewer registers per thread would leave the softmax
+            // warpgroups waiting for registers, so it is refused here
+            cudaFuncAttributes fa;
+            if (int e = check_cuda(cudaFuncGetAttributes(&fa, kern), "cudaFuncGetAttributes(prefill)"))
+                return e;
+            if (fa.numRegs != kPfRegsLaunch)
+                return set_error(GQA_ERR_UNSUPPORTED,
+                                 "prefill kernel built with %d registers per thread, %d expected",
+                                 fa.numRegs, kPfRegsLaunch);
+            return check_cuda(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                   smem), "cudaFuncSetAttribute(prefill)");
+        }))
         return rc;
     kern<<<static_cast<unsigned>(blocks), kPfThreads, smem, stream>>>(tq, tk, tv, prm);
     return check_cuda(cudaGetLastError(), "prefill_kernel launch");
 }
 
+void set_prefill_grid_cap(int max_ctas) {
+    g_prefill_grid_cap.store(max_ctas > 0 ? max_ctas : 0, std::memory_order_relaxed);
+}
+
 int launch_prefill(const void *q, const void *k, const void *v, void *o, float *lse, int B,
                    int Tq, int Tkv, int Hq, int Hkv, int d, int causal, int window, int sinks,
-                   float scale, cudaStream_t stream, int tq_pitch, int tkv_pitch) {
+                   float scale, cudaStream_t stream, int tq_pitch, int tkv_pitch, float rope_theta,
+                   int q_pos0) {
+    const bool rope = rope_theta > 0.0f;
     if (d == 128)
-        return launch_prefill_d<128>(q, k, v, o, lse, B, Tq, Tkv, Hq, Hkv, causal, window, sinks,
-                                     scale, stream, tq_pitch, tkv_pitch);
-    return launch_prefill_d<64>(q, k, v, o, lse, B, Tq, Tkv, Hq, Hkv, causal, window, sinks,
-                                scale, stream, tq_pitch, tkv_pitch);
+        return rope ? launch_prefill_d<128, true>(q, k, v, o, lse, B, Tq, Tkv, Hq, Hkv, causal,
+                                                  window, sinks, scale, stream, tq_pitch, tkv_pitch,
+                                                  q_pos0, rope_theta)
+                    : launch_prefill_d<128, false>(q, k, v, o, lse, B, Tq, Tkv, Hq, Hkv, causal,
+                                                   window, sinks, scale, stream, tq_pitch,
+                                                   tkv_pitch, 0, 0.0f);
+    return rope ? launch_prefill_d<64, true>(q, k, v, o, lse, B, Tq, Tkv, Hq, Hkv, causal, window,
+                                             sinks, scale, stream, tq_pitch, tkv_pitch, q_pos0,
+                                             rope_theta)
+                : launch_prefill_d<64, false>(q, k, v, o, lse, B, Tq, Tkv, Hq, Hkv, causal, window,
+                                              sinks, scale, stream, tq_pitch, tkv_pitch, 0, 0.0f);
 }
 
 }  // namespace gqa

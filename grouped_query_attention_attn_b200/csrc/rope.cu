@@ -8,9 +8,9 @@
 //     of up to kRopeBatch head rows of one token (a batch: q's heads, then k's,
 //     in groups of kRopeBatch), computes those four sine / cosine pairs and
 //     applies them to that column of every row of the batch;
-//   * the angle m * theta_i reaches ~10^4 rad at long context, so the number of
-//     turns m * theta_i / (2 pi) is formed and reduced to [-1/2, 1/2] in double,
-//     then sincospif gives the fp32 sine and cosine of 2 pi times that fraction;
+//   * the angle and the rotation are device.cuh's rope_cos_sin and
+//     rope_rotate_pair (turns reduced in double, fp32 sine / cosine), shared
+//     with the attention kernels that rotate q as they load it;
 //   * all loads of a batch are issued before any store, and the batches of a
 //     token are spread over threads so that enough loads are in flight.
 #include <cuda_bf16.h>
@@ -24,11 +24,6 @@ constexpr int kRopeMaxHalf = 128;    // d <= 256
 constexpr int kRopeThreads = 256;
 constexpr int kRopeBatch = 8;
 
-__device__ __forceinline__ uint32_t rotate_pair(uint32_t w, float cs, float sn) {
-    const float2 a = bf16x2_to_float2(w);
-    return pack_bf16x2(a.x * cs - a.y * sn, a.x * sn + a.y * cs);
-}
-
 // Rotates column c8 of n (<= kRopeBatch) head rows starting at row0 (rows d8
 // vectors apart).
 __device__ __forceinline__ void rope_rows(uint4 *__restrict__ row0, int n, int d8,
@@ -40,10 +35,10 @@ __device__ __forceinline__ void rope_rows(uint4 *__restrict__ row0, int n, int d
 #pragma unroll
     for (int j = 0; j < kRopeBatch; ++j) {
         if (j < n) {
-            w[j].x = rotate_pair(w[j].x, cs[0], sn[0]);
-            w[j].y = rotate_pair(w[j].y, cs[1], sn[1]);
-            w[j].z = rotate_pair(w[j].z, cs[2], sn[2]);
-            w[j].w = rotate_pair(w[j].w, cs[3], sn[3]);
+            w[j].x = rope_rotate_pair(w[j].x, cs[0], sn[0]);
+            w[j].y = rope_rotate_pair(w[j].y, cs[1], sn[1]);
+            w[j].z = rope_rotate_pair(w[j].z, cs[2], sn[2]);
+            w[j].w = rope_rotate_pair(w[j].w, cs[3], sn[3]);
             row0[static_cast<size_t>(j) * d8] = w[j];
         }
     }
@@ -60,9 +55,7 @@ rope_kernel(uint4 *__restrict__ x0, int H0, uint4 *__restrict__ x1, int H1, long
     __shared__ double turns[kRopeMaxHalf];         // theta_i / (2 pi)
     const int d8 = blockDim.x, half = 4 * d8;
     const int tid = threadIdx.y * d8 + threadIdx.x;
-    for (int i = tid; i < half; i += d8 * blockDim.y)
-        turns[i] = exp(-static_cast<double>(i) / half * log_theta) *
-                   0.15915494309189533576888376337251;
+    for (int i = tid; i < half; i += d8 * blockDim.y) turns[i] = rope_turns(i, half, log_theta);
     __syncthreads();
     const long long w = static_cast<long long>(blockIdx.x) * blockDim.y + threadIdx.y;
     if (w >= n_work) return;
@@ -72,11 +65,7 @@ rope_kernel(uint4 *__restrict__ x0, int H0, uint4 *__restrict__ x1, int H1, long
     const int m = seqlens ? max(seqlens[b] - 1, 0) : pos0 + (tok - b * T);
     float cs[4], sn[4];
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {
-        const double t = static_cast<double>(m) * turns[c8 * 4 + e];
-        const float fr = static_cast<float>(t - rint(t));    // in [-1/2, 1/2]
-        sincospif(2.0f * fr, &sn[e], &cs[e]);
-    }
+    for (int e = 0; e < 4; ++e) rope_cos_sin(m, turns[c8 * 4 + e], cs[e], sn[e]);
     const int b0 = (H0 + kRopeBatch - 1) / kRopeBatch;
     if (bi < b0) {
         const int h = bi * kRopeBatch;

@@ -64,9 +64,9 @@ typedef enum {
  *   (callers normally pass 1/sqrt(d)).  Pointers must be 16-byte aligned
  *   (tensor-memory-access copies need it).
  * The kernel is persistent: min(#work units, #SMs) CTAs, a unit being two
- * 128-row tiles of one (batch, KV head).  If the environment variable
- * GQA_PREFILL_MAX_CTAS holds a positive integer, it caps that grid (read at
- * every launch; the tests use it to put many units on each CTA).
+ * 128-row tiles of one (batch, KV head); gqa_set_prefill_grid_cap can lower
+ * that bound.  Host work per call: argument checks and three tensor-map
+ * encodings; the kernel's attributes are set once per CUDA context.
  */
 int gqa_attn_fwd(const void *q, const void *k, const void *v, void *o,
                  int B, int Tq, int Tkv, int Hq, int Hkv, int d,
@@ -81,6 +81,23 @@ int gqa_attn_fwd(const void *q, const void *k, const void *v, void *o,
 int gqa_attn_fwd_lse(const void *q, const void *k, const void *v, void *o, float *lse,
                      int B, int Tq, int Tkv, int Hq, int Hkv, int d,
                      int causal, float scale, gqa_stream_t stream);
+
+/*
+ * gqa_attn_fwd_rope -- gqa_attn_fwd_lse with rotary position embedding applied
+ * to q as it is loaded (course "Неделя 7. Внимание", step 3: pair (2i, 2i+1)
+ * of the row at position m turns by m * theta^(-2i/d); only q and k rotate).
+ * Query row t sits at position q_pos0 + t (q_pos0 >= 0; for self-attention
+ * over a whole sequence q_pos0 = Tkv - Tq, the key positions being 0..Tkv-1).
+ * q in memory is NOT modified; k must already be rotated (gqa_rope, once,
+ * when the keys enter the cache: a key tile is read by every query tile of
+ * its group, so rotating it on each load would repeat the work).  The
+ * rotation is the same arithmetic as gqa_rope's, so the result equals
+ * gqa_rope(q) followed by gqa_attn_fwd_lse bit for bit.  theta > 0 and
+ * finite; everything else as gqa_attn_fwd_lse.
+ */
+int gqa_attn_fwd_rope(const void *q, const void *k, const void *v, void *o, float *lse,
+                      int B, int Tq, int Tkv, int Hq, int Hkv, int d, int causal, float scale,
+                      int q_pos0, float theta, gqa_stream_t stream);
 
 /*
  * gqa_attn_fwd_host -- gqa_attn_fwd for host-resident tensors (same operation,
@@ -100,8 +117,8 @@ int gqa_attn_fwd_lse(const void *q, const void *k, const void *v, void *o, float
  * copies up after the work on `stream` at the time of the call and its first
  * attention chunk after the previous call's copies down (on this device).
  * The host buffers must stay allocated and unchanged until the call completes.
- * The copy streams and their events are created once per device on first use
- * and kept (no device memory is allocated); concurrent calls from several
+ * The copy streams and their events are created on first use in each CUDA
+ * context and kept (no device memory is allocated); concurrent calls from several
  * host threads are serialised while they enqueue.  Errors as
  * gqa_attn_fwd_lse, plus GQA_ERR_CUDA for a failed copy.
  */
@@ -166,6 +183,19 @@ int gqa_decode(const void *q, const void *k_cache, const void *v_cache,
                void *workspace, size_t workspace_bytes, gqa_stream_t stream);
 
 /*
+ * gqa_decode_rope -- gqa_decode with rotary position embedding applied to the
+ * query as it is loaded (course step 3): sequence b's new token sits at
+ * position max(seqlens[b] - 1, 0), as for gqa_rope_decode_q; q in memory is
+ * not modified and the cached keys must already be rotated.  The result
+ * equals gqa_rope_decode_q followed by gqa_decode bit for bit.  theta > 0 and
+ * finite; everything else (layouts, workspace, errors) as gqa_decode.
+ */
+int gqa_decode_rope(const void *q, const void *k_cache, const void *v_cache,
+                    const int32_t *seqlens, void *o,
+                    int B, int Hq, int Hkv, int d, int Lmax, float scale, float theta,
+                    void *workspace, size_t workspace_bytes, gqa_stream_t stream);
+
+/*
  * gqa_decode_window -- gqa_decode with a sliding window and attention sinks
  * (course step 3): the newest token of sequence b sees cache rows
  * j >= seqlens[b] - window and rows j < sinks.  window >= 1, sinks >= 0;
@@ -199,9 +229,12 @@ int gqa_decode_window(const void *q, const void *k_cache, const void *v_cache,
  *     gqa_decode_workspace_size(...) exceeds it are rejected with
  *     GQA_ERR_WORKSPACE and nothing is launched (B=64, Hq=32, d=128,
  *     Lmax=8192 fits).
- *   - The first call with a given device current looks up the scratch's
- *     device address (cudaGetSymbolAddress) and caches it; make that first
- *     call on each device before any stream capture.
+ *   - The first call in a CUDA context (the first call with a device
+ *     current, and the first one after a cudaDeviceReset of that device)
+ *     looks up the scratch's device address (cudaGetSymbolAddress) and
+ *     caches it for that context; make that first call before any stream
+ *     capture.  Arguments are checked exactly as gqa_decode checks them, and
+ *     before the lookup.
  *   - All calls on a device share the one scratch array, which keeps the last
  *     call's contents.  Nothing in it needs to start at zero, but calls whose
  *     kernels overlap on the GPU (different streams, or several host threads)
@@ -310,6 +343,28 @@ int gqa_device_status(int reset);
  * hanging or faulting the GPU; synchronises the device; resets the record.
  */
 int gqa_selftest_wait_timeout(int timeout_us);
+
+/*
+ * gqa_selftest_exp2_poly -- evaluates, on the GPU, the FMA-pipe 2^x
+ * polynomial the prefill softmax uses for part of its exponentials (the
+ * max-subtracted softmax of TT Lab step 4 / course step 1 needs
+ * exp(s - m) = 2^((s - m) log2 e)): y[i] = poly 2^x[i] for n points (n even,
+ * x and y device float arrays, 4-byte aligned).  Range reduction
+ * x = n + f, f in [-1/2, 1/2], a degree-3 minimax fit of 2^f (relative error
+ * <= 7.5e-5), 2^n added to the exponent field; x is clamped to >= -125
+ * (which keeps every result a normal float), so every x <= -125 gives 2^-125
+ * (to the same relative error).  Asynchronous on `stream`.  For tests of that
+ * bound.
+ */
+int gqa_selftest_exp2_poly(const float *x, float *y, int n, gqa_stream_t stream);
+
+/*
+ * gqa_set_prefill_grid_cap -- testing aid: caps the persistent prefill grid
+ * (gqa_attn_fwd and its variants) at max_ctas CTAs for every later launch in
+ * the process, so each CTA walks many work units; max_ctas <= 0 removes the
+ * cap.  The output does not depend on the grid.  Not needed in normal use.
+ */
+void gqa_set_prefill_grid_cap(int max_ctas);
 
 #ifdef __cplusplus
 }

@@ -204,3 +204,25 @@ def test_backward_rejects(gqa_lib):
     assert bwd(ws_bytes=16) == b.GQA_ERR_WORKSPACE
     assert bwd(B=0) == b.GQA_OK
     assert b.gqa_attn_bwd_workspace_size(2, 100, 8) >= 2 * 100 * 8 * 4
+
+
+def test_fused_rope_entry_points_reject(gqa_lib):
+    # the fused-RoPE forward and decode check theta and the position offset first
+    fwd = dict(q=FAKE, k=FAKE, v=FAKE, o=FAKE, lse=NULL, B=1, Tq=8, Tkv=8, Hq=4, Hkv=2, d=128,
+               causal=1, scale=0.088, q_pos0=0, theta=10000.0)
+
+    def call(**kw):
+        a = dict(fwd)
+        a.update(kw)
+        return b.gqa_attn_fwd_rope(*a.values(), NULL)
+
+    assert call(theta=0.0) == b.GQA_ERR_INVALID_ARG
+    assert call(theta=float("inf")) == b.GQA_ERR_INVALID_ARG
+    assert call(q_pos0=-1) == b.GQA_ERR_INVALID_ARG
+    assert call(Hkv=3) == b.GQA_ERR_INVALID_ARG
+    assert call(d=96) == b.GQA_ERR_UNSUPPORTED
+    assert call(B=0) == b.GQA_OK
+    assert b.gqa_decode_rope(FAKE, FAKE, FAKE, FAKE, FAKE, 4, 8, 2, 128, 100, 0.088, -1.0,
+                             FAKE, 1 << 20, NULL) == b.GQA_ERR_INVALID_ARG
+    assert b.gqa_decode_rope(NULL, FAKE, FAKE, FAKE, FAKE, 4, 8, 2, 128, 100, 0.088, 1e4,
+                             FAKE, 1 << 20, NULL) == b.GQA_ERR_INVALID_ARG

@@ -1,4 +1,4 @@
-"""Split-KV decode + log-sum-exp combine against the double oracle (2e-2 max-abs).
+"""Split-KV decode with the in-kernel log-sum-exp merge of the splits, against the double oracle (2e-2 max-abs).
 
 Cache rows past each sequence's length are NaN, so any read of them poisons
 the output and fails the comparison."""
@@ -74,3 +74,63 @@ def test_undersized_workspace_rejected(gqa_lib):
     ws = torch.empty(need - 256, dtype=torch.uint8, device="cuda")
     with pytest.raises(ValueError):
         gqa.decode(q.cuda(), kc.cuda(), vc.cuda(), sl.cuda(), workspace=ws)
+
+
+# ---- the in-kernel merge: arrival words in the workspace --------------------
+
+def test_workspace_garbage_and_reuse_across_shapes(gqa_lib):
+    # The last split of each (sequence, KV head) is found with an arrival word
+    # in the workspace.  Neither leftover words of other calls (other shapes,
+    # other splits counts) nor arbitrary bytes on entry may change the result.
+    cases = [(8, 32, 8, 128, 3000, [3000, 1, 2048, 0, 1025, 513, 2999, 64]),
+             (5, 8, 2, 64, 1100, [1100, 700, 0, 1, 1024]),
+             (3, 32, 1, 128, 5000, [4097, 5000, 1])]
+    need = max(gqa.decode_workspace_size(B, Hq, Hkv, d, L) for B, Hq, Hkv, d, L, _ in cases)
+    ws = torch.full((need,), 0xFF, dtype=torch.uint8, device="cuda")
+    for rep in range(2):
+        for i, (B, Hq, Hkv, d, Lmax, lengths) in enumerate(cases):
+            q, kc, vc, sl = workloads.decode_inputs(B, Hq, Hkv, d, 1, Lmax, lengths=lengths,
+                                                    seeds=(50 + i, 60 + i, 70 + i, 0))
+            o_ref, _ = ref.decode(q, kc, vc, sl)
+            o = gqa.decode(q.cuda(), kc.cuda(), vc.cuda(), sl.cuda(), workspace=ws)
+            gqa.device_status()
+            assert max_abs(o, o_ref) <= BF16_TOL, (rep, i)
+        if rep == 0:
+            ws.random_(0, 256)                   # arbitrary bytes before the second round
+
+
+def test_cuda_graph_replays_of_one_launch(gqa_lib):
+    # A captured launch replays with the same call id; the merging split leaves
+    # the word counting from zero, so every replay merges correctly.
+    B, Hq, Hkv, d, Lmax = 6, 32, 8, 128, 2100
+    lengths = [2100, 1, 1024, 1025, 0, 2048]
+    q, kc, vc, sl = workloads.decode_inputs(B, Hq, Hkv, d, 1, Lmax, lengths=lengths)
+    qd, kd, vd, sd = q.cuda(), kc.cuda(), vc.cuda(), sl.cuda()
+    ws = torch.empty(gqa.decode_workspace_size(B, Hq, Hkv, d, Lmax), dtype=torch.uint8,
+                     device="cuda")
+    o = torch.empty_like(qd)
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        gqa.decode(qd, kd, vd, sd, workspace=ws, out=o)          # warm-up outside capture
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=s):
+            gqa.decode(qd, kd, vd, sd, workspace=ws, out=o)
+    for rep in range(3):
+        qn = workloads.randn((B, Hq, d), 900 + rep)
+        qd.copy_(qn)
+        o.fill_(float("nan"))
+        g.replay()
+        torch.cuda.synchronize()
+        o_ref, _ = ref.decode(qn, kc, vc, sl)
+        assert max_abs(o, o_ref) <= BF16_TOL, rep
+    gqa.device_status()
+
+
+def test_empty_cache_gives_zeros(gqa_lib):
+    q = workloads.randn((3, 8, 128), 5).cuda()
+    kc = torch.empty((3, 0, 2, 128), dtype=torch.bfloat16, device="cuda")
+    sl = torch.zeros(3, dtype=torch.int32, device="cuda")
+    o = gqa.decode(q, kc, kc.clone(), sl)
+    gqa.device_status()
+    assert torch.all(o == 0)

@@ -79,3 +79,70 @@ def test_rope_qk_headline_shape(gqa_lib):
         want = ref.rope_tensor(x, 0)
         rel = np.abs(got.float().cpu().numpy() - want) / np.maximum(np.abs(want), 1e-30)
         assert np.max(np.where(np.abs(want) > 1e-3, rel, 0.0)) <= 2.0 ** -8
+
+
+# ---- RoPE fused into the attention kernels' loads ---------------------------
+
+FUSED_PREFILL = [
+    # B, Tq, Tkv, Hq, Hkv, d, causal, q_pos0 (None: Tkv - Tq)
+    (1, 500, 500, 8, 2, 128, True, None),
+    (2, 300, 300, 32, 8, 128, True, None),
+    (1, 200, 700, 8, 1, 64, True, None),          # chunk of a longer sequence
+    (1, 129, 129, 4, 4, 128, False, 0),           # MHA: one position per row
+    (1, 260, 260, 32, 1, 128, True, 1000),        # MQA, offset positions
+    (1, 100, 100, 6, 2, 64, True, 31000),         # G = 3 (ragged M tile), long positions
+]
+
+
+@pytest.mark.parametrize("B,Tq,Tkv,Hq,Hkv,d,causal,q_pos0", FUSED_PREFILL)
+def test_fused_rope_prefill(gqa_lib, B, Tq, Tkv, Hq, Hkv, d, causal, q_pos0):
+    # q rotated as each tile is loaded equals rotating q first (the same bits),
+    # and both match the oracle's rotation + attention
+    q, k, v = workloads.prefill_inputs(B, Tq, Hq, Hkv, d, Tkv=Tkv, seeds=(Tq, Tkv, Hq + d))
+    pos0 = Tkv - Tq if q_pos0 is None else q_pos0
+    kr = gqa.rope_(k.cuda(), 0)                           # keys at positions 0..Tkv-1
+    qd = q.cuda()
+    o, lse = gqa.attn(qd, kr, v.cuda(), causal=causal, return_lse=True, rope_theta=10000.0,
+                      q_pos0=pos0)
+    gqa.device_status()
+    assert torch.equal(qd.cpu(), q)                       # q in memory is not modified
+    o2, lse2 = gqa.attn(gqa.rope_(q.cuda(), pos0), kr, v.cuda(), causal=causal, return_lse=True)
+    assert torch.equal(o, o2) and torch.equal(lse, lse2)
+    qr = bf16_round(ref.rope_tensor(q, pos0))
+    kro = bf16_round(ref.rope_tensor(k, 0))
+    o_ref, lse_ref = ref.attn_fwd(qr, kro, v, causal=causal)
+    assert max_abs(o, o_ref) <= BF16_TOL
+    l = lse.cpu().numpy().astype(np.float64)
+    fin = np.isfinite(lse_ref)
+    assert np.array_equal(np.isneginf(l), ~fin)
+    assert np.max(np.abs(l[fin] - lse_ref[fin]), initial=0.0) <= BF16_TOL
+
+
+def test_fused_rope_prefill_headline_shape(gqa_lib):
+    # the B=1, T=4096, 32 / 8 head workload: fused rotation of q against rotating
+    # first (bit for bit) and against the oracle on every row
+    q, k, v = workloads.prefill_inputs(1, 4096, 32, 8, 128)
+    kr = gqa.rope_(k.cuda(), 0)
+    o, lse = gqa.attn(q.cuda(), kr, v.cuda(), causal=True, return_lse=True, rope_theta=10000.0)
+    gqa.device_status()
+    qg = gqa.rope_(q.cuda(), 0)
+    o2 = gqa.attn(qg, kr, v.cuda(), causal=True)
+    assert torch.equal(o, o2)
+    o_ref, lse_ref = ref.attn_fwd(qg.cpu(), kr.cpu(), v, causal=True)
+    assert max_abs(o, o_ref) <= BF16_TOL
+    assert np.max(np.abs(lse.cpu().numpy() - lse_ref)) <= BF16_TOL
+
+
+@pytest.mark.parametrize("Hq,Hkv,d", [(32, 8, 128), (8, 1, 64), (32, 1, 128)])
+def test_fused_rope_decode(gqa_lib, Hq, Hkv, d):
+    lengths = [1, 700, 0, 1025, 3000, 64]
+    q, kc, vc, sl = workloads.decode_inputs(len(lengths), Hq, Hkv, d, 1, 3000, lengths=lengths,
+                                            seeds=(Hq, Hkv, d, 0))
+    qd = q.cuda()
+    o = gqa.decode(qd, kc.cuda(), vc.cuda(), sl.cuda(), rope_theta=10000.0)
+    gqa.device_status()
+    assert torch.equal(qd.cpu(), q)
+    o2 = gqa.decode(gqa.rope_decode_q_(q.cuda(), sl.cuda()), kc.cuda(), vc.cuda(), sl.cuda())
+    assert torch.equal(o, o2)
+    o_ref, _ = ref.decode(bf16_round(ref.rope_decode_q(q, sl)), kc, vc, sl)
+    assert max_abs(o, o_ref) <= BF16_TOL

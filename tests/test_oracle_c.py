@@ -250,6 +250,24 @@ def test_fold_tensor_matches_lab_fold():
                 assert torch.equal(out[b, t], want)
 
 
+@pytest.mark.parametrize("g", [8, 1])
+def test_fold_tensor_matches_lab_mean_at_the_sweep_folds(g):
+    # The head-sharing sweep folds its 32-head K and V to 8 and to 1 heads.  On
+    # positions of those very tensors, the oracle's float32 fold (head order,
+    # then one rounding to bf16) equals the lab's double mean rounded to bf16,
+    # element for element (TT Lab step 2).
+    _, k32, v32 = workloads.prefill_inputs(4, 2048, 32, 32, 128)
+    pos = np.random.default_rng(g).choice(2048, size=16, replace=False)
+    for kv in (k32, v32):
+        block = kv[:, pos]                                   # [4, 16, 32, 128]
+        out = ref.fold_kv_tensor(block, g)
+        rows = block.double().reshape(64, 32, 128)          # (b, t) pairs as rows
+        heads = [rows[:, h].tolist() for h in range(32)]     # [head][row][col]
+        want = torch.tensor(lab.fold_kv(heads, g), dtype=torch.float64)   # [g][row][col]
+        want = want.permute(1, 0, 2).reshape(4, 16, g, 128).to(torch.bfloat16)
+        assert torch.equal(out, want)
+
+
 def test_fold_tensor_identity_and_errors():
     kv = workloads.randn((1, 3, 4, 8), 34)
     assert torch.equal(ref.fold_kv_tensor(kv, 4), kv)
