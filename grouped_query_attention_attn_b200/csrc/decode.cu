@@ -383,18 +383,40 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tm_k,
     __threadfence();                                 // every split's partial rows are visible
     const size_t plane = static_cast<size_t>(B) * Hq;
     const size_t grow0 = static_cast<size_t>(b) * Hq + static_cast<size_t>(kvh) * G;
+    // Batches of 8 splits keep their loads in flight together (the partial
+    // rows sit in L2); the running max is taken first, then the sums.
+    constexpr int kBatch = 8;
     for (int idx = threadIdx.x; idx < G * D / 2; idx += kDecWarps * 32) {
         const int r = idx / (D / 2), c = (idx % (D / 2)) * 2;
+        const float *lse_r = part_lse + grow0 + r;
+        const float *o_r = part_o + (grow0 + r) * D + c;
         float M = -INFINITY;
-        for (int sp = 0; sp < n_splits; ++sp) M = fmaxf(M, __ldcg(part_lse + sp * plane + grow0 + r));
+        for (int sp0 = 0; sp0 < n_splits; sp0 += kBatch) {
+            float l[kBatch];
+#pragma unroll
+            for (int e = 0; e < kBatch; ++e)
+                l[e] = sp0 + e < n_splits ? __ldcg(lse_r + (sp0 + e) * plane) : -INFINITY;
+#pragma unroll
+            for (int e = 0; e < kBatch; ++e) M = fmaxf(M, l[e]);
+        }
         float wsum = 0.0f, a0 = 0.0f, a1 = 0.0f;
-        for (int sp = 0; sp < n_splits; ++sp) {
-            const float w = __expf(__ldcg(part_lse + sp * plane + grow0 + r) - M);
-            const float2 v = __ldcg(reinterpret_cast<const float2 *>(
-                part_o + (sp * plane + grow0 + r) * D + c));
-            wsum += w;
-            a0 += w * v.x;
-            a1 += w * v.y;
+        for (int sp0 = 0; sp0 < n_splits; sp0 += kBatch) {
+            float l[kBatch];
+            float2 v[kBatch];
+#pragma unroll
+            for (int e = 0; e < kBatch; ++e) {
+                const bool in = sp0 + e < n_splits;
+                l[e] = in ? __ldcg(lse_r + (sp0 + e) * plane) : -INFINITY;
+                v[e] = in ? __ldcg(reinterpret_cast<const float2 *>(o_r + (sp0 + e) * plane * D))
+                          : make_float2(0.0f, 0.0f);
+            }
+#pragma unroll
+            for (int e = 0; e < kBatch; ++e) {
+                const float w = __expf(l[e] - M);          // 0 for the padding entries
+                wsum += w;
+                a0 += w * v[e].x;
+                a1 += w * v[e].y;
+            }
         }
         const float inv = 1.0f / wsum;
         *reinterpret_cast<__nv_bfloat162 *>(o + (grow0 + r) * D + c) =

@@ -39,17 +39,18 @@ static std::atomic<int> g_prefill_grid_cap{0};
 
 constexpr int kPfBM = 128;      // rows per M tile
 constexpr int kPfBN = 128;      // keys per K/V tile
-constexpr int kPfThreads = 384;   // 4 warps producer / MMA + 2 x 4 softmax warps
+constexpr int kPfThreads = 640;   // 4 warps producer / MMA + 2 x 8 softmax warps
 constexpr int kPfStages = 2;
-// Register budget per warpgroup (setmaxnreg): 384 threads launch with 168
-// registers each; warpgroup 0 (producer, MMA, two idle warps) drops to 104 and
-// each softmax thread, which holds a whole 128-score row, gets 200 (the
-// smallest producer budget that compiles without spills; the sum is the
-// launch budget exactly).
-constexpr int kPfRegsLaunch = 168;
-constexpr int kPfRegsIo = 104;
-constexpr int kPfRegsSoftmax = 200;
-static_assert(4 * 32 * kPfRegsIo + 8 * 32 * kPfRegsSoftmax <= kPfThreads * kPfRegsLaunch,
+// Register budget per warpgroup (setmaxnreg): 640 threads launch with 96
+// registers each; warpgroup 0 (producer, MMA, rotation warps) and the
+// softmax warpgroups (64 scores per thread) split them.
+#ifndef GQA_PF_REGS_IO
+#define GQA_PF_REGS_IO 80
+#endif
+constexpr int kPfRegsLaunch = 96;
+constexpr int kPfRegsIo = GQA_PF_REGS_IO;
+constexpr int kPfRegsSoftmax = ((kPfThreads * kPfRegsLaunch - 4 * 32 * kPfRegsIo) / (16 * 32)) / 8 * 8;
+static_assert(4 * 32 * kPfRegsIo + 16 * 32 * kPfRegsSoftmax <= kPfThreads * kPfRegsLaunch,
               "register split");
 constexpr float kRescaleLog2 = 8.0f;  // lazy rescale threshold (log2 units)
 #ifndef GQA_POLY_PER4
@@ -185,10 +186,10 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             mbar_init(&q_full[k], 1);
             mbar_init(&q_empty[k], 1);
             mbar_init(&s_full[k], 1);
-            mbar_init(&p_full[k][0], 4);   // every softmax warp of the tile, per key half
-            mbar_init(&p_full[k][1], 4);
+            mbar_init(&p_full[k][0], 8);   // every softmax warp of the tile, per chunk
+            mbar_init(&p_full[k][1], 8);
             mbar_init(&o_done[k], 1);
-            mbar_init(&o_free[k], 4);
+            mbar_init(&o_free[k], 8);
             mbar_init(&q_ready[k], 2);     // the two rotating warps (kRope only)
         }
         mbar_init(&mma_drain, 1);
@@ -314,17 +315,21 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             }
             __syncwarp();
         };
-        // O_k (+)= P_k V_st over the keys of half `hf` (64 keys): P from tensor
-        // memory, V MN-major (d contiguous)
+        // O_k (+)= P_k V_st over the keys of chunk `hf`: the softmax releases
+        // P in two chunks, keys [32 hf, 32 hf + 32) and [64 + 32 hf, 96 + 32 hf)
+        // (each thread of a row pair holds one 64-key half); 16 keys per
+        // instruction.  P from tensor memory, V MN-major (d contiguous).
         auto issue_pv = [&](int k, int st, int hf, bool acc) {
             const uint32_t ts = tmem + (k ? Lay::kColS1 : Lay::kColS0);
             const uint32_t to = tmem + (k ? Lay::kColO1 : Lay::kColO0);
             const uint64_t bv = st ? dv1 : dv0;
             if (leader) {
 #pragma unroll
-                for (int kk = hf * (kPfBN / 32); kk < (hf + 1) * (kPfBN / 32); ++kk)
+                for (int i = 0; i < 4; ++i) {
+                    const int kk = 2 * hf + (i & 1) + 4 * (i >> 1);
                     umma_ts(to, ts + kk * 8, bv + kk * (2048 >> 4), idesc_o,
-                            (acc || kk > 0) ? 1u : 0u);
+                            (acc || i > 0) ? 1u : 0u);
+                }
             }
             __syncwarp();
         };
@@ -423,16 +428,32 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                 if (!ok) break;
                 if (active) {
                     uint8_t *tile = sQ + k * Lay::kQTile + panel * Lay::kQPanel;
+                    auto word_of = [&](int r) {
+                        return reinterpret_cast<uint32_t *>(tile + r * 128 +
+                                                            ((chunk ^ (r & 7)) << 4) + word * 4);
+                    };
                     const int first = u.t0 + k * p.P;            // position of the tile's row 0
                     const int n_pos = min(p.P, p.Tq - first);    // rows past Tq are zero fill
-                    for (int pl = 0; pl < n_pos; ++pl) {
-                        float cs, sn;
-                        rope_cos_sin(p.q_pos0 + first + pl, turns, cs, sn);
-                        for (int g = 0; g < p.G; ++g) {
-                            const int r = pl * p.G + g;
-                            uint32_t *w = reinterpret_cast<uint32_t *>(
-                                tile + r * 128 + ((chunk ^ (r & 7)) << 4) + word * 4);
-                            *w = rope_rotate_pair(*w, cs, sn);
+                    // four positions' angles at a time, four rows' loads in flight
+                    for (int pl0 = 0; pl0 < n_pos; pl0 += 4) {
+                        float cs[4], sn[4];
+#pragma unroll
+                        for (int e = 0; e < 4; ++e)
+                            rope_cos_sin(p.q_pos0 + first + pl0 + e, turns, cs[e], sn[e]);
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            if (pl0 + e >= n_pos) break;
+                            const int r0 = (pl0 + e) * p.G;
+                            for (int g0 = 0; g0 < p.G; g0 += 4) {
+                                uint32_t *w[4], v[4];
+#pragma unroll
+                                for (int x = 0; x < 4; ++x) w[x] = word_of(r0 + min(g0 + x, p.G - 1));
+#pragma unroll
+                                for (int x = 0; x < 4; ++x) v[x] = *w[x];
+#pragma unroll
+                                for (int x = 0; x < 4; ++x)   // a clamped tail row repeats the last one
+                                    if (g0 + x < p.G) *w[x] = rope_rotate_pair(v[x], cs[e], sn[e]);
+                            }
                         }
                     }
                 }
@@ -447,14 +468,18 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     } else {
         regs_inc<kPfRegsSoftmax>();      // marks the softmax code's budget for the compiler
         // -------------------------------------------- softmax + epilogue ----
-        // One thread per row: warps 4-7 serve M tile 0, warps 8-11 M tile 1;
-        // warp w reads tensor-memory lanes 32 (w % 4) .. 32 (w % 4) + 31, and
-        // each thread holds all 128 scores of its row, so the row max needs no
-        // exchange between threads.
-        const int k = (warp - 4) >> 2;                  // M tile
-        const int g4 = warp & 3;                        // lane group = SM sub-partition
-        const int r = (g4 << 5) + lane;                 // row = tensor-memory lane
-        const uint32_t lane_addr = tmem + ((static_cast<uint32_t>(g4) * 32u) << 16);
+        // Two threads per row, in one warp: warps 4-11 serve M tile 0, warps
+        // 12-19 M tile 1.  Warp w reads tensor-memory lanes of its quarter
+        // (w % 4), the lower or upper 16 of them; with the .16x32bx2 access
+        // shape, threads t and t + 16 hold the same row, t the scores of keys
+        // 0-63 and t + 16 those of keys 64-127, so the row max and the row sum
+        // cross between the two with one shuffle.
+        const int k = (warp - 4) >> 3;                  // M tile
+        const int hh = ((warp - 4) >> 2) & 1;           // lower / upper 16 lanes of the quarter
+        const int q4 = warp & 3;                        // lane quarter = SM sub-partition
+        const int ch = lane >> 4;                       // column half: keys 64 ch .. 64 ch + 63
+        const int r = q4 * 32 + hh * 16 + (lane & 15);  // row = tensor-memory lane
+        const uint32_t lane_addr = tmem + ((static_cast<uint32_t>(q4 * 32 + hh * 16)) << 16);
         const uint32_t colS = k ? Lay::kColS1 : Lay::kColS0;
         const uint32_t colO = k ? Lay::kColO1 : Lay::kColO0;
         const float c2 = p.scale_log2;
@@ -464,19 +489,25 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         PfUnit u;
         for (int i = 0; ok && pf_unit(p, i, u); ++i) {
             const int pos = u.t0 + k * p.P + r / p.G;
-            const int head = u.kvh * p.G + r % p.G;
             const bool row_real = (r < p.P * p.G) && (pos < p.Tq);
-            __nv_bfloat16 *dst =
-                p.o + ((static_cast<size_t>(u.b) * p.tq_pitch + pos) * p.Hq + head) * D;
-            float *lse_dst = p.lse ? p.lse + (static_cast<size_t>(u.b) * p.Hq + head) * p.Tq + pos
-                                   : nullptr;
+            // output row and lse slot, formed only where they are written
+            auto out_row = [&]() {
+                const int head = u.kvh * p.G + r % p.G;
+                return p.o + ((static_cast<size_t>(u.b) * p.tq_pitch + pos) * p.Hq + head) * D +
+                       (D / 2) * ch;
+            };
+            auto lse_slot = [&]() {
+                const int head = u.kvh * p.G + r % p.G;
+                return p.lse + (static_cast<size_t>(u.b) * p.Hq + head) * p.Tq + pos;
+            };
             if (u.n_kv == 0) {
                 // no visible key for any row of the unit: o = 0, lse = -inf
                 if (row_real) {
+                    __nv_bfloat16 *dst = out_row();
 #pragma unroll
-                    for (int e = 0; e < D / 8; ++e)
+                    for (int e = 0; e < D / 16; ++e)
                         reinterpret_cast<uint4 *>(dst)[e] = make_uint4(0u, 0u, 0u, 0u);
-                    if (lse_dst) *lse_dst = -INFINITY;
+                    if (p.lse && ch == 0) *lse_slot() = -INFINITY;
                 }
                 continue;
             }
@@ -490,44 +521,44 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             // scaled by exp2(-m_ref) and m_ref only moves when the row's max
             // exceeds it by more than kRescaleLog2 (P then stays <=
             // 2^kRescaleLog2).  Exact in real arithmetic: the epilogue divides
-            // by l taken at the same m_ref.
+            // by l taken at the same m_ref.  Both threads of a row see the same
+            // row max, so they take identical m_ref / alpha decisions; each
+            // keeps the partial l of its keys.
             float m_ref = -INFINITY, l_run = 0.0f;
             for (int j = 0; j < u.n_kv; ++j, ++gi) {
                 // warp-uniform outcome: the tensor-memory accesses below are .sync.aligned
                 ok = __all_sync(0xffffffffu, mbar_wait(&s_full[k], gi & 1, &abort_flag, p.status));
                 if (!ok) break;
                 tc_fence_after();
-                uint32_t sr[4][32];
-                tmem_ld64(lane_addr + colS, sr[0], sr[1]);
-                tmem_ld64(lane_addr + colS + 64, sr[2], sr[3]);
+                uint32_t sr[64];
+                tmem_ld_16x32bx2_x64<64>(lane_addr + colS, sr);
                 tmem_wait_ld();
-                const int key0 = u.tile(j) * kPfBN;             // key of column 0
+                const int key0 = u.tile(j) * kPfBN + 64 * ch;   // key of my first column
                 const bool masked = __any_sync(
-                    0xffffffffu, key0 + kPfBN - 1 > lim || (key0 < lo && key0 + kPfBN - 1 >= n_sinks));
+                    0xffffffffu, key0 + 63 > lim || (key0 < lo && key0 + 63 >= n_sinks));
                 if (masked) {
 #pragma unroll
-                    for (int c = 0; c < 4; ++c)
-#pragma unroll
-                        for (int e = 0; e < 32; ++e) {
-                            const int key = key0 + 32 * c + e;
-                            if (key > lim || (key < lo && key >= n_sinks))
-                                sr[c][e] = __float_as_uint(-INFINITY);
-                        }
+                    for (int e = 0; e < 64; ++e) {
+                        const int key = key0 + e;
+                        if (key > lim || (key < lo && key >= n_sinks))
+                            sr[e] = __float_as_uint(-INFINITY);
+                    }
                 }
-                // row max of the raw scores (scale > 0 keeps the order):
-                // 8 independent chains of 16 scores
-                float mx8[8];
+                // row max of the raw scores (scale > 0 keeps the order): 4
+                // chains of 16 scores, then the partner thread's half
+                float mx4[4];
 #pragma unroll
-                for (int c = 0; c < 8; ++c) {
-                    const uint32_t *v = &sr[c >> 1][(c & 1) * 16];
+                for (int c = 0; c < 4; ++c) {
+                    const uint32_t *v = &sr[16 * c];
                     float m = __uint_as_float(v[0]);
 #pragma unroll
                     for (int e = 1; e < 15; e += 2)
                         m = max3f(m, __uint_as_float(v[e]), __uint_as_float(v[e + 1]));
-                    mx8[c] = fmaxf(m, __uint_as_float(v[15]));
+                    mx4[c] = fmaxf(m, __uint_as_float(v[15]));
                 }
-                const float mxs = max3f(max3f(mx8[0], mx8[1], mx8[2]), max3f(mx8[3], mx8[4], mx8[5]),
-                                        fmaxf(mx8[6], mx8[7])) * c2;
+                float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
+                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
+                const float mxs = mx * c2;
                 const bool move = mxs > m_ref + kRescaleLog2;  // always true on the first key seen
                 float alpha = 1.0f;
                 if (move) {
@@ -535,14 +566,13 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                     m_ref = mxs;
                 }
                 // O holds tiles < j at the old reference: rescale rows whose
-                // reference moved, before this tile's first PV half is released
+                // reference moved, before this tile's first P chunk is released
                 if (j > 0 && __any_sync(0xffffffffu, move)) {
                     const float2 a2 = make_float2(alpha, alpha);
-                    // 16 columns at a time: the row's 128 scores stay live meanwhile
 #pragma unroll 1
-                    for (int c = 0; c < D / 16; ++c) {
+                    for (int c = 0; c < D / 32; ++c) {
                         uint32_t orr[16];
-                        tmem_ld16(lane_addr + colO + 16 * c, orr);
+                        tmem_ld_16x32bx2_x16<D / 2>(lane_addr + colO + 16 * c, orr);
                         tmem_wait_ld();
 #pragma unroll
                         for (int e = 0; e < 16; e += 2) {
@@ -551,7 +581,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                             orr[e] = __float_as_uint(v2.x);
                             orr[e + 1] = __float_as_uint(v2.y);
                         }
-                        tmem_st16(lane_addr + colO + 16 * c, orr);
+                        tmem_st_16x32bx2_x16<D / 2>(lane_addr + colO + 16 * c, orr);
                     }
                 }
                 const float m_use = (m_ref == -INFINITY) ? 0.0f : m_ref;
@@ -559,22 +589,21 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                 float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
                 // P = exp2(s * scale * log2e - m_ref), truncated to bf16; P
                 // overwrites the first 64 columns of S (keys 2c, 2c + 1 in packed
-                // column c).  l sums exactly the bf16 weights the PV product
-                // uses, so O / l is a convex combination of V rows.  Tiles with
-                // masked (-inf) scores use the MUFU exp only; full tiles send part
-                // of the pairs to the FMA-pipe polynomial.  Each half of the keys
-                // is released to the PV product as soon as it is stored.
+                // column c; this thread's keys 64 ch + [0, 64) in packed columns
+                // 32 ch + [0, 32)).  l sums exactly the bf16 weights the PV
+                // product uses, so O / l is a convex combination of V rows.
+                // Tiles with masked (-inf) scores use the MUFU exp only; full
+                // tiles send part of the pairs to the FMA-pipe polynomial.  The
+                // chunk of 32 keys is released to the PV product once stored.
 #pragma unroll
                 for (int hf = 0; hf < 2; ++hf) {
-#pragma unroll
-                    for (int c = 2 * hf; c < 2 * hf + 2; ++c) {
-                        uint32_t pk[16];
-                        if (masked)
-                            softmax_chunk<false>(sr[c], cc, nm, pk, acc);
-                        else
-                            softmax_chunk<true>(sr[c], cc, nm, pk, acc);
-                        tmem_st16(lane_addr + colS + 16 * c, pk);
-                    }
+                    uint32_t pk[16];
+                    const uint32_t(&src)[32] = *reinterpret_cast<const uint32_t(*)[32]>(&sr[32 * hf]);
+                    if (masked)
+                        softmax_chunk<false>(src, cc, nm, pk, acc);
+                    else
+                        softmax_chunk<true>(src, cc, nm, pk, acc);
+                    tmem_st_16x32bx2_x16<32>(lane_addr + colS + 16 * hf, pk);
                     tmem_wait_st();
                     tc_fence_before();
                     __syncwarp();
@@ -583,27 +612,30 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                 l_run = l_run * alpha + ((acc[0] + acc[1]) + (acc[2] + acc[3]));
             }
             if (!ok) break;
-            // ---- epilogue: O / l -> bf16, lse ----
+            // ---- epilogue: O / l -> bf16, lse (each thread writes its D/2 columns) ----
             // O_k is read out of tensor memory, then released to the next
             // unit's first PV before the conversion and the global stores.
             ok = __all_sync(0xffffffffu, mbar_wait(&o_done[k], ui & 1, &abort_flag, p.status));
             if (!ok) break;
             tc_fence_after();
-            uint32_t orr[D / 32][32];
+            uint32_t orr[D / 32][16];
 #pragma unroll
-            for (int c = 0; c < D / 32; ++c) tmem_ld32(lane_addr + colO + 32 * c, orr[c]);
+            for (int c = 0; c < D / 32; ++c)
+                tmem_ld_16x32bx2_x16<D / 2>(lane_addr + colO + 16 * c, orr[c]);
             tmem_wait_ld();
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&o_free[k]);
             ++ui;
-            const float inv_l = (l_run > 0.0f) ? 1.0f / l_run : 0.0f;
+            const float l_row = l_run + __shfl_xor_sync(0xffffffffu, l_run, 16);
+            const float inv_l = (l_row > 0.0f) ? 1.0f / l_row : 0.0f;
             if (row_real) {
+                __nv_bfloat16 *dst = out_row();
 #pragma unroll
                 for (int c = 0; c < D / 32; ++c) {
-                    uint4 *d4 = reinterpret_cast<uint4 *>(dst + 32 * c);
+                    uint4 *d4 = reinterpret_cast<uint4 *>(dst + 16 * c);
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) {
+                    for (int e = 0; e < 2; ++e) {
                         const uint32_t *v = &orr[c][8 * e];
                         d4[e] = make_uint4(
                             pack_bf16x2(__uint_as_float(v[0]) * inv_l, __uint_as_float(v[1]) * inv_l),
@@ -612,9 +644,9 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                             pack_bf16x2(__uint_as_float(v[6]) * inv_l, __uint_as_float(v[7]) * inv_l));
                     }
                 }
-                if (lse_dst)
-                    *lse_dst = (l_run > 0.0f) ? (m_ref + __log2f(l_run)) * 0.69314718055994531f
-                                              : -INFINITY;
+                if (p.lse && ch == 0)
+                    *lse_slot() = (l_row > 0.0f) ? (m_ref + __log2f(l_row)) * 0.69314718055994531f
+                                                 : -INFINITY;
             }
         }
     }
