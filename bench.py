@@ -10,8 +10,9 @@ One step = one pass of the whole hot path over one batch of synthetic input:
      uniform on [1024, 8192], split-KV kernel whose last split per group
      merges the splits (log-sum-exp).
 Inputs are seeded synthetic tensors already resident in HBM.  L2 (126 MB) is
-flushed by writing a 256 MB buffer before every timed launch; each launch is
-timed with CUDA events on the stream it runs on.
+flushed before every timed launch by writing a 256 MB buffer and reading it
+back (so no dirty lines are left for the timed kernel to write back); each
+launch is timed with CUDA events on the stream it runs on.
 
 The JSON line's ``value`` is prefill TFLOP/s (algorithmic FLOPs: 4*B*Hq*d*
 unmasked pairs, all ranks) and ``decode.value`` is decode KV GB/s.  ``e2e``
@@ -269,7 +270,7 @@ def run_reference(args, world, rank):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic", "impl": "reference",
         "config": {"workload": WORKLOAD, "prefill": c, "decode": DECODE,
-                   "l2": "flushed (256 MB write) before every timed launch",
+                   "l2": "flushed before every timed launch (256 MB written, then read back: clean lines)",
                    "parallelism": "1 GPU"},
         "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
                          "sample": f"{rows} random query rows of the causal T=4096 "
@@ -295,13 +296,27 @@ def visible_pairs(Tq, Tkv, causal=True, window=0, sinks=0):
     return int(n.sum())
 
 
+class L2Flush:
+    """Flushes L2 (126 MB) before a timed launch: writes a 256 MB buffer, then reads
+    it back.  The read leaves L2 holding clean lines only, so the timed kernel does
+    not pay for writing back the flush's dirty lines (a write-only flush left ~126 MB
+    of them, which added ~15 us to the DRAM-bound decode and nothing to the prefill)."""
+
+    def __init__(self, dev, nbytes=256 * 1024 * 1024):
+        self.buf = torch.empty(nbytes, dtype=torch.uint8, device=dev)
+
+    def __call__(self):
+        self.buf.zero_()
+        return self.buf.sum()
+
+
 def time_median(fn, flush, stream, reps):
     """Median CUDA-event time (ms) of fn() with L2 flushed before each launch."""
     for _ in range(3):
         fn()
     ts = []
     for _ in range(reps):
-        flush.zero_()
+        flush()
         s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         s0.record(stream)
         fn()
@@ -477,7 +492,7 @@ def run_ours(args, world, rank, local):
 
     c, dc = PREFILL, DECODE
     stream = torch.cuda.current_stream(dev)
-    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    flush = L2Flush(dev)
     if args.only == "next":
         # the rows beyond the hot path alone (profiling runs of their kernels)
         peaks, peak_kind = load_peaks()
@@ -500,14 +515,14 @@ def run_ours(args, world, rank, local):
 
     def step(evs=None):
         if do_pre:
-            flush.zero_()
+            flush()
             if evs:
                 evs[0].record(stream)
             gqa.attn(q, k, v, causal=True, out=o)
             if evs:
                 evs[1].record(stream)
         if do_dec:
-            flush.zero_()
+            flush()
             if evs:
                 evs[2].record(stream)
             gqa.decode(dq, kc, vc, sl, workspace=ws, out=do)
@@ -614,6 +629,33 @@ def run_ours(args, world, rank, local):
         dec = {"value": world * d_bytes * K / (dec_ms / 1e3) / 1e9, "unit": "GB/s",
                "roofline": dec_roof}
 
+    # host time to enqueue one call through the C ABI (argument checks, tensor
+    # maps, launch), averaged over back-to-back calls; outside the timed region
+    enqueue = {}
+    if not args.no_enqueue:
+        from grouped_query_attention_attn_b200 import _binding as cabi
+        st = stream.cuda_stream
+
+        def per_call_us(fn, n=200):
+            torch.cuda.synchronize(dev)
+            t = time.perf_counter()
+            for _ in range(n):
+                fn()
+            t = time.perf_counter() - t
+            torch.cuda.synchronize(dev)
+            return 1e6 * t / n
+
+        if do_pre:
+            enqueue["gqa_attn_fwd"] = per_call_us(lambda: cabi.gqa_attn_fwd(
+                q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), c["B"], c["T"], c["T"],
+                c["Hq"], c["Hkv"], c["d"], 1, c["d"] ** -0.5, st))
+        if do_dec:
+            enqueue["gqa_decode"] = per_call_us(lambda: cabi.gqa_decode(
+                dq.data_ptr(), kc.data_ptr(), vc.data_ptr(), sl.data_ptr(), do.data_ptr(),
+                dc["B"], dc["Hq"], dc["Hkv"], dc["d"], dc["Lmax"], dc["d"] ** -0.5,
+                ws.data_ptr(), ws.numel(), st))
+        gqa.device_status()
+
     nxt = None
     if args.only is None and not args.no_next:
         nxt = measure_next_rows(dev, stream, flush, peaks, peak_kind, args.next_reps)
@@ -627,13 +669,14 @@ def run_ours(args, world, rank, local):
             "data": "synthetic",
             "config": {"workload": WORKLOAD if args.only is None else args.only,
                        "prefill": c if do_pre else None, "decode": dc if do_dec else None,
-                       "l2": "flushed (256 MB write) before every timed launch",
+                       "l2": "flushed before every timed launch (256 MB written, then read back: clean lines)",
                        "parallelism": f"{world} independent replicas" if world > 1 else "1 GPU"},
             "decode": dec,
             "roofline": roofline if do_pre else (dec or {}).get("roofline"),
             "clocks": clocks,
             "e2e": e2e,
             "gpu_launches": K * ((1 if do_pre else 0) + (1 if do_dec else 0)),
+            "host_enqueue_us_per_call": enqueue or None,
             "wall_s_timed_region": wall,
             "cpu_baseline": cpu,
             "next_rows": nxt,
@@ -657,6 +700,8 @@ def main():
     ap.add_argument("--only", choices=["prefill", "decode", "next"], default=None,
                     help="time one kernel family only (profiling runs)")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-enqueue", action="store_true",
+                    help="skip the host enqueue-time measurement")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--no-next", action="store_true",
                     help="skip the measurements of the rows beyond the hot path")

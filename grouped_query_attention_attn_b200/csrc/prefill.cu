@@ -17,8 +17,10 @@
 //               a 2-deep ring of V tiles (128 keys x d, 128-byte swizzle).
 //   warp 1      one thread issues tcgen05.mma:  S_k = Q_k K_j^T into tensor
 //               memory, then O_k += P_k V_j with P_k read from tensor memory.
-//   warps 4-7   softmax + epilogue of M tile 0 (thread = row = TMEM lane),
-//   warps 8-11  the same for M tile 1.
+//   warps 4-11  softmax + epilogue of M tile 0, two threads per row (the
+//               .16x32bx2 tensor-memory shape), warps 12-19 the same for M
+//               tile 1; with rotary embedding they also rotate their tile's Q
+//               rows in shared memory at the start of each unit.
 // Tensor memory (512 columns): S_0 | S_1 | O_0 | O_1; P_k (bf16) overwrites
 // the first 64 columns of S_k.  The tensor pipe executes one thread's MMAs in
 // issue order, so S_k(j+1) never overwrites P_k(j) before PV_k(j) has read it.
@@ -157,8 +159,9 @@ __device__ __forceinline__ bool pf_unit(const PfParams &p, int i, PfUnit &u) {
 // the current unit's epilogue.  Iteration counters run over all units of the
 // CTA (ring stages and barrier phases), unit counters over units with at
 // least one KV tile.
-// kRope: warps 2 and 3 rotate each Q tile in shared memory (rotary position
-// embedding) after its TMA copy lands and before the first S product reads it.
+// kRope: each tile's softmax warps rotate its Q rows in shared memory
+// (rotary position embedding) after the TMA copy lands and before the first S
+// product reads them.
 template <int D, bool kRope>
 __global__ void __launch_bounds__(kPfThreads, 1)
 prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -190,7 +193,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             mbar_init(&p_full[k][1], 8);
             mbar_init(&o_done[k], 1);
             mbar_init(&o_free[k], 8);
-            mbar_init(&q_ready[k], 2);     // the two rotating warps (kRope only)
+            mbar_init(&q_ready[k], 8);     // the tile's softmax warps, once rotated (kRope)
         }
         mbar_init(&mma_drain, 1);
         abort_flag = 0;
@@ -407,63 +410,6 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         // every MMA this warp issued has finished before tensor memory is freed
         commit(&mma_drain);
         mbar_wait(&mma_drain, 0, &abort_flag, p.status, 1000000000ull);
-    } else if (kRope) {
-        // -------------------------------------------- Q rotation (RoPE) ----
-        // Thread i of warps 2-3 owns coordinate pair i (columns 2i, 2i+1) of
-        // every row of the tile: one cosine / sine per position, applied to the
-        // G rows (heads) of that position.  Pairs never straddle a 16-byte
-        // chunk, so the 128-byte swizzle only moves whole pairs; a warp touches
-        // one 128-byte row of one panel at a time (no bank conflicts).
-        const int i = (warp - 2) * 32 + lane;
-        const bool active = i < D / 2;
-        const double turns = active ? rope_turns(i, D / 2, p.log_theta) : 0.0;
-        const int panel = (2 * i) / 64, chunk = ((2 * i) % 64) / 8, word = ((2 * i) % 8) / 2;
-        int ui = 0;
-        bool ok = true;
-        PfUnit u;
-        for (int it = 0; ok && pf_unit(p, it, u); ++it) {
-            if (u.n_kv == 0) continue;
-            for (int k = 0; k < 2; ++k) {
-                ok = __all_sync(0xffffffffu, mbar_wait(&q_full[k], ui & 1, &abort_flag, p.status));
-                if (!ok) break;
-                if (active) {
-                    uint8_t *tile = sQ + k * Lay::kQTile + panel * Lay::kQPanel;
-                    auto word_of = [&](int r) {
-                        return reinterpret_cast<uint32_t *>(tile + r * 128 +
-                                                            ((chunk ^ (r & 7)) << 4) + word * 4);
-                    };
-                    const int first = u.t0 + k * p.P;            // position of the tile's row 0
-                    const int n_pos = min(p.P, p.Tq - first);    // rows past Tq are zero fill
-                    // four positions' angles at a time, four rows' loads in flight
-                    for (int pl0 = 0; pl0 < n_pos; pl0 += 4) {
-                        float cs[4], sn[4];
-#pragma unroll
-                        for (int e = 0; e < 4; ++e)
-                            rope_cos_sin(p.q_pos0 + first + pl0 + e, turns, cs[e], sn[e]);
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            if (pl0 + e >= n_pos) break;
-                            const int r0 = (pl0 + e) * p.G;
-                            for (int g0 = 0; g0 < p.G; g0 += 4) {
-                                uint32_t *w[4], v[4];
-#pragma unroll
-                                for (int x = 0; x < 4; ++x) w[x] = word_of(r0 + min(g0 + x, p.G - 1));
-#pragma unroll
-                                for (int x = 0; x < 4; ++x) v[x] = *w[x];
-#pragma unroll
-                                for (int x = 0; x < 4; ++x)   // a clamped tail row repeats the last one
-                                    if (g0 + x < p.G) *w[x] = rope_rotate_pair(v[x], cs[e], sn[e]);
-                            }
-                        }
-                    }
-                }
-                // the tensor core reads the tile through the async proxy
-                fence_proxy_async_smem();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&q_ready[k]);
-            }
-            ++ui;
-        }
     }
     } else {
         regs_inc<kPfRegsSoftmax>();      // marks the softmax code's budget for the compiler
@@ -484,6 +430,53 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         const uint32_t colO = k ? Lay::kColO1 : Lay::kColO0;
         const float c2 = p.scale_log2;
         const int n_sinks = p.window > 0 ? p.sinks : 0;
+        // Rotary embedding (kRope): the tile's 256 threads rotate its Q rows in
+        // shared memory at the start of each unit, before its first S product.
+        // Thread tt owns coordinate pair i (columns 2i, 2i+1) of a block of
+        // consecutive rows; pairs never straddle a 16-byte chunk, so the
+        // 128-byte swizzle moves whole pairs, and a warp's 32 pairs of one row
+        // are 32 different banks.
+        constexpr int kHalfD = D / 2, kPhases = 256 / kHalfD, kRowsPerPhase = kPfBM / kPhases;
+        const int tt = ((warp - 4) & 7) * 32 + lane;   // thread of the tile, 0..255
+        const int rope_i = tt % kHalfD, rope_ph = tt / kHalfD;
+        const double rope_trn = kRope ? rope_turns(rope_i, kHalfD, p.log_theta) : 0.0;
+        uint8_t *rope_base = sQ + k * Lay::kQTile + ((2 * rope_i) / 64) * Lay::kQPanel;
+        const int rope_ck = ((2 * rope_i) % 64) / 8, rope_wd = ((2 * rope_i) % 8) / 2;
+        // Rotates this tile's Q rows of unit uu (the unit's Q copy completes
+        // phase `parity` of q_full[k]) and releases them to the S product.
+        auto rotate_q = [&](const PfUnit &uu, uint32_t parity) {
+            if (!__all_sync(0xffffffffu, mbar_wait(&q_full[k], parity, &abort_flag, p.status)))
+                return false;
+            auto word_of = [&](int row) {
+                return reinterpret_cast<uint32_t *>(rope_base + row * 128 +
+                                                    ((rope_ck ^ (row & 7)) << 4) + rope_wd * 4);
+            };
+            const int first = uu.t0 + k * p.P;                              // position of row 0
+            const int real_rows = max(0, min(p.P, p.Tq - first)) * p.G;     // rest: zero fill
+            const int r_end = min((rope_ph + 1) * kRowsPerPhase, real_rows);
+            for (int r0 = rope_ph * kRowsPerPhase; r0 < r_end;) {
+                const int pl = r0 / p.G;                                     // one position's rows
+                const int r1 = min(r_end, (pl + 1) * p.G);
+                float cs, sn;
+                rope_cos_sin(p.q_pos0 + first + pl, rope_trn, cs, sn);
+                for (int rr = r0; rr < r1; rr += 4) {                        // four loads in flight
+                    uint32_t *w[4], v[4];
+#pragma unroll
+                    for (int x = 0; x < 4; ++x) w[x] = word_of(min(rr + x, r1 - 1));
+#pragma unroll
+                    for (int x = 0; x < 4; ++x) v[x] = *w[x];
+#pragma unroll
+                    for (int x = 0; x < 4; ++x)   // a clamped tail row repeats the last one
+                        if (rr + x < r1) *w[x] = rope_rotate_pair(v[x], cs, sn);
+                }
+                r0 = r1;
+            }
+            // the tensor core reads the tile through the async proxy
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&q_ready[k]);
+            return true;
+        };
         int gi = 0, ui = 0;
         bool ok = true;
         PfUnit u;
@@ -510,6 +503,10 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                     if (p.lse && ch == 0) *lse_slot() = -INFINITY;
                 }
                 continue;
+            }
+            // the unit's Q rows are rotated before its first S product
+            if constexpr (kRope) {
+                if (!(ok = rotate_q(u, ui & 1))) break;
             }
             // visible keys of this row: key <= lim, and key >= lo or key < sinks
             // (keys past Tkv never count; lo / sinks only with a sliding window)
