@@ -106,15 +106,24 @@ rowdot_kernel(const __nv_bfloat16 *__restrict__ dout, const __nv_bfloat16 *__res
 //                 row, one per 32-query quarter);
 //   tensor pipe   dV += P^T dO and dK += dS^T Q with P^T / dS^T read from
 //                 tensor memory (dV and dK accumulate over all items).
-// S^T and dP^T are committed separately and P^T and dS^T are published
-// separately, so the tensor pipe computes dV(i) while the warps form dS^T(i)
-// and the next item's dP^T while they form its P^T.
-// Tensor memory (512 columns): S^T | dP^T | dV | dK.  Shared memory: K, V,
-// and a 2-deep ring of (Q, dO, lse, D) per item.
+// Issue order S(0) dP(0) | dV(0) S(1) | dK(0) dP(1) | dV(1) S(2) | ...: the
+// next S^T is issued right behind the dV product that reads the P^T it
+// overwrites (products run in issue order), so it runs while the warps form
+// dS^T and is ready when they finish; dP^T(i+1) follows dK(i), which reads
+// dS^T(i) from the region it overwrites.  S^T(i+1) therefore needs Q(i+1)
+// about one elementwise phase after dK(i-1) has released a Q stage: Q has a
+// 3-deep ring, dO (released by dV, earlier) a 2-deep one, each with its own
+// barriers.  The item's lse travels with Q; its D (read by the warps after dV
+// has released dO) has a 2-deep buffer of its own that the warps release.
+// Tensor memory (512 columns): S^T | dP^T | dV | dK.  Shared memory (all of
+// it dynamic, 1024-byte aligned, barriers at the end): K, V, the Q and dO
+// rings, lse and D.
 constexpr int kTcBK = 128;       // keys per CTA
 constexpr int kTcBQ = 128;       // query rows per item
 constexpr int kTcThreads = 640;  // producer, MMA, 2 idle, 16 elementwise warps
 constexpr int kTcElemWarps = 16;   // 4 per tensor-memory lane group, 32 columns each
+constexpr int kTcQStages = 3;
+constexpr int kTcOStages = 2;
 
 template <int D>
 struct TcLayout {
@@ -122,13 +131,19 @@ struct TcLayout {
     static constexpr int kPanel = 128 * 128;               // 128 rows x 64 bf16
     static constexpr int kTile = kPanels * kPanel;
     static constexpr int kOffK = 0, kOffV = kTile;
-    static constexpr int kOffQ = 2 * kTile;                // [2] Q tiles
-    static constexpr int kOffO = kOffQ + 2 * kTile;        // [2] dO tiles
-    static constexpr int kOffL = kOffO + 2 * kTile;        // [2][2][128] floats: L, D
-    static constexpr int kBytes = kOffL + 2 * 2 * kTcBQ * 4;
-    static constexpr int kSmemBytes = kBytes + 1024;
+    static constexpr int kOffQ = 2 * kTile;                          // [kTcQStages]
+    static constexpr int kOffO = kOffQ + kTcQStages * kTile;         // [kTcOStages]
+    static constexpr int kOffL = kOffO + kTcOStages * kTile;         // [kTcQStages][128] f32
+    static constexpr int kOffD = kOffL + kTcQStages * kTcBQ * 4;     // [2][128] f32
+    // barriers: kv_full, q_full[3], q_empty[3], o_full[2], o_empty[2],
+    // d_full[2], d_empty[2], s_full, dp_full, p_full, ds_full, acc_done
+    static constexpr int kNumBars = 1 + 2 * kTcQStages + 2 * kTcOStages + 4 + 5;
+    static constexpr int kOffBar = kOffD + 2 * kTcBQ * 4;
+    static constexpr int kOffMisc = kOffBar + kNumBars * 8;          // tmem base, abort flag
+    static constexpr int kSmemBytes = kOffMisc + 16;
     static constexpr uint32_t kColS = 0, kColP = 128, kColDV = 256, kColDK = 256 + D;
 };
+static_assert(TcLayout<128>::kSmemBytes <= 232448, "dK/dV shared memory");
 
 struct TcParams {
     int B, Tq, Tkv, Hq, Hkv, G;
@@ -146,13 +161,23 @@ dkdv_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
                const TcParams p) {
     using Lay = TcLayout<D>;
-    extern __shared__ uint8_t smem_raw[];
-    uint8_t *smem = reinterpret_cast<uint8_t *>(
-        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-    __shared__ uint64_t kv_full, qo_full[2], qo_empty[2], s_full, dp_full, p_full, ds_full,
-        acc_done;
-    __shared__ uint32_t tmem_base_sh;
-    __shared__ int abort_flag;
+    // the whole budget is used: the window must start 1024-byte aligned (the
+    // 128-byte swizzle's requirement) with no room to align it here
+    extern __shared__ __align__(1024) uint8_t smem[];
+    if (smem_u32(smem) & 1023u) {
+        if (threadIdx.x == 0) record_status(p.status, GQA_ERR_CUDA);
+        return;
+    }
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + Lay::kOffBar);
+    uint64_t *kv_full = bars, *q_full = bars + 1, *q_empty = q_full + kTcQStages;
+    uint64_t *o_full = q_empty + kTcQStages, *o_empty = o_full + kTcOStages;
+    uint64_t *d_full = o_empty + kTcOStages, *d_empty = d_full + 2;
+    uint64_t *s_full = d_empty + 2, *dp_full = s_full + 1, *p_full = s_full + 2;
+    uint64_t *ds_full = s_full + 3, *acc_done = s_full + 4;
+    uint32_t *tmem_base_sh = reinterpret_cast<uint32_t *>(smem + Lay::kOffMisc);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + Lay::kOffMisc + 4);
+    float *sL = reinterpret_cast<float *>(smem + Lay::kOffL);
+    float *sD = reinterpret_cast<float *>(smem + Lay::kOffD);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
     const int bhs = p.Hkv * p.B, lin = blockIdx.x;
@@ -171,218 +196,292 @@ dkdv_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     const int n_items = p.G * n_qb;
 
     if (threadIdx.x == 0) {
-        mbar_init(&kv_full, 1);
-        for (int s = 0; s < 2; ++s) {
-            mbar_init(&qo_full[s], 1);
-            mbar_init(&qo_empty[s], 1);
+        mbar_init(kv_full, 1);
+        for (int s = 0; s < kTcQStages; ++s) {
+            mbar_init(&q_full[s], 2);    // the copy's arrival and the lse stores'
+            mbar_init(&q_empty[s], 1);
         }
-        mbar_init(&s_full, 1);
-        mbar_init(&dp_full, 1);
-        mbar_init(&p_full, kTcElemWarps);
-        mbar_init(&ds_full, kTcElemWarps);
-        mbar_init(&acc_done, 1);
-        abort_flag = 0;
+        for (int s = 0; s < kTcOStages; ++s) {
+            mbar_init(&o_full[s], 1);
+            mbar_init(&o_empty[s], 1);
+        }
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(&d_full[s], 1);
+            mbar_init(&d_empty[s], kTcElemWarps);
+        }
+        mbar_init(s_full, 1);
+        mbar_init(dp_full, 1);
+        mbar_init(p_full, kTcElemWarps);
+        mbar_init(ds_full, kTcElemWarps);
+        mbar_init(acc_done, 1);
+        *abort_flag = 0;
         fence_mbar_init();
     }
     if (warp == 0) {
-        tmem_alloc(&tmem_base_sh, 512);
+        tmem_alloc(tmem_base_sh, 512);
         tmem_relinquish();
     }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    const uint32_t tmem = tmem_base_sh;
-    float *sLD = reinterpret_cast<float *>(smem + Lay::kOffL);   // [stage][L | D][128]
+    const uint32_t tmem = *tmem_base_sh;
 
+    if (warp < 4) {
     if (warp == 0) {
         // ------------------------------------------------ TMA producer ----
+        // Per item: Q and its lse (the copy is issued first and the lse stored
+        // while it flies), dO, then D once the warps have released its buffer.
         const bool leader = elect_one();
         if (n_items > 0) {
             if (leader) {
                 tma_prefetch_desc(&tm_q);
                 tma_prefetch_desc(&tm_o);
-                mbar_expect_tx(&kv_full, 2 * Lay::kTile);
+                mbar_expect_tx(kv_full, 2 * Lay::kTile);
                 for (int pn = 0; pn < Lay::kPanels; ++pn) {
-                    tma_load_4d(smem + Lay::kOffK + pn * Lay::kPanel, &tm_k, &kv_full, pn * 64,
+                    tma_load_4d(smem + Lay::kOffK + pn * Lay::kPanel, &tm_k, kv_full, pn * 64,
                                 kvh, k0, b);
-                    tma_load_4d(smem + Lay::kOffV + pn * Lay::kPanel, &tm_v, &kv_full, pn * 64,
+                    tma_load_4d(smem + Lay::kOffV + pn * Lay::kPanel, &tm_v, kv_full, pn * 64,
                                 kvh, k0, b);
                 }
             }
             __syncwarp();
-            int issued = 0;
+            int issued_q = 0, issued_o = 0;
             for (int it = 0; it < n_items; ++it) {
-                const int st = it & 1;
                 const int g = it / n_qb, q0 = (qb0 + it % n_qb) * kTcBQ, hq = kvh * p.G + g;
-                if (!__all_sync(0xffffffffu, mbar_wait(&qo_empty[st], ((it >> 1) & 1) ^ 1,
-                                                       &abort_flag, p.status)))
-                    break;
-                // the item's softmax statistics, lse in log2 units (rows past Tq: 0)
                 const size_t lrow = (static_cast<size_t>(b) * p.Hq + hq) * p.Tq;
-                float *L = sLD + st * 2 * kTcBQ, *Dd = L + kTcBQ;
+                const int qs = it % kTcQStages, os = it % kTcOStages;
+                if (!__all_sync(0xffffffffu, mbar_wait(&q_empty[qs], ((it / kTcQStages) & 1) ^ 1,
+                                                       abort_flag, p.status)))
+                    break;
+                if (leader) {
+                    mbar_expect_tx(&q_full[qs], Lay::kTile);
+                    for (int pn = 0; pn < Lay::kPanels; ++pn)
+                        tma_load_4d(smem + Lay::kOffQ + qs * Lay::kTile + pn * Lay::kPanel, &tm_q,
+                                    &q_full[qs], pn * 64, hq, q0, b);
+                }
+                // lse in log2 units (rows past Tq: 0)
 #pragma unroll
                 for (int e = 0; e < kTcBQ / 32; ++e) {
                     const int r = lane + 32 * e, qi = q0 + r;
-                    L[r] = qi < p.Tq ? p.lse[lrow + qi] * 1.4426950408889634f : 0.0f;
-                    Dd[r] = qi < p.Tq ? p.Dsum[lrow + qi] : 0.0f;
+                    sL[qs * kTcBQ + r] = qi < p.Tq ? p.lse[lrow + qi] * 1.4426950408889634f : 0.0f;
                 }
                 __syncwarp();
+                if (leader) mbar_arrive(&q_full[qs]);
+                __syncwarp();
+                issued_q = it + 1;
+                if (!__all_sync(0xffffffffu, mbar_wait(&o_empty[os], ((it / kTcOStages) & 1) ^ 1,
+                                                       abort_flag, p.status)))
+                    break;
                 if (leader) {
-                    mbar_expect_tx(&qo_full[st], 2 * Lay::kTile);
-                    for (int pn = 0; pn < Lay::kPanels; ++pn) {
-                        tma_load_4d(smem + Lay::kOffQ + st * Lay::kTile + pn * Lay::kPanel, &tm_q,
-                                    &qo_full[st], pn * 64, hq, q0, b);
-                        tma_load_4d(smem + Lay::kOffO + st * Lay::kTile + pn * Lay::kPanel, &tm_o,
-                                    &qo_full[st], pn * 64, hq, q0, b);
-                    }
+                    mbar_expect_tx(&o_full[os], Lay::kTile);
+                    for (int pn = 0; pn < Lay::kPanels; ++pn)
+                        tma_load_4d(smem + Lay::kOffO + os * Lay::kTile + pn * Lay::kPanel, &tm_o,
+                                    &o_full[os], pn * 64, hq, q0, b);
                 }
                 __syncwarp();
-                issued = it + 1;
+                issued_o = it + 1;
+                const int ds_ = it & 1;
+                if (!__all_sync(0xffffffffu, mbar_wait(&d_empty[ds_], ((it >> 1) & 1) ^ 1,
+                                                       abort_flag, p.status)))
+                    break;
+#pragma unroll
+                for (int e = 0; e < kTcBQ / 32; ++e) {
+                    const int r = lane + 32 * e, qi = q0 + r;
+                    sD[ds_ * kTcBQ + r] = qi < p.Tq ? p.Dsum[lrow + qi] : 0.0f;
+                }
+                __syncwarp();
+                if (leader) mbar_arrive(&d_full[ds_]);
+                __syncwarp();
             }
             // copies still in flight land before the block exits
-            mbar_wait(&kv_full, 0, &abort_flag, p.status, 1000000ull);
-            for (int it = max(0, issued - 2); it < issued; ++it)
-                mbar_wait(&qo_full[it & 1], (it >> 1) & 1, &abort_flag, p.status, 1000000ull);
+            mbar_wait(kv_full, 0, abort_flag, p.status, 1000000ull);
+            for (int it = max(0, issued_q - kTcQStages); it < issued_q; ++it)
+                mbar_wait(&q_full[it % kTcQStages], (it / kTcQStages) & 1, abort_flag, p.status,
+                          1000000ull);
+            for (int it = max(0, issued_o - kTcOStages); it < issued_o; ++it)
+                mbar_wait(&o_full[it % kTcOStages], (it / kTcOStages) & 1, abort_flag, p.status,
+                          1000000ull);
         }
-    } else if (warp == 1 && lane == 0) {
+    } else if (warp == 1) {
         // ------------------------------------------------- MMA issuer ----
-        if (n_items > 0) {
+        if (lane == 0 && n_items > 0) {
             constexpr uint32_t idesc_s = umma_idesc_bf16(kTcBK, kTcBQ, 0, 0);
             constexpr uint32_t idesc_o = umma_idesc_bf16(kTcBK, D, 0, 1);
             const uint32_t base = smem_u32(smem);
             const uint64_t dK = umma_smem_desc(base + Lay::kOffK, 16, 1024);
             const uint64_t dV = umma_smem_desc(base + Lay::kOffV, 16, 1024);
             auto wait = [&](uint64_t *bar, uint32_t parity) {
-                return mbar_wait(bar, parity, &abort_flag, p.status);
+                return mbar_wait(bar, parity, abort_flag, p.status);
             };
-            // S^T = K Q^T and dP^T = V dO^T of item it: K-major A and B (+32 B
-            // per 16 of d), each with its own commit
-            auto issue_s = [&](int it, uint32_t col, uint64_t a, uint32_t off_b, uint64_t *bar) {
-                const uint64_t bd = umma_smem_desc(base + off_b + (it & 1) * Lay::kTile, 16, 1024);
+            // S^T = K Q^T or dP^T = V dO^T into `col`: K-major A and B (+32 B per
+            // 16 of d), committed to `bar`
+            auto issue_s = [&](uint32_t col, uint64_t a, uint32_t off_b, uint64_t *bar) {
+                const uint64_t bd = umma_smem_desc(base + off_b, 16, 1024);
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint32_t off = ((kk >> 2) * Lay::kPanel + (kk & 3) * 32) >> 4;
-                    umma_ss(tmem + col, a + off, bd + off, idesc_s, kk > 0);
+                    const uint32_t o = ((kk >> 2) * Lay::kPanel + (kk & 3) * 32) >> 4;
+                    umma_ss(tmem + col, a + o, bd + o, idesc_s, kk > 0);
                 }
                 tc_commit(bar);
             };
             // dV += P^T dO, dK += dS^T Q: A from tensor memory (quarter u of the
             // queries at columns 32 u .. 32 u + 15, 8 per 16 queries), B MN-major
             // (+2048 B per 16 queries)
-            auto issue_acc = [&](int it, uint32_t col_acc, uint32_t col_a, uint32_t off_b) {
-                const uint64_t vb = umma_smem_desc(base + off_b + (it & 1) * Lay::kTile, Lay::kPanel,
-                                                   1024);
+            auto issue_acc = [&](bool first, uint32_t col_acc, uint32_t col_a, uint32_t off_b) {
+                const uint64_t vb = umma_smem_desc(base + off_b, Lay::kPanel, 1024);
 #pragma unroll
                 for (int kk = 0; kk < kTcBQ / 16; ++kk) {
                     const uint32_t ca = (kk >> 1) * 32 + (kk & 1) * 8;
                     umma_ts(tmem + col_acc, tmem + col_a + ca, vb + kk * (2048 >> 4), idesc_o,
-                            (it > 0 || kk > 0) ? 1u : 0u);
+                            (!first || kk > 0) ? 1u : 0u);
                 }
             };
-            // Issue order S(0) dP(0) | dV(0) | dK(0) S(1) dP(1) | dV(1) | ...: dV
-            // runs while the warps form dS^T, the next P^T is formed while dP
-            // runs, and a product always sits between the one that reads a
-            // tensor-memory region and the next one that overwrites it.
-            bool ok = wait(&kv_full, 0) && wait(&qo_full[0], 0);
+            auto q_off = [](int it) { return Lay::kOffQ + (it % kTcQStages) * Lay::kTile; };
+            auto o_off = [](int it) { return Lay::kOffO + (it % kTcOStages) * Lay::kTile; };
+            bool ok = wait(kv_full, 0) && wait(&q_full[0], 0);
             if (ok) {
                 tc_fence_after();
-                issue_s(0, Lay::kColS, dK, Lay::kOffQ, &s_full);
-                issue_s(0, Lay::kColP, dV, Lay::kOffO, &dp_full);
-            }
-            for (int it = 0; ok && it < n_items; ++it) {
-                if (!(ok = wait(&p_full, it & 1))) break;
-                tc_fence_after();
-                issue_acc(it, Lay::kColDV, Lay::kColS, Lay::kOffO);
-                if (!(ok = wait(&ds_full, it & 1))) break;
-                tc_fence_after();
-                issue_acc(it, Lay::kColDK, Lay::kColP, Lay::kOffQ);
-                tc_commit(&qo_empty[it & 1]);
-                if (it + 1 < n_items) {
-                    if (!(ok = wait(&qo_full[(it + 1) & 1], ((it + 1) >> 1) & 1))) break;
+                issue_s(Lay::kColS, dK, q_off(0), s_full);
+                if ((ok = wait(&o_full[0], 0))) {
                     tc_fence_after();
-                    issue_s(it + 1, Lay::kColS, dK, Lay::kOffQ, &s_full);
-                    issue_s(it + 1, Lay::kColP, dV, Lay::kOffO, &dp_full);
+                    issue_s(Lay::kColP, dV, o_off(0), dp_full);
                 }
             }
-            tc_commit(&acc_done);
-            mbar_wait(&acc_done, 0, &abort_flag, p.status, 1000000000ull);
+            for (int it = 0; ok && it < n_items; ++it) {
+                const bool more = it + 1 < n_items;
+                if (!(ok = wait(p_full, it & 1))) break;
+                tc_fence_after();
+                issue_acc(it == 0, Lay::kColDV, Lay::kColS, o_off(it));
+                tc_commit(&o_empty[it % kTcOStages]);
+                if (more) {
+                    const int n = it + 1;
+                    if (!(ok = wait(&q_full[n % kTcQStages], (n / kTcQStages) & 1))) break;
+                    tc_fence_after();
+                    issue_s(Lay::kColS, dK, q_off(n), s_full);
+                }
+                if (!(ok = wait(ds_full, it & 1))) break;
+                tc_fence_after();
+                issue_acc(it == 0, Lay::kColDK, Lay::kColP, q_off(it));
+                tc_commit(&q_empty[it % kTcQStages]);
+                if (more) {
+                    const int n = it + 1;
+                    if (!(ok = wait(&o_full[n % kTcOStages], (n / kTcOStages) & 1))) break;
+                    tc_fence_after();
+                    issue_s(Lay::kColP, dV, o_off(n), dp_full);
+                }
+            }
+            tc_commit(acc_done);
+            mbar_wait(acc_done, 0, abort_flag, p.status, 1000000000ull);
         }
-    } else if (warp >= 4) {
+        __syncwarp();
+    }
+    } else {
         // ---------------------------------------- elementwise + epilogue ----
         const int u = (warp - 4) >> 2;                  // query quarter of an item
         const int g4 = warp & 3;                        // lane group
         const int r = (g4 << 5) + lane;                 // key row = tensor-memory lane
         const int key = k0 + r;
         const uint32_t lane_addr = tmem + ((static_cast<uint32_t>(g4) * 32u) << 16);
+        const uint32_t col = 32 * u;
         bool ok = true;
         for (int it = 0; it < n_items; ++it) {
-            const int st = it & 1, q0 = (qb0 + it % n_qb) * kTcBQ;
-            // qo_full also publishes the item's lse / D the producer stored
+            const int q0 = (qb0 + it % n_qb) * kTcBQ;
+            const int qs = it % kTcQStages, db = it & 1;
+            // q_full also publishes the item's lse the producer stored
             if (!(ok = __all_sync(0xffffffffu,
-                                  mbar_wait(&qo_full[st], (it >> 1) & 1, &abort_flag, p.status) &&
-                                  mbar_wait(&s_full, it & 1, &abort_flag, p.status))))
+                                  mbar_wait(&q_full[qs], (it / kTcQStages) & 1, abort_flag,
+                                            p.status) &&
+                                  mbar_wait(s_full, it & 1, abort_flag, p.status))))
                 break;
             tc_fence_after();
-            const uint32_t col = 32 * u;
             uint32_t sv[32];
             tmem_ld32(lane_addr + Lay::kColS + col, sv);
             const bool full = block_visible(p.vis, q0, kTcBQ, k0, kTcBK);
             // the quarter's lse / D: the same 32 values for every lane (broadcast)
-            const float4 *L4 = reinterpret_cast<const float4 *>(sLD + st * 2 * kTcBQ + col);
-            const float4 *D4 = reinterpret_cast<const float4 *>(sLD + st * 2 * kTcBQ + kTcBQ + col);
+            const float4 *L4 = reinterpret_cast<const float4 *>(sL + qs * kTcBQ + col);
+            const float4 *D4 = reinterpret_cast<const float4 *>(sD + db * kTcBQ + col);
             tmem_wait_ld();
-            // P^T, over columns this thread has already read (its own quarter)
-            float pr[32];
+            // P^T, over columns this thread has already read (its own quarter);
+            // one pair in four takes 2^x on the FMA pipe (the MUFU unit is the
+            // busiest one here).  P^T is kept as the bf16 pairs the products use.
             uint32_t pk[16];
             const float2 cc = make_float2(p.scale_log2, p.scale_log2);
+            auto p_quad = [&](int e4, float (&pr)[4]) {
+                const float4 l4 = L4[e4];
+                const float2 x0 = fma2(make_float2(__uint_as_float(sv[4 * e4]),
+                                                   __uint_as_float(sv[4 * e4 + 1])),
+                                       cc, make_float2(-l4.x, -l4.y));
+                const float2 x1 = fma2(make_float2(__uint_as_float(sv[4 * e4 + 2]),
+                                                   __uint_as_float(sv[4 * e4 + 3])),
+                                       cc, make_float2(-l4.z, -l4.w));
+                const float2 e1 = (e4 & 1) ? exp2_poly2(x1)
+                                           : make_float2(fast_exp2(x1.x), fast_exp2(x1.y));
+                pr[0] = fast_exp2(x0.x);
+                pr[1] = fast_exp2(x0.y);
+                pr[2] = e1.x;
+                pr[3] = e1.y;
+            };
+            if (full) {
 #pragma unroll
-            for (int e2 = 0; e2 < 16; ++e2) {
-                const float2 l2 = reinterpret_cast<const float2 *>(L4)[e2];
-                const float2 x = fma2(make_float2(__uint_as_float(sv[2 * e2]),
-                                                  __uint_as_float(sv[2 * e2 + 1])),
-                                      cc, make_float2(-l2.x, -l2.y));
-                const float2 pe = make_float2(fast_exp2(x.x), fast_exp2(x.y));
-                pr[2 * e2] = pe.x;
-                pr[2 * e2 + 1] = pe.y;
-                if (!full) {
-                    if (!p.vis(q0 + col + 2 * e2, key)) pr[2 * e2] = 0.0f;
-                    if (!p.vis(q0 + col + 2 * e2 + 1, key)) pr[2 * e2 + 1] = 0.0f;
+                for (int e4 = 0; e4 < 8; ++e4) {
+                    float pr[4];
+                    p_quad(e4, pr);
+                    pk[2 * e4] = pack_bf16x2(pr[0], pr[1]);
+                    pk[2 * e4 + 1] = pack_bf16x2(pr[2], pr[3]);
                 }
-                pk[e2] = pack_bf16x2(pr[2 * e2], pr[2 * e2 + 1]);
+            } else {
+#pragma unroll
+                for (int e4 = 0; e4 < 8; ++e4) {
+                    float pr[4];
+                    p_quad(e4, pr);
+#pragma unroll
+                    for (int t = 0; t < 4; ++t)
+                        if (!p.vis(q0 + col + 4 * e4 + t, key)) pr[t] = 0.0f;
+                    pk[2 * e4] = pack_bf16x2(pr[0], pr[1]);
+                    pk[2 * e4 + 1] = pack_bf16x2(pr[2], pr[3]);
+                }
             }
             tmem_st16(lane_addr + Lay::kColS + col, pk);
             tmem_wait_st();
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&p_full);
+            if (lane == 0) mbar_arrive(p_full);
             // dS^T = P^T (dP^T - D), over the same columns of the dP^T region
-            if (!(ok = __all_sync(0xffffffffu, mbar_wait(&dp_full, it & 1, &abort_flag, p.status))))
+            if (!(ok = __all_sync(0xffffffffu,
+                                  mbar_wait(dp_full, it & 1, abort_flag, p.status) &&
+                                  mbar_wait(&d_full[db], (it >> 1) & 1, abort_flag, p.status))))
                 break;
             tc_fence_after();
             uint32_t dp[32];
             tmem_ld32(lane_addr + Lay::kColP + col, dp);
             tmem_wait_ld();
+            // dS^T from the bf16 P^T the dV product used (masked entries are 0)
             uint32_t dk[16];
 #pragma unroll
             for (int e4 = 0; e4 < 8; ++e4) {
                 const float4 d4 = D4[e4];
-                const float dv[4] = {d4.x, d4.y, d4.z, d4.w};
-                float ds[4];
-#pragma unroll
-                for (int t = 0; t < 4; ++t)
-                    ds[t] = pr[4 * e4 + t] * (__uint_as_float(dp[4 * e4 + t]) - dv[t]);
-                dk[2 * e4] = pack_bf16x2(ds[0], ds[1]);
-                dk[2 * e4 + 1] = pack_bf16x2(ds[2], ds[3]);
+                const float2 ds0 = mul2(bf16x2_to_float2(pk[2 * e4]),
+                                        add2(make_float2(__uint_as_float(dp[4 * e4]),
+                                                         __uint_as_float(dp[4 * e4 + 1])),
+                                             make_float2(-d4.x, -d4.y)));
+                const float2 ds1 = mul2(bf16x2_to_float2(pk[2 * e4 + 1]),
+                                        add2(make_float2(__uint_as_float(dp[4 * e4 + 2]),
+                                                         __uint_as_float(dp[4 * e4 + 3])),
+                                             make_float2(-d4.z, -d4.w)));
+                dk[2 * e4] = pack_bf16x2(ds0.x, ds0.y);
+                dk[2 * e4 + 1] = pack_bf16x2(ds1.x, ds1.y);
             }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&d_empty[db]);   // this warp is done with D
             tmem_st16(lane_addr + Lay::kColP + col, dk);
             tmem_wait_st();
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&ds_full);
+            if (lane == 0) mbar_arrive(ds_full);
         }
         // ---- epilogue: dV, dK * scale -> bf16 (quarter u writes columns 32 u ..) ----
         if (ok && n_items > 0)
-            ok = __all_sync(0xffffffffu, mbar_wait(&acc_done, 0, &abort_flag, p.status));
+            ok = __all_sync(0xffffffffu, mbar_wait(acc_done, 0, abort_flag, p.status));
         tc_fence_after();
         // the tensor-memory loads are warp-collective: every lane loads, and
         // only rows of real keys are stored
@@ -480,8 +579,12 @@ static int launch_dkdv_tc(const void *q, const void *k, const void *v, const voi
 // Once the warps hold S(j) and dP(j) in registers the next tile's S and dP are
 // computed, overlapping the elementwise work; the warps write dS(j) after
 // dQ(j-1) has read dS(j-1).  Tensor memory: S | dP | dQ | dS.  Shared memory:
-// Q, dO, 2-deep K and V rings.
+// Q, dO, a 3-deep K ring (K(j) serves S(j) and, a tile later, dQ(j), so the
+// copy of K(j+2) must not wait for dQ(j)) and a 2-deep V ring (V(j) is free
+// once dP(j) has run).
 constexpr int kDqBN = 128;       // keys per tile
+constexpr int kDqKStages = 3;
+constexpr int kDqVStages = 2;
 
 template <int D>
 struct DqLayout {
@@ -489,9 +592,9 @@ struct DqLayout {
     static constexpr int kPanel = 128 * 128;               // 128 rows x 64 bf16
     static constexpr int kTile = kPanels * kPanel;
     static constexpr int kOffQ = 0, kOffO = kTile;
-    static constexpr int kOffK = 2 * kTile;                // [2]
-    static constexpr int kOffV = kOffK + 2 * kTile;        // [2]
-    static constexpr int kBytes = kOffV + 2 * kTile;
+    static constexpr int kOffK = 2 * kTile;                // [kDqKStages]
+    static constexpr int kOffV = kOffK + kDqKStages * kTile;   // [kDqVStages]
+    static constexpr int kBytes = kOffV + kDqVStages * kTile;
     static constexpr int kSmemBytes = kBytes + 1024;
     // S | dP | dQ | dS (bf16, keys 32 u .. 32 u + 31 at 384 + 16 u)
     static constexpr uint32_t kColS = 0, kColP = 128, kColDQ = 256, kColDS = 384;
@@ -516,8 +619,8 @@ dq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-    __shared__ uint64_t qo_full, kv_full[2], kv_empty[2], s_full, s_free, p_full, dq_done,
-        acc_done;
+    __shared__ uint64_t qo_full, k_full[kDqKStages], k_empty[kDqKStages], v_full[kDqVStages],
+        v_empty[kDqVStages], s_full, s_free, p_full, dq_done, acc_done;
     __shared__ uint32_t tmem_base_sh;
     __shared__ int abort_flag;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -541,9 +644,13 @@ dq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
 
     if (threadIdx.x == 0) {
         mbar_init(&qo_full, 1);
-        for (int s = 0; s < 2; ++s) {
-            mbar_init(&kv_full[s], 1);
-            mbar_init(&kv_empty[s], 1);
+        for (int s = 0; s < kDqKStages; ++s) {
+            mbar_init(&k_full[s], 1);
+            mbar_init(&k_empty[s], 1);
+        }
+        for (int s = 0; s < kDqVStages; ++s) {
+            mbar_init(&v_full[s], 1);
+            mbar_init(&v_empty[s], 1);
         }
         mbar_init(&s_full, 1);
         mbar_init(&s_free, kTcElemWarps);
@@ -579,29 +686,42 @@ dq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
                 }
             }
             __syncwarp();
-            int issued = 0;
+            int issued_k = 0, issued_v = 0;
             for (int j = 0; j < n_kv; ++j) {
-                const int st = j & 1;
-                if (!__all_sync(0xffffffffu, mbar_wait(&kv_empty[st], ((j >> 1) & 1) ^ 1,
-                                                       &abort_flag, p.status)))
+                const int row = tile_of(j) * kDqBN;
+                const int ks = j % kDqKStages, kph = (j / kDqKStages) & 1;
+                const int vs = j % kDqVStages, vph = (j / kDqVStages) & 1;
+                if (!__all_sync(0xffffffffu,
+                                mbar_wait(&k_empty[ks], kph ^ 1, &abort_flag, p.status)))
                     break;
                 if (leader) {
-                    mbar_expect_tx(&kv_full[st], 2 * Lay::kTile);
-                    const int row = tile_of(j) * kDqBN;
-                    for (int pn = 0; pn < Lay::kPanels; ++pn) {
-                        tma_load_4d(smem + Lay::kOffK + st * Lay::kTile + pn * Lay::kPanel, &tm_k,
-                                    &kv_full[st], pn * 64, kvh, row, b);
-                        tma_load_4d(smem + Lay::kOffV + st * Lay::kTile + pn * Lay::kPanel, &tm_v,
-                                    &kv_full[st], pn * 64, kvh, row, b);
-                    }
+                    mbar_expect_tx(&k_full[ks], Lay::kTile);
+                    for (int pn = 0; pn < Lay::kPanels; ++pn)
+                        tma_load_4d(smem + Lay::kOffK + ks * Lay::kTile + pn * Lay::kPanel, &tm_k,
+                                    &k_full[ks], pn * 64, kvh, row, b);
                 }
                 __syncwarp();
-                issued = j + 1;
+                issued_k = j + 1;
+                if (!__all_sync(0xffffffffu,
+                                mbar_wait(&v_empty[vs], vph ^ 1, &abort_flag, p.status)))
+                    break;
+                if (leader) {
+                    mbar_expect_tx(&v_full[vs], Lay::kTile);
+                    for (int pn = 0; pn < Lay::kPanels; ++pn)
+                        tma_load_4d(smem + Lay::kOffV + vs * Lay::kTile + pn * Lay::kPanel, &tm_v,
+                                    &v_full[vs], pn * 64, kvh, row, b);
+                }
+                __syncwarp();
+                issued_v = j + 1;
             }
             // copies still in flight land before the block exits
             mbar_wait(&qo_full, 0, &abort_flag, p.status, 1000000ull);
-            for (int j = max(0, issued - 2); j < issued; ++j)
-                mbar_wait(&kv_full[j & 1], (j >> 1) & 1, &abort_flag, p.status, 1000000ull);
+            for (int j = max(0, issued_k - kDqKStages); j < issued_k; ++j)
+                mbar_wait(&k_full[j % kDqKStages], (j / kDqKStages) & 1, &abort_flag, p.status,
+                          1000000ull);
+            for (int j = max(0, issued_v - kDqVStages); j < issued_v; ++j)
+                mbar_wait(&v_full[j % kDqVStages], (j / kDqVStages) & 1, &abort_flag, p.status,
+                          1000000ull);
         }
     } else if (warp == 1 && lane == 0) {
         // ------------------------------------------------- MMA issuer ----
@@ -614,29 +734,33 @@ dq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
             auto wait = [&](uint64_t *bar, uint32_t parity) {
                 return mbar_wait(bar, parity, &abort_flag, p.status);
             };
-            // S = Q K_j^T, dP = dO V_j^T: K-major A and B (+32 B per 16 of d)
+            // S = Q K_j^T, dP = dO V_j^T: K-major A and B (+32 B per 16 of d);
+            // V_j's stage is released as soon as dP has run
             auto issue_s = [&](int j) {
-                const int st = j & 1;
-                if (!wait(&kv_full[st], (j >> 1) & 1)) return false;
+                const int ks = j % kDqKStages, vs = j % kDqVStages;
+                if (!wait(&k_full[ks], (j / kDqKStages) & 1)) return false;
                 tc_fence_after();
-                const uint64_t bk = umma_smem_desc(base + Lay::kOffK + st * Lay::kTile, 16, 1024);
-                const uint64_t bv = umma_smem_desc(base + Lay::kOffV + st * Lay::kTile, 16, 1024);
+                const uint64_t bk = umma_smem_desc(base + Lay::kOffK + ks * Lay::kTile, 16, 1024);
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
                     const uint32_t o16 = ((kk >> 2) * Lay::kPanel + (kk & 3) * 32) >> 4;
                     umma_ss(tmem + Lay::kColS, dQt + o16, bk + o16, idesc_s, kk > 0);
                 }
+                if (!wait(&v_full[vs], (j / kDqVStages) & 1)) return false;
+                tc_fence_after();
+                const uint64_t bv = umma_smem_desc(base + Lay::kOffV + vs * Lay::kTile, 16, 1024);
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
                     const uint32_t o16 = ((kk >> 2) * Lay::kPanel + (kk & 3) * 32) >> 4;
                     umma_ss(tmem + Lay::kColP, dOt + o16, bv + o16, idesc_s, kk > 0);
                 }
                 tc_commit(&s_full);
+                tc_commit(&v_empty[vs]);
                 return true;
             };
             bool ok = wait(&qo_full, 0) && issue_s(0);
             for (int j = 0; ok && j < n_kv; ++j) {
-                const int st = j & 1;
+                const int ks = j % kDqKStages;
                 // the warps hold S(j), dP(j) in registers: the next tile's may be written
                 if (!(ok = wait(&s_free, j & 1))) break;
                 if (j + 1 < n_kv && !(ok = issue_s(j + 1))) break;
@@ -645,13 +769,13 @@ dq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
                 // dQ += dS K: dS from tensor memory (keys 32 u .. at 384 + 16 u,
                 // 8 columns per 16 keys), K MN-major (+2048 B per 16 keys)
                 const uint64_t km =
-                    umma_smem_desc(base + Lay::kOffK + st * Lay::kTile, Lay::kPanel, 1024);
+                    umma_smem_desc(base + Lay::kOffK + ks * Lay::kTile, Lay::kPanel, 1024);
 #pragma unroll
                 for (int kk = 0; kk < kDqBN / 16; ++kk)
                     umma_ts(tmem + Lay::kColDQ, tmem + Lay::kColDS + kk * 8, km + kk * (2048 >> 4),
                             idesc_o, (j > 0 || kk > 0) ? 1u : 0u);
                 tc_commit(&dq_done);
-                tc_commit(&kv_empty[st]);
+                tc_commit(&k_empty[ks]);
             }
             tc_commit(&acc_done);
             mbar_wait(&acc_done, 0, &abort_flag, p.status, 1000000000ull);
@@ -683,22 +807,39 @@ dq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
             const int key0 = tile_of(j) * kDqBN + col;
             const bool full = block_visible(p.vis, t0, p.P, tile_of(j) * kDqBN, kDqBN) &&
                               __all_sync(0xffffffffu, row_real || r >= p.P * p.G);
+            // dS = P (dP - D); one pair in four takes 2^x on the FMA pipe (the MUFU
+            // unit is the busiest one here).  Tiles the mask leaves whole skip the
+            // per-element test.
             uint32_t pk[16];
             const float2 cc = make_float2(p.scale_log2, p.scale_log2), nl = make_float2(-Lr, -Lr);
-#pragma unroll
-            for (int e = 0; e < 32; e += 2) {
+            const float2 nd = make_float2(-Dr, -Dr);
+            auto ds_pair = [&](int e) {
                 const float2 x = fma2(make_float2(__uint_as_float(sv[e]), __uint_as_float(sv[e + 1])),
                                       cc, nl);
-                const float2 pr = make_float2(fast_exp2(x.x), fast_exp2(x.y));
-                float ds[2] = {pr.x * (__uint_as_float(dp[e]) - Dr),
-                               pr.y * (__uint_as_float(dp[e + 1]) - Dr)};
+                const float2 pr = ((e >> 1) & 3) == 3 ? exp2_poly2(x)
+                                                      : make_float2(fast_exp2(x.x), fast_exp2(x.y));
+                return mul2(pr, add2(make_float2(__uint_as_float(dp[e]), __uint_as_float(dp[e + 1])),
+                                     nd));
+            };
+            if (full) {
 #pragma unroll
-                for (int t = 0; t < 2; ++t) {
-                    const bool vis = row_real && (full || p.vis(pos, key0 + e + t));
-                    // rows past the tile's real ones hold stale operands: exact zeros
-                    if (!vis) ds[t] = 0.0f;
+                for (int e = 0; e < 32; e += 2) {
+                    const float2 ds = ds_pair(e);
+                    pk[e / 2] = pack_bf16x2(ds.x, ds.y);
                 }
-                pk[e / 2] = pack_bf16x2(ds[0], ds[1]);
+                // rows past the tile's real ones hold stale operands: exact zeros
+                if (!row_real) {
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) pk[e] = 0u;
+                }
+            } else {
+#pragma unroll
+                for (int e = 0; e < 32; e += 2) {
+                    float2 ds = ds_pair(e);
+                    if (!(row_real && p.vis(pos, key0 + e))) ds.x = 0.0f;
+                    if (!(row_real && p.vis(pos, key0 + e + 1))) ds.y = 0.0f;
+                    pk[e / 2] = pack_bf16x2(ds.x, ds.y);
+                }
             }
             // dQ(j-1) has read the dS region
             if (j > 0 && !(ok = __all_sync(0xffffffffu, mbar_wait(&dq_done, (j - 1) & 1,
