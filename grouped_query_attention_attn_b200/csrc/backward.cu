@@ -669,13 +669,16 @@ dq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
     tc_fence_after();
     const uint32_t tmem = tmem_base_sh;
 
-    if (warp == 0) {
-        // ------------------------------------------------ TMA producer ----
+    if (warp == 0 || warp == 2) {
+        // ---------------------------------------------- TMA producers ----
+        // Warp 0 loads Q, dO and the K ring, warp 2 the V ring: each waits only
+        // on its own ring's releases (K(j) is held until dQ(j), V(j) only
+        // until dP(j)), so a late K stage never holds back a V copy.
         const bool leader = elect_one();
+        const bool is_k = warp == 0;
         if (n_kv > 0) {
-            if (leader) {
+            if (leader && is_k) {
                 tma_prefetch_desc(&tm_k);
-                tma_prefetch_desc(&tm_v);
                 const uint32_t box = 64u * p.G * p.P * 2u;
                 mbar_expect_tx(&qo_full, 2 * Lay::kPanels * box);
                 for (int pn = 0; pn < Lay::kPanels; ++pn) {
@@ -685,43 +688,30 @@ dq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
                                 kvh * p.G, t0, b);
                 }
             }
+            if (leader && !is_k) tma_prefetch_desc(&tm_v);
             __syncwarp();
-            int issued_k = 0, issued_v = 0;
+            const int stages = is_k ? kDqKStages : kDqVStages;
+            uint64_t *full = is_k ? k_full : v_full, *empty = is_k ? k_empty : v_empty;
+            const CUtensorMap *tm = is_k ? &tm_k : &tm_v;
+            const int off0 = is_k ? Lay::kOffK : Lay::kOffV;
+            int issued = 0;
             for (int j = 0; j < n_kv; ++j) {
-                const int row = tile_of(j) * kDqBN;
-                const int ks = j % kDqKStages, kph = (j / kDqKStages) & 1;
-                const int vs = j % kDqVStages, vph = (j / kDqVStages) & 1;
-                if (!__all_sync(0xffffffffu,
-                                mbar_wait(&k_empty[ks], kph ^ 1, &abort_flag, p.status)))
+                const int st = j % stages, ph = (j / stages) & 1;
+                if (!__all_sync(0xffffffffu, mbar_wait(&empty[st], ph ^ 1, &abort_flag, p.status)))
                     break;
                 if (leader) {
-                    mbar_expect_tx(&k_full[ks], Lay::kTile);
+                    mbar_expect_tx(&full[st], Lay::kTile);
                     for (int pn = 0; pn < Lay::kPanels; ++pn)
-                        tma_load_4d(smem + Lay::kOffK + ks * Lay::kTile + pn * Lay::kPanel, &tm_k,
-                                    &k_full[ks], pn * 64, kvh, row, b);
+                        tma_load_4d(smem + off0 + st * Lay::kTile + pn * Lay::kPanel, tm, &full[st],
+                                    pn * 64, kvh, tile_of(j) * kDqBN, b);
                 }
                 __syncwarp();
-                issued_k = j + 1;
-                if (!__all_sync(0xffffffffu,
-                                mbar_wait(&v_empty[vs], vph ^ 1, &abort_flag, p.status)))
-                    break;
-                if (leader) {
-                    mbar_expect_tx(&v_full[vs], Lay::kTile);
-                    for (int pn = 0; pn < Lay::kPanels; ++pn)
-                        tma_load_4d(smem + Lay::kOffV + vs * Lay::kTile + pn * Lay::kPanel, &tm_v,
-                                    &v_full[vs], pn * 64, kvh, row, b);
-                }
-                __syncwarp();
-                issued_v = j + 1;
+                issued = j + 1;
             }
             // copies still in flight land before the block exits
-            mbar_wait(&qo_full, 0, &abort_flag, p.status, 1000000ull);
-            for (int j = max(0, issued_k - kDqKStages); j < issued_k; ++j)
-                mbar_wait(&k_full[j % kDqKStages], (j / kDqKStages) & 1, &abort_flag, p.status,
-                          1000000ull);
-            for (int j = max(0, issued_v - kDqVStages); j < issued_v; ++j)
-                mbar_wait(&v_full[j % kDqVStages], (j / kDqVStages) & 1, &abort_flag, p.status,
-                          1000000ull);
+            if (is_k) mbar_wait(&qo_full, 0, &abort_flag, p.status, 1000000ull);
+            for (int j = max(0, issued - stages); j < issued; ++j)
+                mbar_wait(&full[j % stages], (j / stages) & 1, &abort_flag, p.status, 1000000ull);
         }
     } else if (warp == 1 && lane == 0) {
         // ------------------------------------------------- MMA issuer ----
