@@ -49,8 +49,10 @@ def test_wide_window_equals_causal(gqa_lib):
     assert torch.equal(gqa.attn(*args, causal=True), gqa.attn(*args, causal=True, window=333))
 
 
+# windows that take 512-, 768- and 1024-key splits (Lmax = 3000)
 @pytest.mark.parametrize("Hq,Hkv,window,sinks", [(8, 2, 300, 0), (32, 8, 1000, 4),
-                                                 (8, 1, 64, 2000), (16, 2, 1, 1), (8, 2, 2100, 3)])
+                                                 (8, 1, 64, 2000), (16, 2, 1, 1), (8, 2, 2100, 3),
+                                                 (8, 2, 4000, 2)])
 def test_decode_window(gqa_lib, Hq, Hkv, window, sinks):
     lengths = [1, 15, 700, 1023, 1024, 1025, 2500, 0, 3000, 129]
     q, kc, vc, sl = workloads.decode_inputs(len(lengths), Hq, Hkv, 128, 1, 3000, lengths=lengths,
