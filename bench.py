@@ -567,6 +567,10 @@ def run_ours(args, world, rank, local):
                     "launch_ms": launch_ms}
         roofline["frac"] = roofline["achieved"] / roofline["peak"]
         roofline["frac_of_nominal_2250"] = roofline["achieved"] / 2250.0
+        # time x median SM clock under load: the launch in SM cycles, which
+        # separates a slow kernel from a slow clock
+        if clocks.get("sm_mhz"):
+            roofline["sm_cycles_per_launch"] = launch_ms * 1e3 * clocks["sm_mhz"]
 
         # ---- end to end through host buffers (the headline metric) ----
         if not args.no_e2e:
@@ -627,6 +631,8 @@ def run_ours(args, world, rank, local):
                     "kernels": "decode_split_kernel<128,1> (split merge fused)"}
         dec_roof["frac"] = dec_roof["achieved"] / dec_roof["peak"]
         dec_roof["frac_of_nominal_8000"] = dec_roof["achieved"] / 8000.0
+        if clocks.get("sm_mhz"):
+            dec_roof["sm_cycles_per_launch"] = launch_ms * 1e3 * clocks["sm_mhz"]
         dec = {"value": world * d_bytes * K / (dec_ms / 1e3) / 1e9, "unit": "GB/s",
                "roofline": dec_roof}
 

@@ -184,7 +184,7 @@ int gqa_decode(const void *q, const void *k_cache, const void *v_cache,
 
 /*
  * gqa_decode_rope -- gqa_decode with rotary position embedding applied to the
- * query as it is loaded (course step 3): sequence b's new token sits at
+ * query as it is loaded (course "Неделя 7. Внимание", step 3): sequence b's new token sits at
  * position max(seqlens[b] - 1, 0), as for gqa_rope_decode_q; q in memory is
  * not modified and the cached keys must already be rotated.  The result
  * equals gqa_rope_decode_q followed by gqa_decode bit for bit.  theta > 0 and
@@ -197,7 +197,7 @@ int gqa_decode_rope(const void *q, const void *k_cache, const void *v_cache,
 
 /*
  * gqa_decode_window -- gqa_decode with a sliding window and attention sinks
- * (course step 3): the newest token of sequence b sees cache rows
+ * (course "Неделя 7. Внимание", step 3): the newest token of sequence b sees cache rows
  * j >= seqlens[b] - window and rows j < sinks.  window >= 1, sinks >= 0;
  * everything else (layouts, workspace and its size, errors) as gqa_decode.
  * The KV splits start at the window's first row, and split 0 also reads the
@@ -311,7 +311,8 @@ int gqa_rope_decode_q(void *q, const int32_t *seqlens, int B, int H, int d, floa
 
 /*
  * gqa_fold_kv -- MHA -> GQA conversion of a K or V tensor by mean pooling
- * (TT Lab step 2, course step 2: average the heads of each contiguous group).
+ * (TT Lab "キー・バリューヘッドだけ減らしてみる", step 2; course "Неделя 7. Внимание",
+ * step 2: average the heads of each contiguous group).
  *   in  [B, T, H, d] bf16, out [B, T, g, d] bf16 (written), H % g == 0.
  * Members of a group are added in head order in fp32, divided by H/g in fp32
  * and rounded to bf16 (nearest even).  d must be a multiple of 8 and both
@@ -347,7 +348,7 @@ int gqa_selftest_wait_timeout(int timeout_us);
 /*
  * gqa_selftest_exp2_poly -- evaluates, on the GPU, the FMA-pipe 2^x
  * polynomial the prefill softmax uses for part of its exponentials (the
- * max-subtracted softmax of TT Lab step 4 / course step 1 needs
+ * max-subtracted softmax of the TT Lab page, step 4, and the course page, step 1, needs
  * exp(s - m) = 2^((s - m) log2 e)): y[i] = poly 2^x[i] for n points (n even,
  * x and y device float arrays, 4-byte aligned).  Range reduction
  * x = n + f, f in [-1/2, 1/2], a degree-3 minimax fit of 2^f (relative error
