@@ -1,17 +1,22 @@
 // host_pipeline.cu -- attention forward on host-resident q / k / v / o.
 //
-// The host <-> device copies are the long pole (PCIe moves ~50 GB/s, the
-// prefill kernel reads the same bytes at several TB/s), so the query
-// positions are cut into chunks and three queues overlap: chunk c's q rows and
-// the k / v rows it newly needs go up on one copy stream while chunk c - 1's
-// attention runs on the caller's stream and chunk c - 2's o comes down on a
-// second copy stream.  With a causal mask chunk c needs keys [0, last row of
-// c + Tkv - Tq], so k / v travel in the same chunks as q.  Each chunk's
-// attention is the prefill kernel on views of the staging buffers (bottom-right
-// alignment makes a chunk of rows against its key prefix exactly the same
-// computation as in the whole problem).  With a completion event the caller's
-// stream is not held for the copies down, so the next call's copies up start
-// when this call's attention is done and overlap this call's copies down.
+// The host <-> device copies are the long pole (PCIe moves ~55 GB/s each way,
+// the prefill kernel reads the same bytes at several TB/s), so three queues
+// overlap: k and v go up whole first, then the query positions in chunks on
+// one copy stream, while the previous chunk's attention runs on the caller's
+// stream and the chunk before's o comes down on a second copy stream.  Each
+// chunk's attention is the prefill kernel on views of the staging buffers
+// (bottom-right alignment makes a chunk of rows against its key prefix exactly
+// the same computation as in the whole problem).  The chunks go last rows
+// first: with a causal mask the last rows see the most keys, and the chunk
+// that ends a call sets how long the next call's copies up wait for this
+// call's attention (they overwrite the staging buffers it reads).  With a
+// completion event the caller's stream is not held for the copies down, so
+// the next call's copies up overlap this call's copies down.
+// Measured on one B200 host (PCIe: 55 GB/s up, 57 down, 0.96 ms for one
+// step's 50 MB up and 34 MB down together), causal T = 4096, 32 / 8 heads:
+// 8 chunks with k / v in step 1.35 ms per call, 4 chunks with k / v first
+// 1.19 ms, the same last rows first 1.15 ms.
 #include <mutex>
 
 #include "internal.h"
@@ -85,8 +90,9 @@ int launch_fwd_host_pipeline(const void *q_host, const void *k_host, const void 
     PipeRes *r = nullptr;
     if (int rc = pipe_res(dev, ctx_id, &r)) return rc;
 
-    // chunks of at least 256 rows, at most kMaxChunks of them
-    int rows = (Tq + 7) / 8;
+    // 4 chunks of at least 256 rows (fewer chunks measured faster: each one
+    // adds a launch and two cross-stream waits)
+    int rows = (Tq + 3) / 4;
     if (rows < 256) rows = 256;
     if ((Tq + rows - 1) / rows > kMaxChunks) rows = (Tq + kMaxChunks - 1) / kMaxChunks;
     const int n_chunks = (Tq + rows - 1) / rows;
@@ -102,25 +108,21 @@ int launch_fwd_host_pipeline(const void *q_host, const void *k_host, const void 
     // and o_dev may still be on its way down from the previous call
     if (int rc = check_cuda(cudaStreamWaitEvent(stream, ev_done, 0), "cudaStreamWaitEvent"))
         return rc;
-    int kv_have = 0;
-    for (int c = 0; c < n_chunks; ++c) {
+    // ---- up: all of k and v ----
+    if (int rc = copy_rows(k_dev, k_host, B, Tkv, Hkv, d, 0, Tkv, cudaMemcpyHostToDevice, r->up))
+        return rc;
+    if (int rc = copy_rows(v_dev, v_host, B, Tkv, Hkv, d, 0, Tkv, cudaMemcpyHostToDevice, r->up))
+        return rc;
+    for (int cc = 0; cc < n_chunks; ++cc) {
+        const int c = n_chunks - 1 - cc;            // last rows first
         const int a = c * rows, b = a + rows < Tq ? a + rows : Tq;
         int kv_need = Tkv;
         if (causal) {
             kv_need = b + (Tkv - Tq);
             kv_need = kv_need < 0 ? 0 : (kv_need > Tkv ? Tkv : kv_need);
         }
-        cudaEvent_t ev_in = r->ev[2 * c], ev_out = r->ev[2 * c + 1];
-        // ---- up: the rows this chunk adds ----
-        if (kv_need > kv_have) {
-            if (int rc = copy_rows(k_dev, k_host, B, Tkv, Hkv, d, kv_have, kv_need,
-                                   cudaMemcpyHostToDevice, r->up))
-                return rc;
-            if (int rc = copy_rows(v_dev, v_host, B, Tkv, Hkv, d, kv_have, kv_need,
-                                   cudaMemcpyHostToDevice, r->up))
-                return rc;
-            kv_have = kv_need;
-        }
+        cudaEvent_t ev_in = r->ev[2 * cc], ev_out = r->ev[2 * cc + 1];
+        // ---- up: this chunk's q rows ----
         if (int rc = copy_rows(q_dev, q_host, B, Tq, Hq, d, a, b, cudaMemcpyHostToDevice, r->up))
             return rc;
         if (int rc = check_cuda(cudaEventRecord(ev_in, r->up), "cudaEventRecord")) return rc;
@@ -147,7 +149,6 @@ int launch_fwd_host_pipeline(const void *q_host, const void *k_host, const void 
         if (int rc = copy_rows(o_host, o_dev, B, Tq, Hq, d, a, b, cudaMemcpyDeviceToHost, r->down))
             return rc;
     }
-    // every key row went up with some chunk (the last one needs all of them)
     if (int rc = check_cuda(cudaEventRecord(ev_done, r->down), "cudaEventRecord")) return rc;
     if (done) return check_cuda(cudaEventRecord(done, r->down), "cudaEventRecord");
     // without a completion event the caller's stream completes once o is back
