@@ -14,7 +14,7 @@ pytestmark = pytest.mark.gpu
 
 
 @pytest.mark.parametrize("B,Tq,Tkv,Hq,Hkv,d,causal", [
-    (1, 3000, 3000, 8, 2, 128, True),      # 8 chunks of 375 rows, ragged end
+    (1, 3000, 3000, 8, 2, 128, True),      # 4 chunks of 750 rows, last rows first
     (2, 700, 700, 8, 2, 128, True),        # B = 2: strided copies
     (1, 1000, 300, 8, 2, 128, True),       # Tq > Tkv: leading chunks see no key
     (2, 300, 1000, 4, 1, 64, True),        # Tq < Tkv
@@ -69,9 +69,33 @@ def test_host_forward_with_completion_event(gqa_lib):
         assert max_abs(o, o_ref) <= BF16_TOL
 
 
+def test_host_forward_alternating_staging(gqa_lib):
+    # consecutive overlapped calls alternating two staging sets, then a third,
+    # larger set, then a set that is a view into it, with the shapes changing in
+    # between: every output against the oracle
+    specs = [(2, 800, 8, 2, 128), (2, 800, 8, 2, 128), (2, 800, 8, 2, 128),
+             (1, 1700, 8, 2, 128), (2, 800, 8, 2, 128)]
+    inputs = [workloads.prefill_inputs(B, T, Hq, Hkv, d, seeds=(41 + 3 * i, 42 + 3 * i, 43 + 3 * i))
+              for i, (B, T, Hq, Hkv, d) in enumerate(specs)]
+    pinned = [tuple(t.pin_memory() for t in x) for x in inputs]
+    big = gqa.host_staging(inputs[3][0], inputs[3][1])
+    sets = [gqa.host_staging(inputs[0][0], inputs[0][1]) for _ in range(2)]
+    # a set that is a view into the big one overlaps it
+    view = tuple(t.view(-1)[: s.numel()].view(s.shape) for t, s in zip(big, sets[0]))
+    order = [sets[0], sets[1], sets[0], big, view]
+    outs = [torch.empty(x[0].shape, dtype=torch.bfloat16).pin_memory() for x in inputs]
+    events = [torch.cuda.Event() for _ in inputs]
+    for (q, k, v), o, st, ev in zip(pinned, outs, order, events):
+        gqa.attn_host(q, k, v, out=o, staging=st, done=ev)
+    for (q, k, v), o, ev in zip(inputs, outs, events):
+        ev.synchronize()
+        o_ref, _ = ref.attn_fwd(q, k, v, True)
+        assert max_abs(o, o_ref) <= BF16_TOL
+
+
 def test_host_forward_headline_shape(gqa_lib):
     # the end-to-end path the bench times: causal B=1, T=4096, 32 / 8 heads from
-    # pinned host tensors (16 chunks of 256 rows), sampled rows against the oracle
+    # pinned host tensors (4 chunks of 1024 rows), sampled rows against the oracle
     q, k, v = workloads.prefill_inputs(1, 4096, 32, 8, 128)
     qp, kp, vp = q.pin_memory(), k.pin_memory(), v.pin_memory()
     o = gqa.attn_host(qp, kp, vp, causal=True)
