@@ -620,7 +620,7 @@ dq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
     uint8_t *smem = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
     __shared__ uint64_t qo_full, k_full[kDqKStages], k_empty[kDqKStages], v_full[kDqVStages],
-        v_empty[kDqVStages], s_full, s_free, p_full, dq_done, acc_done;
+        v_empty[kDqVStages], s_full, s_free, p_full, dq_done, acc_done, s_drain;
     __shared__ uint32_t tmem_base_sh;
     __shared__ int abort_flag;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -657,6 +657,7 @@ dq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
         mbar_init(&p_full, kTcElemWarps);
         mbar_init(&dq_done, 1);
         mbar_init(&acc_done, 1);
+        mbar_init(&s_drain, 1);
         abort_flag = 0;
         fence_mbar_init();
     }
@@ -713,8 +714,14 @@ dq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
             for (int j = max(0, issued - stages); j < issued; ++j)
                 mbar_wait(&full[j % stages], (j / stages) & 1, &abort_flag, p.status, 1000000ull);
         }
-    } else if (warp == 1 && lane == 0) {
-        // ------------------------------------------------- MMA issuer ----
+    } else if ((warp == 1 || warp == 3) && lane == 0) {
+        // ------------------------------------------------ MMA issuers ----
+        // Warp 1 issues S and dP, warp 3 issues dQ.  The two streams touch
+        // disjoint tensor-memory regions (S | dP against dQ, reading dS) and
+        // shared-memory stages released through their own barriers, so they need
+        // no order between them; with one issuer a dQ(j) whose dS was ready sat
+        // behind the whole S / dP(j+1) group (tcgen05.mma blocks the issuing
+        // thread once its queue is full), and S / dP(j+2) behind dQ(j).
         if (n_kv > 0) {
             constexpr uint32_t idesc_s = umma_idesc_bf16(128, kDqBN, 0, 0);
             constexpr uint32_t idesc_o = umma_idesc_bf16(128, D, 0, 1);
@@ -724,51 +731,62 @@ dq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
             auto wait = [&](uint64_t *bar, uint32_t parity) {
                 return mbar_wait(bar, parity, &abort_flag, p.status);
             };
-            // S = Q K_j^T, dP = dO V_j^T: K-major A and B (+32 B per 16 of d);
-            // V_j's stage is released as soon as dP has run
-            auto issue_s = [&](int j) {
-                const int ks = j % kDqKStages, vs = j % kDqVStages;
-                if (!wait(&k_full[ks], (j / kDqKStages) & 1)) return false;
-                tc_fence_after();
-                const uint64_t bk = umma_smem_desc(base + Lay::kOffK + ks * Lay::kTile, 16, 1024);
+            if (warp == 1) {
+                // S = Q K_j^T, dP = dO V_j^T: K-major A and B (+32 B per 16 of d);
+                // V_j's stage is released as soon as dP has run
+                auto issue_s = [&](int j) {
+                    const int ks = j % kDqKStages, vs = j % kDqVStages;
+                    if (!wait(&k_full[ks], (j / kDqKStages) & 1)) return false;
+                    tc_fence_after();
+                    const uint64_t bk =
+                        umma_smem_desc(base + Lay::kOffK + ks * Lay::kTile, 16, 1024);
 #pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint32_t o16 = ((kk >> 2) * Lay::kPanel + (kk & 3) * 32) >> 4;
-                    umma_ss(tmem + Lay::kColS, dQt + o16, bk + o16, idesc_s, kk > 0);
-                }
-                if (!wait(&v_full[vs], (j / kDqVStages) & 1)) return false;
-                tc_fence_after();
-                const uint64_t bv = umma_smem_desc(base + Lay::kOffV + vs * Lay::kTile, 16, 1024);
+                    for (int kk = 0; kk < D / 16; ++kk) {
+                        const uint32_t o16 = ((kk >> 2) * Lay::kPanel + (kk & 3) * 32) >> 4;
+                        umma_ss(tmem + Lay::kColS, dQt + o16, bk + o16, idesc_s, kk > 0);
+                    }
+                    if (!wait(&v_full[vs], (j / kDqVStages) & 1)) return false;
+                    tc_fence_after();
+                    const uint64_t bv =
+                        umma_smem_desc(base + Lay::kOffV + vs * Lay::kTile, 16, 1024);
 #pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint32_t o16 = ((kk >> 2) * Lay::kPanel + (kk & 3) * 32) >> 4;
-                    umma_ss(tmem + Lay::kColP, dOt + o16, bv + o16, idesc_s, kk > 0);
-                }
-                tc_commit(&s_full);
-                tc_commit(&v_empty[vs]);
-                return true;
-            };
-            bool ok = wait(&qo_full, 0) && issue_s(0);
-            for (int j = 0; ok && j < n_kv; ++j) {
-                const int ks = j % kDqKStages;
+                    for (int kk = 0; kk < D / 16; ++kk) {
+                        const uint32_t o16 = ((kk >> 2) * Lay::kPanel + (kk & 3) * 32) >> 4;
+                        umma_ss(tmem + Lay::kColP, dOt + o16, bv + o16, idesc_s, kk > 0);
+                    }
+                    tc_commit(&s_full);
+                    tc_commit(&v_empty[vs]);
+                    return true;
+                };
+                bool ok = wait(&qo_full, 0) && issue_s(0);
                 // the warps hold S(j), dP(j) in registers: the next tile's may be written
-                if (!(ok = wait(&s_free, j & 1))) break;
-                if (j + 1 < n_kv && !(ok = issue_s(j + 1))) break;
-                if (!(ok = wait(&p_full, j & 1))) break;
-                tc_fence_after();
-                // dQ += dS K: dS from tensor memory (keys 32 u .. at 384 + 16 u,
-                // 8 columns per 16 keys), K MN-major (+2048 B per 16 keys)
-                const uint64_t km =
-                    umma_smem_desc(base + Lay::kOffK + ks * Lay::kTile, Lay::kPanel, 1024);
+                for (int j = 0; ok && j + 1 < n_kv; ++j)
+                    ok = wait(&s_free, j & 1) && issue_s(j + 1);
+                // its last products have finished before the block exits
+                tc_commit(&s_drain);
+                mbar_wait(&s_drain, 0, &abort_flag, p.status, 1000000000ull);
+            } else {
+                bool ok = true;
+                for (int j = 0; ok && j < n_kv; ++j) {
+                    const int ks = j % kDqKStages;
+                    // dS(j) is in tensor memory; K(j) has landed (S(j) read it)
+                    if (!(ok = wait(&p_full, j & 1) && wait(&k_full[ks], (j / kDqKStages) & 1)))
+                        break;
+                    tc_fence_after();
+                    // dQ += dS K: dS from tensor memory (keys 32 u .. at 384 + 16 u,
+                    // 8 columns per 16 keys), K MN-major (+2048 B per 16 keys)
+                    const uint64_t km =
+                        umma_smem_desc(base + Lay::kOffK + ks * Lay::kTile, Lay::kPanel, 1024);
 #pragma unroll
-                for (int kk = 0; kk < kDqBN / 16; ++kk)
-                    umma_ts(tmem + Lay::kColDQ, tmem + Lay::kColDS + kk * 8, km + kk * (2048 >> 4),
-                            idesc_o, (j > 0 || kk > 0) ? 1u : 0u);
-                tc_commit(&dq_done);
-                tc_commit(&k_empty[ks]);
+                    for (int kk = 0; kk < kDqBN / 16; ++kk)
+                        umma_ts(tmem + Lay::kColDQ, tmem + Lay::kColDS + kk * 8,
+                                km + kk * (2048 >> 4), idesc_o, (j > 0 || kk > 0) ? 1u : 0u);
+                    tc_commit(&dq_done);
+                    tc_commit(&k_empty[ks]);
+                }
+                tc_commit(&acc_done);
+                mbar_wait(&acc_done, 0, &abort_flag, p.status, 1000000000ull);
             }
-            tc_commit(&acc_done);
-            mbar_wait(&acc_done, 0, &abort_flag, p.status, 1000000000ull);
         }
     } else if (warp >= 4) {
         // ---------------------------------------- elementwise + epilogue ----
