@@ -105,11 +105,10 @@ int gqa_attn_fwd_rope(const void *q, const void *k, const void *v, void *o, floa
  * written (pinned host memory for the copies to run asynchronously; pageable
  * memory works, slower); q_dev, k_dev, v_dev, o_dev are caller-owned device
  * staging buffers of the full tensor sizes (16-byte aligned), overwritten.
- * The query rows are cut into at most 16 chunks of >= 256 rows; chunk c's q
- * rows and the k / v rows it newly needs (with the causal mask, keys up to
- * its last row + Tkv - Tq) are copied up on a library-owned copy stream
- * while chunk c - 1's attention runs on `stream` and chunk c - 2's o is
- * copied down on a second library-owned stream.  Asynchronous: with
+ * k and v are copied up whole first, then the query rows in 4 chunks of
+ * >= 256 rows, last rows first, on a library-owned copy stream; each chunk's
+ * attention runs on `stream` once its rows have landed, while the previous
+ * chunk's o is copied down on a second library-owned stream.  Asynchronous: with
  * done_event == NULL, o_host is complete when the work enqueued on `stream` so
  * far is; otherwise done_event (a cudaEvent_t created by the caller) is
  * recorded when o_host is complete and `stream` is not held for the copies
