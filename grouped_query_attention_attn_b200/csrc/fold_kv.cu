@@ -16,13 +16,19 @@ namespace gqa {
 constexpr int kFoldBatch = 4;   // group members loaded before any is added
 
 // Index type I: 32-bit when every vector index fits, so the per-vector
-// divisions stay cheap.
-template <typename I>
+// divisions stay cheap.  kD8: d / 8 known at compile time (d = 64, 128: the
+// index math becomes shifts), 0 for any other d.
+template <typename I, int kD8>
 __global__ void __launch_bounds__(256, 5)
 fold_kv_kernel(const uint4 *__restrict__ in, uint4 *__restrict__ out, I n_vec, int H, int g,
-               int d8) {
+               int d8_arg) {
+    const int d8 = kD8 > 0 ? kD8 : d8_arg;
     const int size = H / g;
     const float divisor = static_cast<float>(size);
+    // dividing by a power of two is exact, so it is a multiplication by the
+    // reciprocal; any other group size takes the correctly rounded division
+    const bool pow2 = (size & (size - 1)) == 0;
+    const float inv = 1.0f / divisor;
     const I stride = static_cast<I>(gridDim.x) * blockDim.x;
     for (I t = static_cast<I>(blockIdx.x) * blockDim.x + threadIdx.x; t < n_vec; t += stride) {
         const I c8 = t % d8, rest = t / d8;
@@ -53,8 +59,9 @@ fold_kv_kernel(const uint4 *__restrict__ in, uint4 *__restrict__ out, I n_vec, i
         uint32_t *rw = reinterpret_cast<uint32_t *>(&r);
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-            __nv_bfloat162 pr = __floats2bfloat162_rn(__fdiv_rn(acc[2 * e], divisor),
-                                                      __fdiv_rn(acc[2 * e + 1], divisor));
+            const float lo = pow2 ? acc[2 * e] * inv : __fdiv_rn(acc[2 * e], divisor);
+            const float hi = pow2 ? acc[2 * e + 1] * inv : __fdiv_rn(acc[2 * e + 1], divisor);
+            __nv_bfloat162 pr = __floats2bfloat162_rn(lo, hi);
             rw[e] = *reinterpret_cast<uint32_t *>(&pr);
         }
         out[t] = r;
@@ -70,12 +77,18 @@ int launch_fold_kv(const void *in, void *out, int B, int T, int H, int g, int d,
     if (blocks > 0x7fffffffull) blocks = 0x7fffffffull;
     const uint4 *src = static_cast<const uint4 *>(in);
     uint4 *dst = static_cast<uint4 *>(out);
-    if (n_vec + static_cast<size_t>(blocks) * 256 <= 0xffffffffull)
-        fold_kv_kernel<uint32_t><<<static_cast<unsigned>(blocks), 256, 0, stream>>>(
-            src, dst, static_cast<uint32_t>(n_vec), H, g, d8);
-    else
-        fold_kv_kernel<size_t><<<static_cast<unsigned>(blocks), 256, 0, stream>>>(src, dst, n_vec,
-                                                                                H, g, d8);
+    const unsigned nb = static_cast<unsigned>(blocks);
+    if (n_vec + static_cast<size_t>(blocks) * 256 <= 0xffffffffull) {
+        const uint32_t n32 = static_cast<uint32_t>(n_vec);
+        if (d8 == 16)
+            fold_kv_kernel<uint32_t, 16><<<nb, 256, 0, stream>>>(src, dst, n32, H, g, d8);
+        else if (d8 == 8)
+            fold_kv_kernel<uint32_t, 8><<<nb, 256, 0, stream>>>(src, dst, n32, H, g, d8);
+        else
+            fold_kv_kernel<uint32_t, 0><<<nb, 256, 0, stream>>>(src, dst, n32, H, g, d8);
+    } else {
+        fold_kv_kernel<size_t, 0><<<nb, 256, 0, stream>>>(src, dst, n_vec, H, g, d8);
+    }
     return check_cuda(cudaGetLastError(), "fold_kv_kernel launch");
 }
 

@@ -12,7 +12,8 @@ from oracle import ref
 pytestmark = pytest.mark.gpu
 
 
-@pytest.mark.parametrize("H,g,d", [(32, 8, 128), (32, 1, 128), (8, 8, 64), (12, 3, 16), (6, 2, 8)])
+@pytest.mark.parametrize("H,g,d", [(32, 8, 128), (32, 1, 128), (8, 8, 64), (12, 3, 16), (6, 2, 8),
+                                   (12, 2, 128), (10, 2, 64)])   # group sizes 6, 5: rounded division
 def test_fold_bit_exact(gqa_lib, H, g, d):
     kv = workloads.randn((2, 37, H, d), H * g + d)
     out = gqa.fold_kv(kv.cuda(), g)
