@@ -14,8 +14,13 @@
 //           in tensor memory with no atomics
 //   dq      tcgen05: one CTA per 128-row M tile (the group's heads packed by
 //           position, as in the forward), looping over the visible keys
+// dkdv and dq read the same inputs and write disjoint outputs, so after
+// rowdot they run side by side: dkdv on a second stream of the highest
+// priority (its blocks are dispatched first, its longest CTAs start at once),
+// dq on the caller's stream filling the SMs that dkdv's tail leaves idle.
 #include <cuda_bf16.h>
 #include <climits>
+#include <mutex>
 
 #include "device.cuh"
 #include "internal.h"
@@ -945,6 +950,53 @@ size_t bwd_workspace_bytes(int B, int Tq, int Hq) {
     return ((static_cast<size_t>(B) * Tq * Hq * sizeof(float)) + 255) & ~static_cast<size_t>(255);
 }
 
+namespace {
+
+// The second stream and the fork / join events, created once per CUDA context
+// (again when another context is current, e.g. after a cudaDeviceReset).  The
+// record / wait sequence runs under the lock, so concurrent host threads cannot
+// interleave their records of the shared events.
+struct SideRes {
+    cudaStream_t s = nullptr;
+    cudaEvent_t fork = nullptr, join = nullptr;
+    unsigned long long ctx_id = 0;
+    bool ready = false;
+};
+
+std::mutex g_side_mu;
+SideRes g_side[kMaxDevices];
+
+int side_res(SideRes **out) {
+    int dev = 0;
+    unsigned long long ctx_id = 0;
+    if (int rc = current_ctx_key(&dev, &ctx_id)) return rc;
+    SideRes &r = g_side[dev];
+    if (!r.ready || (ctx_id != 0 && r.ctx_id != ctx_id)) {
+        r.ready = false;
+        int least = 0, greatest = 0;
+        if (int rc = check_cuda(cudaDeviceGetStreamPriorityRange(&least, &greatest),
+                                "cudaDeviceGetStreamPriorityRange"))
+            return rc;
+        if (int rc = check_cuda(cudaStreamCreateWithPriority(&r.s, cudaStreamNonBlocking, greatest),
+                                "cudaStreamCreateWithPriority"))
+            return rc;
+        if (int rc = check_cuda(cudaEventCreateWithFlags(&r.fork, cudaEventDisableTiming),
+                                "cudaEventCreateWithFlags"))
+            return rc;
+        if (int rc = check_cuda(cudaEventCreateWithFlags(&r.join, cudaEventDisableTiming),
+                                "cudaEventCreateWithFlags"))
+            return rc;
+        int dev2 = 0;
+        unsigned long long id2 = 0;
+        r.ctx_id = (current_ctx_key(&dev2, &id2) == GQA_OK && dev2 == dev) ? id2 : 0;
+        r.ready = true;
+    }
+    *out = &r;
+    return GQA_OK;
+}
+
+}  // namespace
+
 template <int D>
 static int launch_bwd_d(const void *q, const void *k, const void *v, const void *o,
                         const void *dout, const float *lse, void *dq, void *dk, void *dv, int B,
@@ -964,10 +1016,23 @@ static int launch_bwd_d(const void *q, const void *k, const void *v, const void 
     if (Tkv == 0)   // no key: every query gradient is zero
         return check_cuda(cudaMemsetAsync(dq, 0, static_cast<size_t>(B) * Tq * Hq * D * 2, stream),
                           "cudaMemsetAsync(dq)");
-    if (int rc = launch_dkdv_tc<D>(q, k, v, dout, lse, Dsum, dk, dv, B, Tq, Tkv, Hq, Hkv, vis, scale,
-                                   stream))
+    std::lock_guard<std::mutex> lock(g_side_mu);
+    SideRes *r = nullptr;
+    if (int rc = side_res(&r)) return rc;
+    // fork: the side stream waits for rowdot; dkdv is enqueued before dq
+    if (int rc = check_cuda(cudaEventRecord(r->fork, stream), "cudaEventRecord(fork)")) return rc;
+    if (int rc = check_cuda(cudaStreamWaitEvent(r->s, r->fork, 0), "cudaStreamWaitEvent(fork)"))
         return rc;
-    return launch_dq_tc<D>(q, k, v, dout, lse, Dsum, dq, B, Tq, Tkv, Hq, Hkv, vis, scale, stream);
+    int rc = launch_dkdv_tc<D>(q, k, v, dout, lse, Dsum, dk, dv, B, Tq, Tkv, Hq, Hkv, vis, scale,
+                               r->s);
+    if (rc == GQA_OK)
+        rc = launch_dq_tc<D>(q, k, v, dout, lse, Dsum, dq, B, Tq, Tkv, Hq, Hkv, vis, scale, stream);
+    // join, on every path: the caller's stream (and a capture in progress on
+    // it) then covers all the side stream's work
+    const int rj = check_cuda(cudaEventRecord(r->join, r->s), "cudaEventRecord(join)");
+    const int rw = rj ? rj : check_cuda(cudaStreamWaitEvent(stream, r->join, 0),
+                                        "cudaStreamWaitEvent(join)");
+    return rc ? rc : rw;
 }
 
 int launch_bwd(const void *q, const void *k, const void *v, const void *o, const void *dout,
