@@ -10,5 +10,5 @@ streams only.  The library is loaded on first use and there is no CPU
 fallback: a missing or unloadable library raises.
 """
 
-from .api import (attn, attn_bwd, attn_f32, attn_host, decode, decode_workspace_size, device_status, fold_kv,  # noqa: F401
+from .api import (attn, attn_bwd, attn_bwd_workspace_size, attn_f32, attn_host, decode, decode_workspace_size, device_status, fold_kv,  # noqa: F401
                   host_staging, rope_, rope_decode_q_, rope_qk_)

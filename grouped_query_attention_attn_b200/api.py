@@ -212,6 +212,10 @@ def fold_kv(kv, g):
     return out
 
 
+def attn_bwd_workspace_size(B, Tq, Hq):
+    return int(_b.gqa_attn_bwd_workspace_size(B, Tq, Hq))
+
+
 def attn_bwd(q, k, v, o, lse, dout, causal=True, scale=None, window=None, sinks=0,
              workspace=None):
     """Gradients (dq, dk, dv) of attn(q, k, v) for the upstream gradient dout.

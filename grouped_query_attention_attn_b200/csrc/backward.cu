@@ -54,7 +54,7 @@ __device__ __forceinline__ bool block_visible(const Vis &v, int i0, int ni, int 
 // D = rowsum(dO o O) per (b, t, h), stored [B, H, T].  A group of D / 8 lanes
 // owns kRowdotRows consecutive rows and reads them as 16-byte vectors (all
 // loads in flight before the products), then reduces each row over the group.
-constexpr int kRowdotRows = 4;
+constexpr int kRowdotRows = 2;
 
 template <int D>
 __global__ void __launch_bounds__(256)

@@ -107,3 +107,42 @@ def test_backward_headline_shape(gqa_lib, g):
     assert rel_err(dq[:, :, hs], rq) <= 2e-2
     assert rel_err(dk[:, :, g:g + 1], rk) <= 2e-2
     assert rel_err(dv[:, :, g:g + 1], rv) <= 2e-2
+
+
+def test_backward_graph_capture_and_streams(gqa_lib):
+    # The dK/dV kernel runs on the library's second stream, forked from and
+    # joined back into the caller's stream.  A CUDA graph captured on a side
+    # stream must hold both kernels, and its replays, as well as calls on the
+    # default stream, must give exactly the eager result (no atomics: the sums
+    # run in a fixed order).
+    B, T, Hq, Hkv, d = 2, 384, 8, 2, 128
+    q, k, v = workloads.prefill_inputs(B, T, Hq, Hkv, d, seeds=(11, 12, 13))
+    qc, kc, vc = q.cuda(), k.cuda(), v.cuda()
+    o, lse = gqa.attn(qc, kc, vc, causal=True, return_lse=True)
+    douts = [workloads.randn((B, T, Hq, d), 40 + i).cuda() for i in range(3)]
+    want = [gqa.attn_bwd(qc, kc, vc, o, lse, dd) for dd in douts]
+    torch.cuda.synchronize()
+    gqa.device_status()
+    dout = douts[0].clone()
+    ws = torch.empty(gqa.attn_bwd_workspace_size(B, T, Hq), dtype=torch.uint8, device="cuda")
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        gqa.attn_bwd(qc, kc, vc, o, lse, dout, workspace=ws)    # warm-up outside capture
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=s):
+            got = gqa.attn_bwd(qc, kc, vc, o, lse, dout, workspace=ws)
+    for rep in (2, 1, 0):
+        dout.copy_(douts[rep])
+        for t in got:
+            t.fill_(float("nan"))
+        g.replay()
+        torch.cuda.synchronize()
+        for a, b in zip(got, want[rep]):
+            assert torch.equal(a, b), rep
+    with torch.cuda.stream(torch.cuda.default_stream()):
+        again = gqa.attn_bwd(qc, kc, vc, o, lse, douts[1])
+    torch.cuda.synchronize()
+    gqa.device_status()
+    for a, b in zip(again, want[1]):
+        assert torch.equal(a, b)
