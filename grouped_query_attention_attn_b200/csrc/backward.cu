@@ -59,8 +59,11 @@ constexpr int kRowdotRows = 2;
 template <int D>
 __global__ void __launch_bounds__(256)
 rowdot_kernel(const __nv_bfloat16 *__restrict__ dout, const __nv_bfloat16 *__restrict__ o,
-              float *__restrict__ Dsum, int B, int T, int H) {
+              float *__restrict__ Dsum, unsigned int *__restrict__ tile_counter, int B, int T,
+              int H) {
     constexpr int kLanes = D / 8;                   // lanes per row: 8 or 16
+    // the dQ kernel's tile counter starts from zero (it runs next on this stream)
+    if (blockIdx.x == 0 && threadIdx.x == 0) *tile_counter = 0u;
     const long long rows = static_cast<long long>(B) * T * H;
     const long long gt = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
     const int c8 = threadIdx.x % kLanes;
@@ -572,9 +575,9 @@ static int launch_dkdv_tc(const void *q, const void *k, const void *v, const voi
 }
 
 // --------------------------------------------------------- dq (tcgen05) ---
-// One CTA per 128-row M tile: the G query heads of one KV group at
-// P = floor(128 / G) positions, as in the forward (one 3-D TMA box; every K / V
-// tile serves the whole group).  For every visible 128-key tile:
+// M tiles of 128 rows: the G query heads of one KV group at P = floor(128 / G)
+// positions, as in the forward (one 3-D TMA box; every K / V tile serves the
+// whole group).  For every visible 128-key tile of an M tile:
 //   tensor pipe   S = Q K^T and dP = dO V^T into tensor memory;
 //   16 warps      load S and dP (four threads per row, one per 32-key
 //                 quarter), release them, and form dS = P (dP - D_row) with
@@ -587,9 +590,18 @@ static int launch_dkdv_tc(const void *q, const void *k, const void *v, const voi
 // Q, dO, a 3-deep K ring (K(j) serves S(j) and, a tile later, dQ(j), so the
 // copy of K(j+2) must not wait for dQ(j)) and a 2-deep V ring (V(j) is free
 // once dP(j) has run).
+//
+// Persistent: one CTA per SM takes M tiles, heaviest first, from a counter in
+// the workspace (zeroed by rowdot, which runs before on the same stream), so
+// CTAs that start late -- the dK/dV kernel runs beside this one -- still share
+// the work evenly.  Every barrier counts across M tiles: the next tile's Q / dO
+// copy and its first S and dP run while the warps finish the current tile's
+// last dS and read its dQ out of tensor memory.  Warp 0 fetches tile indices
+// into a 2-slot ring in shared memory that the other roles read.
 constexpr int kDqBN = 128;       // keys per tile
 constexpr int kDqKStages = 3;
 constexpr int kDqVStages = 2;
+constexpr int kDqConsumers = 3 + kTcElemWarps;   // warps 1, 2, 3 and the elementwise warps
 
 template <int D>
 struct DqLayout {
@@ -608,11 +620,39 @@ struct DqLayout {
 struct DqParams {
     int B, Tq, Tkv, Hq, Hkv, G, P;    // P = positions per M tile
     int n_mt;                         // M tiles per (b, kvh)
+    int n_tiles;                      // n_mt * Hkv * B
     Vis vis;
     float scale, scale_log2;
     const float *lse, *Dsum;
     __nv_bfloat16 *dq;
+    unsigned int *tile_counter;       // zero on entry
     int *status;
+};
+
+// M tile number t (0 = heaviest) of a call: its rows and visible key tiles.
+struct DqTile {
+    int b, kvh, t0, n_kv, n_sink, first;
+    __device__ __forceinline__ DqTile(const DqParams &p, int t) {
+        const int bhs = p.Hkv * p.B;
+        // M tiles in decreasing causal work (the last positions see the most keys)
+        const int mt = p.n_mt - 1 - t / bhs;
+        kvh = t % p.Hkv;
+        b = (t / p.Hkv) % p.B;
+        t0 = mt * p.P;
+        const int last_pos = min(t0 + p.P, p.Tq) - 1;
+        const int off = p.Tkv - p.Tq;
+        int kv_end = p.Tkv;
+        if (p.vis.causal) kv_end = min(p.Tkv, last_pos + off + 1);
+        n_sink = 0;
+        first = 0;
+        if (p.vis.window > 0 && kv_end > 0) {
+            n_sink = (min(p.vis.sinks, kv_end) + kDqBN - 1) / kDqBN;
+            first = max(n_sink, max(t0 + off - p.vis.window + 1, 0) / kDqBN);
+        }
+        const int last = kv_end > 0 ? (kv_end + kDqBN - 1) / kDqBN : 0;
+        n_kv = n_sink + max(0, last - first);
+    }
+    __device__ __forceinline__ int tile_of(int j) const { return j < n_sink ? j : first + (j - n_sink); }
 };
 
 template <int D>
@@ -624,31 +664,17 @@ dq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-    __shared__ uint64_t qo_full, k_full[kDqKStages], k_empty[kDqKStages], v_full[kDqVStages],
-        v_empty[kDqVStages], s_full, s_free, p_full, dq_done, acc_done, s_drain;
+    __shared__ uint64_t qo_full, qo_empty, k_full[kDqKStages], k_empty[kDqKStages],
+        v_full[kDqVStages], v_empty[kDqVStages], s_full, s_free, p_full, dq_done, acc_done,
+        dq_free, drain[2], t_full[2], t_empty[2];
+    __shared__ int t_slot[2];
     __shared__ uint32_t tmem_base_sh;
     __shared__ int abort_flag;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-    // M tiles in decreasing causal work (the last positions see the most keys)
-    const int bhs = p.Hkv * p.B, lin = blockIdx.x;
-    const int mt = p.n_mt - 1 - lin / bhs, kvh = lin % p.Hkv, b = (lin / p.Hkv) % p.B;
-    const int t0 = mt * p.P;
-    const int last_pos = min(t0 + p.P, p.Tq) - 1;
-    const int off = p.Tkv - p.Tq;
-    int kv_end = p.Tkv;
-    if (p.vis.causal) kv_end = min(p.Tkv, last_pos + off + 1);
-    int n_sink = 0, first = 0;
-    if (p.vis.window > 0 && kv_end > 0) {
-        n_sink = (min(p.vis.sinks, kv_end) + kDqBN - 1) / kDqBN;
-        first = max(n_sink, max(t0 + off - p.vis.window + 1, 0) / kDqBN);
-    }
-    const int last = kv_end > 0 ? (kv_end + kDqBN - 1) / kDqBN : 0;
-    const int n_kv = n_sink + max(0, last - first);
-    auto tile_of = [&](int j) { return j < n_sink ? j : first + (j - n_sink); };
-
     if (threadIdx.x == 0) {
         mbar_init(&qo_full, 1);
+        mbar_init(&qo_empty, 1);
         for (int s = 0; s < kDqKStages; ++s) {
             mbar_init(&k_full[s], 1);
             mbar_init(&k_empty[s], 1);
@@ -662,7 +688,13 @@ dq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
         mbar_init(&p_full, kTcElemWarps);
         mbar_init(&dq_done, 1);
         mbar_init(&acc_done, 1);
-        mbar_init(&s_drain, 1);
+        mbar_init(&dq_free, kTcElemWarps);
+        mbar_init(&drain[0], 1);
+        mbar_init(&drain[1], 1);
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(&t_full[s], 1);
+            mbar_init(&t_empty[s], kDqConsumers);
+        }
         abort_flag = 0;
         fence_mbar_init();
     }
@@ -674,86 +706,145 @@ dq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = tmem_base_sh;
+    auto wait = [&](uint64_t *bar, uint32_t parity) {
+        return mbar_wait(bar, parity, &abort_flag, p.status);
+    };
+    // Tile number of iteration `it` (>= p.n_tiles: no more tiles), read by a
+    // consuming warp; lane 0 releases the slot.  -1 after an abort.
+    auto take_tile = [&](int it) {
+        const int slot = it & 1;
+        if (!__all_sync(0xffffffffu, wait(&t_full[slot], (it >> 1) & 1))) return -1;
+        const int t = *reinterpret_cast<volatile int *>(&t_slot[slot]);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&t_empty[slot]);
+        return t;
+    };
 
-    if (warp == 0 || warp == 2) {
-        // ---------------------------------------------- TMA producers ----
-        // Warp 0 loads Q, dO and the K ring, warp 2 the V ring: each waits only
-        // on its own ring's releases (K(j) is held until dQ(j), V(j) only
-        // until dP(j)), so a late K stage never holds back a V copy.
+    if (warp == 0) {
+        // -------------------------- scheduler, Q / dO and K ring producer ----
         const bool leader = elect_one();
-        const bool is_k = warp == 0;
-        if (n_kv > 0) {
-            if (leader && is_k) {
-                tma_prefetch_desc(&tm_k);
+        const int leader_lane = __ffs(__ballot_sync(0xffffffffu, leader)) - 1;
+        if (leader) {
+            tma_prefetch_desc(&tm_q);
+            tma_prefetch_desc(&tm_o);
+            tma_prefetch_desc(&tm_k);
+        }
+        uint32_t kc = 0, qi = 0;   // K copies and Q / dO copies issued
+        bool ok = true;
+        for (int it = 0; ok; ++it) {
+            const int slot = it & 1;
+            if (it >= 2 && !(ok = __all_sync(0xffffffffu, wait(&t_empty[slot], ((it >> 1) & 1) ^ 1))))
+                break;
+            int t = 0;
+            if (leader) {
+                t = static_cast<int>(atomicAdd(p.tile_counter, 1u));
+                if (t > p.n_tiles) t = p.n_tiles;
+                t_slot[slot] = t;
+                mbar_arrive(&t_full[slot]);     // release: the index store comes first
+            }
+            t = __shfl_sync(0xffffffffu, t, leader_lane);
+            if (t >= p.n_tiles) break;
+            const DqTile T(p, t);
+            if (T.n_kv == 0) continue;
+            // Q and dO of the previous tile are free once its last S / dP ran
+            if (qi > 0 && !(ok = __all_sync(0xffffffffu, wait(&qo_empty, (qi - 1) & 1)))) break;
+            if (leader) {
                 const uint32_t box = 64u * p.G * p.P * 2u;
                 mbar_expect_tx(&qo_full, 2 * Lay::kPanels * box);
                 for (int pn = 0; pn < Lay::kPanels; ++pn) {
                     tma_load_4d(smem + Lay::kOffQ + pn * Lay::kPanel, &tm_q, &qo_full, pn * 64,
-                                kvh * p.G, t0, b);
+                                T.kvh * p.G, T.t0, T.b);
                     tma_load_4d(smem + Lay::kOffO + pn * Lay::kPanel, &tm_o, &qo_full, pn * 64,
-                                kvh * p.G, t0, b);
+                                T.kvh * p.G, T.t0, T.b);
                 }
             }
-            if (leader && !is_k) tma_prefetch_desc(&tm_v);
             __syncwarp();
-            const int stages = is_k ? kDqKStages : kDqVStages;
-            uint64_t *full = is_k ? k_full : v_full, *empty = is_k ? k_empty : v_empty;
-            const CUtensorMap *tm = is_k ? &tm_k : &tm_v;
-            const int off0 = is_k ? Lay::kOffK : Lay::kOffV;
-            int issued = 0;
-            for (int j = 0; j < n_kv; ++j) {
-                const int st = j % stages, ph = (j / stages) & 1;
-                if (!__all_sync(0xffffffffu, mbar_wait(&empty[st], ph ^ 1, &abort_flag, p.status)))
-                    break;
+            ++qi;
+            for (int j = 0; j < T.n_kv; ++j, ++kc) {
+                const uint32_t st = kc % kDqKStages, ph = (kc / kDqKStages) & 1;
+                if (!(ok = __all_sync(0xffffffffu, wait(&k_empty[st], ph ^ 1)))) break;
                 if (leader) {
-                    mbar_expect_tx(&full[st], Lay::kTile);
+                    mbar_expect_tx(&k_full[st], Lay::kTile);
                     for (int pn = 0; pn < Lay::kPanels; ++pn)
-                        tma_load_4d(smem + off0 + st * Lay::kTile + pn * Lay::kPanel, tm, &full[st],
-                                    pn * 64, kvh, tile_of(j) * kDqBN, b);
+                        tma_load_4d(smem + Lay::kOffK + st * Lay::kTile + pn * Lay::kPanel, &tm_k,
+                                    &k_full[st], pn * 64, T.kvh, T.tile_of(j) * kDqBN, T.b);
                 }
                 __syncwarp();
-                issued = j + 1;
             }
-            // copies still in flight land before the block exits
-            if (is_k) mbar_wait(&qo_full, 0, &abort_flag, p.status, 1000000ull);
-            for (int j = max(0, issued - stages); j < issued; ++j)
-                mbar_wait(&full[j % stages], (j / stages) & 1, &abort_flag, p.status, 1000000ull);
         }
+        // copies still in flight land before the block exits
+        if (qi > 0) mbar_wait(&qo_full, (qi - 1) & 1, &abort_flag, p.status, 1000000ull);
+        for (uint32_t c = kc > kDqKStages ? kc - kDqKStages : 0; c < kc; ++c)
+            mbar_wait(&k_full[c % kDqKStages], (c / kDqKStages) & 1, &abort_flag, p.status,
+                      1000000ull);
+    } else if (warp == 2) {
+        // ------------------------------------------------ V ring producer ----
+        const bool leader = elect_one();
+        if (leader) tma_prefetch_desc(&tm_v);
+        uint32_t vc = 0;
+        bool ok = true;
+        for (int it = 0; ok; ++it) {
+            const int t = take_tile(it);
+            if (t < 0 || t >= p.n_tiles) break;
+            const DqTile T(p, t);
+            for (int j = 0; j < T.n_kv; ++j, ++vc) {
+                const uint32_t st = vc % kDqVStages, ph = (vc / kDqVStages) & 1;
+                if (!(ok = __all_sync(0xffffffffu, wait(&v_empty[st], ph ^ 1)))) break;
+                if (leader) {
+                    mbar_expect_tx(&v_full[st], Lay::kTile);
+                    for (int pn = 0; pn < Lay::kPanels; ++pn)
+                        tma_load_4d(smem + Lay::kOffV + st * Lay::kTile + pn * Lay::kPanel, &tm_v,
+                                    &v_full[st], pn * 64, T.kvh, T.tile_of(j) * kDqBN, T.b);
+                }
+                __syncwarp();
+            }
+        }
+        for (uint32_t c = vc > kDqVStages ? vc - kDqVStages : 0; c < vc; ++c)
+            mbar_wait(&v_full[c % kDqVStages], (c / kDqVStages) & 1, &abort_flag, p.status,
+                      1000000ull);
     } else if ((warp == 1 || warp == 3) && lane == 0) {
         // ------------------------------------------------ MMA issuers ----
-        // Warp 1 issues S and dP, warp 3 issues dQ.  The two streams touch
-        // disjoint tensor-memory regions (S | dP against dQ, reading dS) and
-        // shared-memory stages released through their own barriers, so they need
-        // no order between them; with one issuer a dQ(j) whose dS was ready sat
-        // behind the whole S / dP(j+1) group (tcgen05.mma blocks the issuing
-        // thread once its queue is full), and S / dP(j+2) behind dQ(j).
-        if (n_kv > 0) {
-            constexpr uint32_t idesc_s = umma_idesc_bf16(128, kDqBN, 0, 0);
-            constexpr uint32_t idesc_o = umma_idesc_bf16(128, D, 0, 1);
-            const uint32_t base = smem_u32(smem);
-            const uint64_t dQt = umma_smem_desc(base + Lay::kOffQ, 16, 1024);
-            const uint64_t dOt = umma_smem_desc(base + Lay::kOffO, 16, 1024);
-            auto wait = [&](uint64_t *bar, uint32_t parity) {
-                return mbar_wait(bar, parity, &abort_flag, p.status);
-            };
+        // Warp 1 issues S and dP, warp 3 issues dQ, one thread each.  The two
+        // streams touch disjoint tensor-memory regions (S | dP against dQ,
+        // reading dS) and release shared-memory stages through their own
+        // barriers, so they need no order between them; with one issuer a dQ(j)
+        // whose dS was ready sat behind the whole S / dP(j+1) group (tcgen05.mma
+        // blocks the issuing thread once its queue is full), and S / dP(j+2)
+        // behind dQ(j).
+        constexpr uint32_t idesc_s = umma_idesc_bf16(128, kDqBN, 0, 0);
+        constexpr uint32_t idesc_o = umma_idesc_bf16(128, D, 0, 1);
+        const uint32_t base = smem_u32(smem);
+        const uint64_t dQt = umma_smem_desc(base + Lay::kOffQ, 16, 1024);
+        const uint64_t dOt = umma_smem_desc(base + Lay::kOffO, 16, 1024);
+        uint32_t g = 0, qi = 0;   // key tiles and M tiles with keys, over the whole block
+        bool ok = true;
+        for (int it = 0; ok; ++it) {
+            const int slot = it & 1;
+            if (!(ok = wait(&t_full[slot], (it >> 1) & 1))) break;
+            const int t = *reinterpret_cast<volatile int *>(&t_slot[slot]);
+            mbar_arrive(&t_empty[slot]);
+            if (t >= p.n_tiles) break;
+            const DqTile T(p, t);
+            if (T.n_kv == 0) continue;
             if (warp == 1) {
                 // S = Q K_j^T, dP = dO V_j^T: K-major A and B (+32 B per 16 of d);
                 // V_j's stage is released as soon as dP has run
-                auto issue_s = [&](int j) {
-                    const int ks = j % kDqKStages, vs = j % kDqVStages;
-                    if (!wait(&k_full[ks], (j / kDqKStages) & 1)) return false;
+                if (!(ok = wait(&qo_full, qi & 1))) break;
+                for (int j = 0; j < T.n_kv; ++j, ++g) {
+                    // the warps hold S, dP of the previous key tile in registers
+                    if (g > 0 && !(ok = wait(&s_free, (g - 1) & 1))) break;
+                    const uint32_t ks = g % kDqKStages, vs = g % kDqVStages;
+                    if (!(ok = wait(&k_full[ks], (g / kDqKStages) & 1))) break;
                     tc_fence_after();
-                    const uint64_t bk =
-                        umma_smem_desc(base + Lay::kOffK + ks * Lay::kTile, 16, 1024);
+                    const uint64_t bk = umma_smem_desc(base + Lay::kOffK + ks * Lay::kTile, 16, 1024);
 #pragma unroll
                     for (int kk = 0; kk < D / 16; ++kk) {
                         const uint32_t o16 = ((kk >> 2) * Lay::kPanel + (kk & 3) * 32) >> 4;
                         umma_ss(tmem + Lay::kColS, dQt + o16, bk + o16, idesc_s, kk > 0);
                     }
-                    if (!wait(&v_full[vs], (j / kDqVStages) & 1)) return false;
+                    if (!(ok = wait(&v_full[vs], (g / kDqVStages) & 1))) break;
                     tc_fence_after();
-                    const uint64_t bv =
-                        umma_smem_desc(base + Lay::kOffV + vs * Lay::kTile, 16, 1024);
+                    const uint64_t bv = umma_smem_desc(base + Lay::kOffV + vs * Lay::kTile, 16, 1024);
 #pragma unroll
                     for (int kk = 0; kk < D / 16; ++kk) {
                         const uint32_t o16 = ((kk >> 2) * Lay::kPanel + (kk & 3) * 32) >> 4;
@@ -761,22 +852,17 @@ dq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
                     }
                     tc_commit(&s_full);
                     tc_commit(&v_empty[vs]);
-                    return true;
-                };
-                bool ok = wait(&qo_full, 0) && issue_s(0);
-                // the warps hold S(j), dP(j) in registers: the next tile's may be written
-                for (int j = 0; ok && j + 1 < n_kv; ++j)
-                    ok = wait(&s_free, j & 1) && issue_s(j + 1);
-                // its last products have finished before the block exits
-                tc_commit(&s_drain);
-                mbar_wait(&s_drain, 0, &abort_flag, p.status, 1000000000ull);
+                }
+                if (!ok) break;
+                // this tile's Q and dO are free once its last products have run
+                tc_commit(&qo_empty);
             } else {
-                bool ok = true;
-                for (int j = 0; ok && j < n_kv; ++j) {
-                    const int ks = j % kDqKStages;
-                    // dS(j) is in tensor memory; K(j) has landed (S(j) read it)
-                    if (!(ok = wait(&p_full, j & 1) && wait(&k_full[ks], (j / kDqKStages) & 1)))
-                        break;
+                // the previous tile's dQ has been read out of tensor memory
+                if (qi > 0 && !(ok = wait(&dq_free, (qi - 1) & 1))) break;
+                for (int j = 0; j < T.n_kv; ++j, ++g) {
+                    const uint32_t ks = g % kDqKStages;
+                    // dS is in tensor memory; K has landed (S read it)
+                    if (!(ok = wait(&p_full, g & 1) && wait(&k_full[ks], (g / kDqKStages) & 1))) break;
                     tc_fence_after();
                     // dQ += dS K: dS from tensor memory (keys 32 u .. at 384 + 16 u,
                     // 8 columns per 16 keys), K MN-major (+2048 B per 16 keys)
@@ -789,111 +875,150 @@ dq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
                     tc_commit(&dq_done);
                     tc_commit(&k_empty[ks]);
                 }
+                if (!ok) break;
                 tc_commit(&acc_done);
-                mbar_wait(&acc_done, 0, &abort_flag, p.status, 1000000000ull);
             }
+            ++qi;
         }
+        // the last products have finished before the block exits
+        uint64_t *dr = &drain[warp == 1 ? 0 : 1];
+        tc_commit(dr);
+        mbar_wait(dr, 0, &abort_flag, p.status, 1000000000ull);
     } else if (warp >= 4) {
         // ---------------------------------------- elementwise + epilogue ----
         const int u = (warp - 4) >> 2;                  // key quarter of a tile
         const int g4 = warp & 3;                        // lane group
         const int r = (g4 << 5) + lane;                 // row = tensor-memory lane
-        const int pos = t0 + r / p.G, head = kvh * p.G + r % p.G;
-        const bool row_real = (r < p.P * p.G) && (pos < p.Tq);
         const uint32_t lane_addr = tmem + ((static_cast<uint32_t>(g4) * 32u) << 16);
-        const size_t li = (static_cast<size_t>(b) * p.Hq + head) * p.Tq + (row_real ? pos : 0);
-        const float Lr = row_real ? p.lse[li] * 1.4426950408889634f : 0.0f;
-        const float Dr = row_real ? p.Dsum[li] : 0.0f;
         const uint32_t col = 32 * u;
+        const float2 cc = make_float2(p.scale_log2, p.scale_log2);
+        // row r of M tile t: position, head, and whether it is a real row
+        auto row_pos = [&](int t) { return DqTile(p, t).t0 + r / p.G; };
+        auto row_real = [&](int t) { return r < p.P * p.G && row_pos(t) < p.Tq; };
+        auto row_index = [&](int t) {   // (b, head, pos) -> index of the row's lse / D
+            const DqTile T(p, t);
+            return (static_cast<size_t>(T.b) * p.Hq + T.kvh * p.G + r % p.G) * p.Tq + row_pos(t);
+        };
+        uint32_t g = 0, qi = 0;
         bool ok = true;
-        for (int j = 0; j < n_kv; ++j) {
-            if (!(ok = __all_sync(0xffffffffu, mbar_wait(&s_full, j & 1, &abort_flag, p.status))))
-                break;
-            tc_fence_after();
-            uint32_t sv[32], dp[32];
-            tmem_ld32(lane_addr + Lay::kColS + col, sv);
-            tmem_ld32(lane_addr + Lay::kColP + col, dp);
-            tmem_wait_ld();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&s_free);        // S and dP may be overwritten
-            const int key0 = tile_of(j) * kDqBN + col;
-            const bool full = block_visible(p.vis, t0, p.P, tile_of(j) * kDqBN, kDqBN) &&
-                              __all_sync(0xffffffffu, row_real || r >= p.P * p.G);
-            // dS = P (dP - D); one pair in four takes 2^x on the FMA pipe (the MUFU
-            // unit is the busiest one here).  Tiles the mask leaves whole skip the
-            // per-element test.
-            uint32_t pk[16];
-            const float2 cc = make_float2(p.scale_log2, p.scale_log2), nl = make_float2(-Lr, -Lr);
-            const float2 nd = make_float2(-Dr, -Dr);
-            auto ds_pair = [&](int e) {
-                const float2 x = fma2(make_float2(__uint_as_float(sv[e]), __uint_as_float(sv[e + 1])),
-                                      cc, nl);
-                const float2 pr = ((e >> 1) & 3) == 3 ? exp2_poly2(x)
-                                                      : make_float2(fast_exp2(x.x), fast_exp2(x.y));
-                return mul2(pr, add2(make_float2(__uint_as_float(dp[e]), __uint_as_float(dp[e + 1])),
-                                     nd));
-            };
-            if (full) {
-#pragma unroll
-                for (int e = 0; e < 32; e += 2) {
-                    const float2 ds = ds_pair(e);
-                    pk[e / 2] = pack_bf16x2(ds.x, ds.y);
-                }
-                // rows past the tile's real ones hold stale operands: exact zeros
-                if (!row_real) {
-#pragma unroll
-                    for (int e = 0; e < 16; ++e) pk[e] = 0u;
-                }
-            } else {
-#pragma unroll
-                for (int e = 0; e < 32; e += 2) {
-                    float2 ds = ds_pair(e);
-                    if (!(row_real && p.vis(pos, key0 + e))) ds.x = 0.0f;
-                    if (!(row_real && p.vis(pos, key0 + e + 1))) ds.y = 0.0f;
-                    pk[e / 2] = pack_bf16x2(ds.x, ds.y);
-                }
-            }
-            // dQ(j-1) has read the dS region
-            if (j > 0 && !(ok = __all_sync(0xffffffffu, mbar_wait(&dq_done, (j - 1) & 1,
-                                                                   &abort_flag, p.status))))
-                break;
-            tc_fence_after();
-            tmem_st16(lane_addr + Lay::kColDS + 16 * u, pk);   // keys 32 u .. 32 u + 31
-            tmem_wait_st();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&p_full);
+        int t = take_tile(0);
+        // lse and D of the row, loaded a tile ahead so that their latency overlaps
+        // the previous tile's epilogue
+        float Lr = 0.0f, Dr = 0.0f;
+        if (t >= 0 && t < p.n_tiles && row_real(t)) {
+            const size_t li = row_index(t);
+            Lr = p.lse[li] * 1.4426950408889634f;
+            Dr = p.Dsum[li];
         }
-        // ---- epilogue: dQ * scale -> bf16 (quarter u writes columns 32 u ..) ----
-        if (ok && n_kv > 0)
-            ok = __all_sync(0xffffffffu, mbar_wait(&acc_done, 0, &abort_flag, p.status));
-        tc_fence_after();
-        const bool have = ok && n_kv > 0;               // warp-uniform
-        __nv_bfloat16 *dst = p.dq + ((static_cast<size_t>(b) * p.Tq + (row_real ? pos : 0)) * p.Hq +
-                                     head) * D + col;
-        if (col < D) {                                  // warp-uniform
-            uint32_t v[32];
-            if (have) {
-                tmem_ld32(lane_addr + Lay::kColDQ + col, v);
-                tmem_wait_ld();
-            } else {
+        for (int it = 0; ok && t >= 0 && t < p.n_tiles; ++it) {
+            bool have = false;                          // warp-uniform
+            {
+                const DqTile T(p, t);
+                const int pos = T.t0 + r / p.G;
+                const bool real = r < p.P * p.G && pos < p.Tq;
+                const float2 nl = make_float2(-Lr, -Lr), nd = make_float2(-Dr, -Dr);
+                have = T.n_kv > 0;
+                for (int j = 0; j < T.n_kv; ++j, ++g) {
+                    if (!(ok = __all_sync(0xffffffffu, wait(&s_full, g & 1)))) break;
+                    tc_fence_after();
+                    uint32_t sv[32], dp[32];
+                    tmem_ld32(lane_addr + Lay::kColS + col, sv);
+                    tmem_ld32(lane_addr + Lay::kColP + col, dp);
+                    tmem_wait_ld();
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&s_free);        // S and dP may be overwritten
+                    const int key0 = T.tile_of(j) * kDqBN + col;
+                    const bool full = block_visible(p.vis, T.t0, p.P, T.tile_of(j) * kDqBN, kDqBN) &&
+                                      __all_sync(0xffffffffu, real || r >= p.P * p.G);
+                    // dS = P (dP - D); one pair in four takes 2^x on the FMA pipe (the
+                    // MUFU unit is the busiest one here).  Tiles the mask leaves whole
+                    // skip the per-element test.
+                    uint32_t pk[16];
+                    auto ds_pair = [&](int e) {
+                        const float2 x = fma2(make_float2(__uint_as_float(sv[e]), __uint_as_float(sv[e + 1])),
+                                              cc, nl);
+                        const float2 pr = ((e >> 1) & 3) == 3 ? exp2_poly2(x)
+                                                              : make_float2(fast_exp2(x.x), fast_exp2(x.y));
+                        return mul2(pr, add2(make_float2(__uint_as_float(dp[e]), __uint_as_float(dp[e + 1])),
+                                             nd));
+                    };
+                    if (full) {
 #pragma unroll
-                for (int e = 0; e < 32; ++e) v[e] = 0u;
-            }
-            if (row_real) {
-                uint4 *d4 = reinterpret_cast<uint4 *>(dst);
-                const float f = p.scale;
+                        for (int e = 0; e < 32; e += 2) {
+                            const float2 ds = ds_pair(e);
+                            pk[e / 2] = pack_bf16x2(ds.x, ds.y);
+                        }
+                        // rows past the tile's real ones hold stale operands: exact zeros
+                        if (!real) {
 #pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const uint32_t *w = &v[8 * e];
-                    d4[e] = make_uint4(
-                        pack_bf16x2(__uint_as_float(w[0]) * f, __uint_as_float(w[1]) * f),
-                        pack_bf16x2(__uint_as_float(w[2]) * f, __uint_as_float(w[3]) * f),
-                        pack_bf16x2(__uint_as_float(w[4]) * f, __uint_as_float(w[5]) * f),
-                        pack_bf16x2(__uint_as_float(w[6]) * f, __uint_as_float(w[7]) * f));
+                            for (int e = 0; e < 16; ++e) pk[e] = 0u;
+                        }
+                    } else {
+#pragma unroll
+                        for (int e = 0; e < 32; e += 2) {
+                            float2 ds = ds_pair(e);
+                            if (!(real && p.vis(pos, key0 + e))) ds.x = 0.0f;
+                            if (!(real && p.vis(pos, key0 + e + 1))) ds.y = 0.0f;
+                            pk[e / 2] = pack_bf16x2(ds.x, ds.y);
+                        }
+                    }
+                    // the previous dQ product has read the dS region
+                    if (g > 0 && !(ok = __all_sync(0xffffffffu, wait(&dq_done, (g - 1) & 1)))) break;
+                    tc_fence_after();
+                    tmem_st16(lane_addr + Lay::kColDS + 16 * u, pk);   // keys 32 u .. 32 u + 31
+                    tmem_wait_st();
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&p_full);
                 }
             }
+            if (!ok) break;
+            // the next tile's index and row statistics, loaded before this tile's
+            // epilogue so that their latency overlaps it
+            const int t_next = take_tile(it + 1);
+            if (t_next >= 0 && t_next < p.n_tiles && row_real(t_next)) {
+                const size_t li = row_index(t_next);
+                Lr = p.lse[li] * 1.4426950408889634f;
+                Dr = p.Dsum[li];
+            }
+            // ---- epilogue: dQ * scale -> bf16 (quarter u writes columns 32 u ..) ----
+            // read 16 columns at a time and pack them at once, to keep few
+            // registers live across the tile loop
+            uint32_t pk[16];
+#pragma unroll
+            for (int e = 0; e < 16; ++e) pk[e] = 0u;
+            if (have) {
+                if (!(ok = __all_sync(0xffffffffu, wait(&acc_done, qi & 1)))) break;
+                tc_fence_after();
+                if (col < D) {                          // warp-uniform
+                    const float f = p.scale;
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        uint32_t v[16];
+                        tmem_ld16(lane_addr + Lay::kColDQ + col + 16 * h, v);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int e = 0; e < 8; ++e)
+                            pk[8 * h + e] = pack_bf16x2(__uint_as_float(v[2 * e]) * f,
+                                                        __uint_as_float(v[2 * e + 1]) * f);
+                    }
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&dq_free);   // the next tile's dQ may start
+                ++qi;
+            }
+            if (col < D && row_real(t)) {
+                const DqTile T(p, t);
+                uint4 *d4 = reinterpret_cast<uint4 *>(
+                    p.dq + ((static_cast<size_t>(T.b) * p.Tq + row_pos(t)) * p.Hq + T.kvh * p.G +
+                            r % p.G) * D + col);
+#pragma unroll
+                for (int e = 0; e < 4; ++e)
+                    d4[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
+            }
+            t = t_next;
         }
     }
 
@@ -908,8 +1033,9 @@ dq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
 
 template <int D>
 static int launch_dq_tc(const void *q, const void *k, const void *v, const void *dout,
-                        const float *lse, const float *Dsum, void *dq, int B, int Tq, int Tkv,
-                        int Hq, int Hkv, Vis vis, float scale, cudaStream_t stream) {
+                        const float *lse, const float *Dsum, unsigned int *tile_counter, void *dq,
+                        int B, int Tq, int Tkv, int Hq, int Hkv, Vis vis, float scale,
+                        cudaStream_t stream) {
     DqParams prm;
     prm.B = B;
     prm.Tq = Tq;
@@ -925,10 +1051,16 @@ static int launch_dq_tc(const void *q, const void *k, const void *v, const void 
     prm.lse = lse;
     prm.Dsum = Dsum;
     prm.dq = static_cast<__nv_bfloat16 *>(dq);
+    prm.tile_counter = tile_counter;
     prm.status = device_status_ptr();
     if (!prm.status) return GQA_ERR_CUDA;
-    const long long blocks = static_cast<long long>(prm.n_mt) * Hkv * B;
-    if (blocks > 0x7fffffffLL) return set_error(GQA_ERR_UNSUPPORTED, "backward grid too large");
+    const long long tiles = static_cast<long long>(prm.n_mt) * Hkv * B;
+    if (tiles > 0x7fffffffLL) return set_error(GQA_ERR_UNSUPPORTED, "backward grid too large");
+    prm.n_tiles = static_cast<int>(tiles);
+    if (tiles == 0) return GQA_OK;
+    int n_sm = 0;
+    if (int rc = sm_count(&n_sm)) return rc;
+    const int blocks = static_cast<int>(tiles < n_sm ? tiles : n_sm);
     CUtensorMap tq, to, tk, tv;
     if (int rc = encode_tmap_bf16_4d(&tq, q, D, Hq, Tq, B, 64, prm.G, prm.P, 1, 1)) return rc;
     if (int rc = encode_tmap_bf16_4d(&to, dout, D, Hq, Tq, B, 64, prm.G, prm.P, 1, 1)) return rc;
@@ -946,9 +1078,13 @@ static int launch_dq_tc(const void *q, const void *k, const void *v, const void 
     return check_cuda(cudaGetLastError(), "dq_tc_kernel launch");
 }
 
-size_t bwd_workspace_bytes(int B, int Tq, int Hq) {
+// D (one float per query row, rounded up to 256 bytes), then the dQ kernel's
+// tile counter (256 bytes).
+static size_t bwd_dsum_bytes(int B, int Tq, int Hq) {
     return ((static_cast<size_t>(B) * Tq * Hq * sizeof(float)) + 255) & ~static_cast<size_t>(255);
 }
+
+size_t bwd_workspace_bytes(int B, int Tq, int Hq) { return bwd_dsum_bytes(B, Tq, Hq) + 256; }
 
 namespace {
 
@@ -1004,13 +1140,16 @@ static int launch_bwd_d(const void *q, const void *k, const void *v, const void 
                         float scale, void *workspace, cudaStream_t stream) {
     using bf = __nv_bfloat16;
     float *Dsum = static_cast<float *>(workspace);
+    auto *tile_counter = reinterpret_cast<unsigned int *>(static_cast<uint8_t *>(workspace) +
+                                                          bwd_dsum_bytes(B, Tq, Hq));
     const long long rows = static_cast<long long>(B) * Tq * Hq;
     const long long threads = (rows + kRowdotRows - 1) / kRowdotRows * (D / 8);
     if ((threads + 255) / 256 > 0x7fffffffLL)
         return set_error(GQA_ERR_UNSUPPORTED, "backward: too many rows");
     if (rows > 0)
         rowdot_kernel<D><<<static_cast<unsigned>((threads + 255) / 256), 256, 0, stream>>>(
-            static_cast<const bf *>(dout), static_cast<const bf *>(o), Dsum, B, Tq, Hq);
+            static_cast<const bf *>(dout), static_cast<const bf *>(o), Dsum, tile_counter, B, Tq,
+            Hq);
     if (int rc = check_cuda(cudaGetLastError(), "rowdot_kernel launch")) return rc;
     Vis vis{Tq, Tkv, causal, causal ? window : 0, sinks};
     if (Tkv == 0)   // no key: every query gradient is zero
@@ -1026,7 +1165,8 @@ static int launch_bwd_d(const void *q, const void *k, const void *v, const void 
     int rc = launch_dkdv_tc<D>(q, k, v, dout, lse, Dsum, dk, dv, B, Tq, Tkv, Hq, Hkv, vis, scale,
                                r->s);
     if (rc == GQA_OK)
-        rc = launch_dq_tc<D>(q, k, v, dout, lse, Dsum, dq, B, Tq, Tkv, Hq, Hkv, vis, scale, stream);
+        rc = launch_dq_tc<D>(q, k, v, dout, lse, Dsum, tile_counter, dq, B, Tq, Tkv, Hq, Hkv, vis,
+                             scale, stream);
     // join, on every path: the caller's stream (and a capture in progress on
     // it) then covers all the side stream's work
     const int rj = check_cuda(cudaEventRecord(r->join, r->s), "cudaEventRecord(join)");

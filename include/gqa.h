@@ -248,7 +248,8 @@ int gqa_decode_static(const void *q, const void *k_cache, const void *v_cache,
 /*
  * gqa_attn_bwd_workspace_size -- bytes of device scratch gqa_attn_bwd needs
  * (one fp32 row statistic per query row: B * Hq * Tq floats, rounded up to
- * 256).  0 for invalid sizes.  Pure host function.
+ * 256, then 256 bytes for the dQ kernel's work counter).  0 for invalid
+ * sizes.  Pure host function.
  */
 size_t gqa_attn_bwd_workspace_size(int B, int Tq, int Hq);
 

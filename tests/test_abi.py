@@ -203,7 +203,9 @@ def test_backward_rejects(gqa_lib):
     assert bwd(ws=NULL) == b.GQA_ERR_WORKSPACE
     assert bwd(ws_bytes=16) == b.GQA_ERR_WORKSPACE
     assert bwd(B=0) == b.GQA_OK
-    assert b.gqa_attn_bwd_workspace_size(2, 100, 8) >= 2 * 100 * 8 * 4
+    # D per query row rounded up to 256 bytes, then 256 bytes for the dQ work counter
+    assert b.gqa_attn_bwd_workspace_size(2, 100, 8) == (2 * 100 * 8 * 4 + 255) // 256 * 256 + 256
+    assert b.gqa_attn_bwd_workspace_size(1, 64, 4) == 1024 + 256
 
 
 def test_fused_rope_entry_points_reject(gqa_lib):
