@@ -146,3 +146,33 @@ def test_backward_graph_capture_and_streams(gqa_lib):
     gqa.device_status()
     for a, b in zip(again, want[1]):
         assert torch.equal(a, b)
+
+
+@pytest.mark.parametrize("B,T,Hq,Hkv,d", [
+    (3, 1000, 16, 2, 128),    # G = 8: 16 positions per M tile, 378 tiles (> SMs)
+    (1, 64, 4, 4, 64),        # one M tile: one CTA takes it, the others find the queue empty
+])
+def test_backward_dq_tile_queue(gqa_lib, B, T, Hq, Hkv, d):
+    # The dQ kernel takes its M tiles from a counter in the workspace that the
+    # rowdot launch resets: a workspace full of stale bytes, and a second call
+    # on the same workspace, give the same gradients as the oracle.
+    q, k, v = workloads.prefill_inputs(B, T, Hq, Hkv, d, seeds=(B + 3, T, Hq))
+    dout = workloads.randn((B, T, Hq, d), 91)
+    qc, kc, vc = q.cuda(), k.cuda(), v.cuda()
+    o, lse = gqa.attn(qc, kc, vc, causal=True, return_lse=True)
+    ws = torch.full((gqa.attn_bwd_workspace_size(B, T, Hq),), 0xFF, dtype=torch.uint8,
+                    device="cuda")
+    first = gqa.attn_bwd(qc, kc, vc, o, lse, dout.cuda(), workspace=ws)
+    second = gqa.attn_bwd(qc, kc, vc, o, lse, dout.cuda(), workspace=ws)
+    torch.cuda.synchronize()
+    gqa.device_status()
+    for a, b in zip(first, second):
+        assert torch.equal(a, b)
+    if B * T <= 1000:
+        rq, rk, rv = ref.attn_bwd(q, k, v, dout, True)
+    else:   # batch 0 only (batches are independent problems)
+        rq, rk, rv = ref.attn_bwd(q[:1], k[:1], v[:1], dout[:1], True)
+        first = tuple(t[:1] for t in first)
+    assert rel_err(first[0], rq) <= 2e-2
+    assert rel_err(first[1], rk) <= 2e-2
+    assert rel_err(first[2], rv) <= 2e-2
