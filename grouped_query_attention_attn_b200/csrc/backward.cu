@@ -723,8 +723,8 @@ dq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
     auto wait = [&](uint64_t *bar, uint32_t parity) {
         return mbar_wait(bar, parity, &abort_flag, p.status);
     };
-    // Tile number of iteration `it` (>= p.n_tiles: no more tiles), read by a
-    // consuming warp; lane 0 releases the slot.  -1 after an abort.
+    // Tile number of iteration `it` (>= p.n_tiles: no more tiles), read by an
+    // elementwise warp; lane 0 releases the slot.  -1 after an abort.
     auto take_tile = [&](int it) {
         const int slot = it & 1;
         if (!__all_sync(0xffffffffu, wait(&t_full[slot], (it >> 1) & 1))) return -1;
@@ -734,56 +734,43 @@ dq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
         return t;
     };
 
-    if (warp == 0) {
+    if (warp == 0 && lane == 0) {
         // -------------------------- scheduler, Q / dO and K ring producer ----
-        const bool leader = elect_one();
-        const int leader_lane = __ffs(__ballot_sync(0xffffffffu, leader)) - 1;
-        if (leader) {
-            tma_prefetch_desc(&tm_q);
-            tma_prefetch_desc(&tm_o);
-            tma_prefetch_desc(&tm_k);
-        }
+        // Both producers and both MMA issuers of this kernel run as one thread
+        // (measured faster here than the warp-wide form the dK/dV kernel uses).
+        tma_prefetch_desc(&tm_q);
+        tma_prefetch_desc(&tm_o);
+        tma_prefetch_desc(&tm_k);
         uint32_t kc = 0, qi = 0;   // K copies and Q / dO copies issued
         bool ok = true;
         for (int it = 0; ok; ++it) {
             const int slot = it & 1;
-            if (it >= 2 && !(ok = __all_sync(0xffffffffu, wait(&t_empty[slot], ((it >> 1) & 1) ^ 1))))
-                break;
-            int t = 0;
-            if (leader) {
-                t = static_cast<int>(atomicAdd(p.tile_counter, 1u));
-                if (t > p.n_tiles) t = p.n_tiles;
-                t_slot[slot] = t;
-                mbar_arrive(&t_full[slot]);     // release: the index store comes first
-            }
-            t = __shfl_sync(0xffffffffu, t, leader_lane);
+            if (it >= 2 && !(ok = wait(&t_empty[slot], ((it >> 1) & 1) ^ 1))) break;
+            int t = static_cast<int>(atomicAdd(p.tile_counter, 1u));
+            if (t > p.n_tiles) t = p.n_tiles;
+            t_slot[slot] = t;
+            mbar_arrive(&t_full[slot]);         // release: the index store comes first
             if (t >= p.n_tiles) break;
             const DqTile T(p, t);
             if (T.n_kv == 0) continue;
             // Q and dO of the previous tile are free once its last S / dP ran
-            if (qi > 0 && !(ok = __all_sync(0xffffffffu, wait(&qo_empty, (qi - 1) & 1)))) break;
-            if (leader) {
-                const uint32_t box = 64u * p.G * p.P * 2u;
-                mbar_expect_tx(&qo_full, 2 * Lay::kPanels * box);
-                for (int pn = 0; pn < Lay::kPanels; ++pn) {
-                    tma_load_4d(smem + Lay::kOffQ + pn * Lay::kPanel, &tm_q, &qo_full, pn * 64,
-                                T.kvh * p.G, T.t0, T.b);
-                    tma_load_4d(smem + Lay::kOffO + pn * Lay::kPanel, &tm_o, &qo_full, pn * 64,
-                                T.kvh * p.G, T.t0, T.b);
-                }
+            if (qi > 0 && !(ok = wait(&qo_empty, (qi - 1) & 1))) break;
+            const uint32_t box = 64u * p.G * p.P * 2u;
+            mbar_expect_tx(&qo_full, 2 * Lay::kPanels * box);
+            for (int pn = 0; pn < Lay::kPanels; ++pn) {
+                tma_load_4d(smem + Lay::kOffQ + pn * Lay::kPanel, &tm_q, &qo_full, pn * 64,
+                            T.kvh * p.G, T.t0, T.b);
+                tma_load_4d(smem + Lay::kOffO + pn * Lay::kPanel, &tm_o, &qo_full, pn * 64,
+                            T.kvh * p.G, T.t0, T.b);
             }
-            __syncwarp();
             ++qi;
             for (int j = 0; j < T.n_kv; ++j, ++kc) {
                 const uint32_t st = kc % kDqKStages, ph = (kc / kDqKStages) & 1;
-                if (!(ok = __all_sync(0xffffffffu, wait(&k_empty[st], ph ^ 1)))) break;
-                if (leader) {
-                    mbar_expect_tx(&k_full[st], Lay::kTile);
-                    for (int pn = 0; pn < Lay::kPanels; ++pn)
-                        tma_load_4d(smem + Lay::kOffK + st * Lay::kTile + pn * Lay::kPanel, &tm_k,
-                                    &k_full[st], pn * 64, T.kvh, T.tile_of(j) * kDqBN, T.b);
-                }
-                __syncwarp();
+                if (!(ok = wait(&k_empty[st], ph ^ 1))) break;
+                mbar_expect_tx(&k_full[st], Lay::kTile);
+                for (int pn = 0; pn < Lay::kPanels; ++pn)
+                    tma_load_4d(smem + Lay::kOffK + st * Lay::kTile + pn * Lay::kPanel, &tm_k,
+                                &k_full[st], pn * 64, T.kvh, T.tile_of(j) * kDqBN, T.b);
             }
         }
         // copies still in flight land before the block exits
@@ -791,26 +778,25 @@ dq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
         for (uint32_t c = kc > kDqKStages ? kc - kDqKStages : 0; c < kc; ++c)
             mbar_wait(&k_full[c % kDqKStages], (c / kDqKStages) & 1, &abort_flag, p.status,
                       1000000ull);
-    } else if (warp == 2) {
+    } else if (warp == 2 && lane == 0) {
         // ------------------------------------------------ V ring producer ----
-        const bool leader = elect_one();
-        if (leader) tma_prefetch_desc(&tm_v);
+        tma_prefetch_desc(&tm_v);
         uint32_t vc = 0;
         bool ok = true;
         for (int it = 0; ok; ++it) {
-            const int t = take_tile(it);
-            if (t < 0 || t >= p.n_tiles) break;
+            const int slot = it & 1;
+            if (!(ok = wait(&t_full[slot], (it >> 1) & 1))) break;
+            const int t = *reinterpret_cast<volatile int *>(&t_slot[slot]);
+            mbar_arrive(&t_empty[slot]);
+            if (t >= p.n_tiles) break;
             const DqTile T(p, t);
             for (int j = 0; j < T.n_kv; ++j, ++vc) {
                 const uint32_t st = vc % kDqVStages, ph = (vc / kDqVStages) & 1;
-                if (!(ok = __all_sync(0xffffffffu, wait(&v_empty[st], ph ^ 1)))) break;
-                if (leader) {
-                    mbar_expect_tx(&v_full[st], Lay::kTile);
-                    for (int pn = 0; pn < Lay::kPanels; ++pn)
-                        tma_load_4d(smem + Lay::kOffV + st * Lay::kTile + pn * Lay::kPanel, &tm_v,
-                                    &v_full[st], pn * 64, T.kvh, T.tile_of(j) * kDqBN, T.b);
-                }
-                __syncwarp();
+                if (!(ok = wait(&v_empty[st], ph ^ 1))) break;
+                mbar_expect_tx(&v_full[st], Lay::kTile);
+                for (int pn = 0; pn < Lay::kPanels; ++pn)
+                    tma_load_4d(smem + Lay::kOffV + st * Lay::kTile + pn * Lay::kPanel, &tm_v,
+                                &v_full[st], pn * 64, T.kvh, T.tile_of(j) * kDqBN, T.b);
             }
         }
         for (uint32_t c = vc > kDqVStages ? vc - kDqVStages : 0; c < vc; ++c)
