@@ -312,10 +312,11 @@ dkdv_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         }
     } else if (warp == 1) {
         // ------------------------------------------------- MMA issuer ----
-        // The whole warp follows the schedule and waits on every barrier; one
-        // elected lane issues the products and commits.  A lone thread running
-        // the same schedule (the other lanes parked at the warp's end) made the
-        // backward 11 % slower on a B200.
+        // The whole warp follows the schedule and waits on every barrier (the
+        // vote in each wait re-converges it); one elected lane issues the
+        // products and commits.  A lone thread running the same schedule (the
+        // other lanes parked at the warp's end) made the backward 11 % slower on
+        // a B200.
         if (n_items > 0) {
             const bool leader = elect_one();
             constexpr uint32_t idesc_s = umma_idesc_bf16(kTcBK, kTcBQ, 0, 0);
@@ -338,7 +339,6 @@ dkdv_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                     }
                     tc_commit(bar);
                 }
-                __syncwarp();
             };
             // dV += P^T dO, dK += dS^T Q: A from tensor memory (quarter u of the
             // queries at columns 32 u .. 32 u + 15, 8 per 16 queries), B MN-major
@@ -353,7 +353,6 @@ dkdv_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                                 (!first || kk > 0) ? 1u : 0u);
                     }
                 }
-                __syncwarp();
             };
             auto q_off = [](int it) { return Lay::kOffQ + (it % kTcQStages) * Lay::kTile; };
             auto o_off = [](int it) { return Lay::kOffO + (it % kTcOStages) * Lay::kTile; };
@@ -372,7 +371,6 @@ dkdv_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                 tc_fence_after();
                 issue_acc(it == 0, Lay::kColDV, Lay::kColS, o_off(it));
                 if (leader) tc_commit(&o_empty[it % kTcOStages]);
-                __syncwarp();
                 if (more) {
                     const int n = it + 1;
                     if (!(ok = wait(&q_full[n % kTcQStages], (n / kTcQStages) & 1))) break;
@@ -383,7 +381,6 @@ dkdv_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                 tc_fence_after();
                 issue_acc(it == 0, Lay::kColDK, Lay::kColP, q_off(it));
                 if (leader) tc_commit(&q_empty[it % kTcQStages]);
-                __syncwarp();
                 if (more) {
                     const int n = it + 1;
                     if (!(ok = wait(&o_full[n % kTcOStages], (n / kTcOStages) & 1))) break;
