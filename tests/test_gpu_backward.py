@@ -176,3 +176,43 @@ def test_backward_dq_tile_queue(gqa_lib, B, T, Hq, Hkv, d):
     assert rel_err(first[0], rq) <= 2e-2
     assert rel_err(first[1], rk) <= 2e-2
     assert rel_err(first[2], rv) <= 2e-2
+
+
+def test_backward_from_two_host_threads(gqa_lib):
+    # The fork / join events and the second stream are shared per context and
+    # used under a lock: two host threads calling the backward at once, each on
+    # its own stream with its own workspace, get exactly the eager results.
+    import threading
+    B, T, Hq, Hkv, d = 1, 512, 8, 2, 128
+    q, k, v = workloads.prefill_inputs(B, T, Hq, Hkv, d, seeds=(21, 22, 23))
+    qc, kc, vc = q.cuda(), k.cuda(), v.cuda()
+    o, lse = gqa.attn(qc, kc, vc, causal=True, return_lse=True)
+    douts = [workloads.randn((B, T, Hq, d), 60 + i).cuda() for i in range(2)]
+    want = [gqa.attn_bwd(qc, kc, vc, o, lse, dd) for dd in douts]
+    torch.cuda.synchronize()
+    got = [None, None]
+    errors = []
+
+    def run(i):
+        try:
+            s = torch.cuda.Stream()
+            ws = torch.empty(gqa.attn_bwd_workspace_size(B, T, Hq), dtype=torch.uint8,
+                             device="cuda")
+            with torch.cuda.stream(s):
+                for _ in range(20):
+                    got[i] = gqa.attn_bwd(qc, kc, vc, o, lse, douts[i], workspace=ws)
+            s.synchronize()
+        except Exception as e:   # surfaced below
+            errors.append(e)
+
+    threads = [threading.Thread(target=run, args=(i,)) for i in range(2)]
+    for t in threads:
+        t.start()
+    for t in threads:
+        t.join(timeout=120)
+    assert not errors, errors
+    torch.cuda.synchronize()
+    gqa.device_status()
+    for i in range(2):
+        for a, b in zip(got[i], want[i]):
+            assert torch.equal(a, b), i
