@@ -267,8 +267,12 @@ size_t gqa_attn_bwd_workspace_size(int B, int Tq, int Hq);
  * backward is a sum, not a mean); dq carries the chain-rule factor `scale`
  * (same notes, "scale 的处理").  P is recomputed from lse; fp32 accumulation.
  * workspace: >= gqa_attn_bwd_workspace_size(B, Tq, Hq) bytes, 256-byte
- * aligned, contents on entry irrelevant.  d in {64, 128}.  Errors as the
- * forward plus GQA_ERR_WORKSPACE.
+ * aligned, contents on entry irrelevant; it holds D and the dQ kernel's work
+ * counter until the call's kernels finish, so calls in flight at the same time
+ * need workspaces of their own.  The dK/dV kernel runs on a second stream of
+ * the library's, forked from `stream` after D is formed and joined back before
+ * the call's work on `stream` ends (CUDA-graph capture on `stream` holds both).
+ * d in {64, 128}.  Errors as the forward plus GQA_ERR_WORKSPACE.
  */
 int gqa_attn_bwd(const void *q, const void *k, const void *v, const void *o, const void *dout,
                  const float *lse, void *dq, void *dk, void *dv,
