@@ -15,9 +15,9 @@
 //   dq      tcgen05: one CTA per 128-row M tile (the group's heads packed by
 //           position, as in the forward), looping over the visible keys
 // dkdv and dq read the same inputs and write disjoint outputs, so after
-// rowdot they run side by side: dkdv on a second stream of the highest
-// priority (its blocks are dispatched first, its longest CTAs start at once),
-// dq on the caller's stream filling the SMs that dkdv's tail leaves idle.
+// rowdot they run side by side: dkdv on a second stream, enqueued first so
+// that its blocks (the longest first) are dispatched first, and dq on the
+// caller's stream, its persistent CTAs taking the SMs that dkdv's tail frees.
 #include <cuda_bf16.h>
 #include <climits>
 #include <mutex>
