@@ -272,6 +272,9 @@ size_t gqa_attn_bwd_workspace_size(int B, int Tq, int Hq);
  * need workspaces of their own.  The dK/dV kernel runs on a second stream of
  * the library's, forked from `stream` after D is formed and joined back before
  * the call's work on `stream` ends (CUDA-graph capture on `stream` holds both).
+ * The first call in a CUDA context creates that stream and two events, so make
+ * one call before capturing (stream and event creation may be refused during a
+ * global-mode capture; the call then returns GQA_ERR_CUDA).
  * d in {64, 128}.  Errors as the forward plus GQA_ERR_WORKSPACE.
  */
 int gqa_attn_bwd(const void *q, const void *k, const void *v, const void *o, const void *dout,
