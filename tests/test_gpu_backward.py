@@ -31,6 +31,9 @@ def rel_err(gpu, want):
     (1, 260, 100, 4, 2, 128, True, 0, 0),       # Tq > Tkv: rows with no key
     (1, 300, 300, 8, 2, 128, True, 64, 3),      # sliding window with sinks
     (1, 96, 96, 32, 1, 128, True, 0, 0),        # MQA
+    (2, 333, 333, 16, 2, 64, True, 100, 2),     # d = 64, G = 8, window + sinks, ragged
+    (1, 513, 700, 12, 4, 128, True, 0, 0),      # G = 3: 126 real rows per M tile, Tq < Tkv
+    (3, 64, 64, 4, 1, 64, False, 0, 0),         # B = 3, one M tile each, non-causal
 ])
 def test_backward_matches_oracle(gqa_lib, B, Tq, Tkv, Hq, Hkv, d, causal, window, sinks):
     q, k, v = workloads.prefill_inputs(B, Tq, Hq, Hkv, d, Tkv=Tkv, seeds=(Tq, Tkv + 1, Hq + d))
